@@ -1,0 +1,467 @@
+#!/usr/bin/env python3
+"""Benchmark of the CSA/HCA hybrid-attention hot path: CSA decode at 1M context.
+
+Workload (N=1): 8 sequences x 1048576 raw tokens -> 262144 compressed CSA entries each,
+128 query heads over one KV head (d = 128), lightning indexer with 16 heads x 64 dims in
+MXFP4, BF16 index scores, top-1024, 128-token raw window, KV rows in E4M3 (non-RoPE dims,
+per-row scale) + BF16 (RoPE dims).  One step = one decode query per sequence through the
+whole path: quantise q_I -> index scores -> top-k -> sparse attention (+ split merge).
+
+Data-parallel over sequences: with N GPUs every rank runs its own 8 sequences (weak
+scaling, no data-path collective); the timing is the max over ranks.
+
+Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle instead.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA/HCA decode queries/s at 1M ctx; achieved HBM GB/s and % of roofline"
+UNIT = "queries/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload():
+    from synth.configs import CSA_1M
+    return CSA_1M
+
+
+def bytes_per_query(cfg):
+    """Algorithmic HBM bytes of one decode query (the whole step, per sequence)."""
+    kI = cfg.Nc * (cfg.dI // 2 + cfg.dI // 32)           # MXFP4 index keys: 34 B / entry
+    rows = (cfg.k + cfg.W) * (cfg.d // 2 + 4 + cfg.d)     # gathered split rows: 196 B / row
+    qo = 2 * cfg.H * cfg.d * 2 + cfg.HI * cfg.dI * 2 + cfg.HI * 4 + 4   # q in, o out, q_I, w
+    return kI + rows + qo
+
+
+def indexer_bytes_per_launch(cfg, B):
+    """Algorithmic bytes of one indexer launch: MXFP4 keys read + bf16 scores written."""
+    return B * cfg.Nc * (cfg.dI // 2 + cfg.dI // 32 + 2)
+
+
+# ------------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sms, maxs, util_sms, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm, smax, util = float(parts[1]), float(parts[2]), float(parts[4])
+            except ValueError:
+                continue
+            sms.append(sm)
+            maxs.append(smax)
+            if util >= 50:
+                util_sms.append(sm)
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        src = util_sms or sms
+        return {"sm_mhz": statistics.median(src) if src else None,
+                "sm_max_mhz": max(maxs) if maxs else None,
+                "reasons": sorted(reasons), "samples": len(self.lines),
+                "samples_under_load": len(util_sms)}
+
+
+# ------------------------------------------------------------------------------------------
+# CPU oracle timing (the baseline / reference arm)
+
+def oracle_query_sample(cfg, seed_b, n_keys):
+    """Inputs of one decode query restricted to the first n_keys compressed entries, as the
+    oracle consumes them (quantised by the oracle)."""
+    import numpy as np
+    import oracle
+    from synth import gen
+    from synth.configs import scaled
+    c = scaled(cfg, B=1)
+    kI = gen.index_keys(scaled(cfg, L=4 * n_keys), [seed_b])
+    kp, ks = oracle.quant_mxfp4(kI)
+    kvc = gen.comp_kv(cfg, [seed_b], n_keys)
+    cn, cs, cr = oracle.quant_kv_fp8(kvc)
+    raw = gen.raw_kv(cfg, [seed_b], cfg.L - cfg.W, cfg.L)
+    rn, rs, rr = oracle.quant_kv_fp8(raw)
+    q, qI, w = gen.queries(c, [seed_b]), gen.index_queries(c, [seed_b]), gen.head_weights(c, [seed_b])
+    pos = np.full((1, 1), 4 * n_keys - 1, np.int32)      # every sampled entry visible
+    return dict(kp=kp, ks=ks, cn=cn, cs=cs, cr=cr, rn=rn, rs=rs, rr=rr, q=q, qI=qI, w=w, pos=pos,
+                n_keys=n_keys)
+
+
+def oracle_step(cfg, s):
+    import oracle
+    qp, qs = oracle.quant_mxfp4(s["qI"])
+    sc = oracle.index_scores(oracle.FMT_MXFP4, qp, s["w"], s["kp"], s["pos"], cfg.m, qI_sf=qs,
+                             kI_sf=s["ks"], bf16_scores=True)
+    idx = oracle.topk(sc, s["pos"], cfg.m, cfg.k)
+    okc = oracle.KV(oracle.FMT_FP8SPLIT, s["cn"], s["n_keys"], scale=s["cs"], rope=s["cr"])
+    # window rows are stored as a ring of W slots holding tokens L-W .. L-1; with the sampled
+    # query position 4*n_keys-1 the window reads the ring's slots through the same t mod W map
+    okr = oracle.KV(oracle.FMT_FP8SPLIT, s["rn"], cfg.W, scale=s["rs"], rope=s["rr"])
+    return oracle.csa_attn(s["q"], okc, idx, okr, cfg.W, s["pos"])
+
+
+def time_oracle(cfg, seconds, min_steps=1, frac=1.0):
+    """Run oracle decode queries (each over frac of the entries) for about `seconds`."""
+    n_keys = max(cfg.k + 1, int(cfg.Nc * frac))
+    s = oracle_query_sample(cfg, 0, n_keys)
+    oracle_step(cfg, s)                                   # warm (thread pool, pages)
+    t0 = time.perf_counter()
+    n = 0
+    while n < min_steps or time.perf_counter() - t0 < seconds:
+        oracle_step(cfg, s)
+        n += 1
+    dt = time.perf_counter() - t0
+    f = n_keys / cfg.Nc
+    return n, dt, f, n_keys
+
+
+def cpu_threads():
+    v = os.environ.get("OMP_NUM_THREADS")
+    return int(v) if v and v.isdigit() else os.cpu_count()
+
+
+# ------------------------------------------------------------------------------------------
+
+def run_reference(args, rank, world):
+    """The oracle, as it stands, on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    cfg = workload()
+    K, Wm = args.steps, args.warmup
+    # each step is one query over a sample of the entries sized so the run stays ~2 minutes
+    est = 1.5                                          # s per full 1M query (order of magnitude)
+    frac = min(1.0, 90.0 / max(1, (K + Wm)) / est)
+    n_keys = max(cfg.k + 1, int(cfg.Nc * frac))
+    s = oracle_query_sample(cfg, 0, n_keys)
+    for _ in range(Wm):
+        oracle_step(cfg, s)
+    t0 = time.perf_counter()
+    for _ in range(K):
+        oracle_step(cfg, s)
+    dt = time.perf_counter() - t0
+    f = n_keys / cfg.Nc
+    value = K * f / dt
+    sample = (f"each step: one decode query over the first {n_keys} of {cfg.Nc} compressed "
+              f"entries (fraction {f:.4f}), full top-k and attention; queries/s scaled by the fraction")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": K, "warmup": Wm, "ms_per_step": 1e3 * dt / max(K, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "B_per_gpu": cfg.B, "L": cfg.L, "Nc": cfg.Nc,
+                       "H": cfg.H, "HI": cfg.HI, "k": cfg.k, "W": cfg.W},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def build_inputs(cfg, B, rank, n_sets, device):
+    """Device-resident inputs of n_sets independent decode problems (GPU-generated values,
+    quantised by libhcl).  Returns pipelines and the per-step host-side query tensors."""
+    import torch
+    from heavily_compressed_long_b200 import api
+    from heavily_compressed_long_b200.api import HCL_BF16, HCL_MXFP4, KV
+    from heavily_compressed_long_b200.pipeline import CsaDecode
+    Nc, W, L, d, HI, dI = cfg.Nc, cfg.W, cfg.L, cfg.d, cfg.HI, cfg.dI
+    sets = []
+    for s in range(n_sets):
+        g = torch.Generator(device=device)
+        g.manual_seed(cfg.seed + 7919 * rank + 104729 * s)
+        kI_p = torch.empty(B, Nc, dI // 2, dtype=torch.uint8, device=device)
+        kI_s = torch.empty(B, Nc, dI // 32, dtype=torch.uint8, device=device)
+        c_n = torch.empty(B, Nc, d // 2, dtype=torch.uint8, device=device)
+        c_s = torch.empty(B, Nc, dtype=torch.float32, device=device)
+        c_r = torch.empty(B, Nc, d // 2, dtype=torch.bfloat16, device=device)
+        for b in range(B):
+            x = torch.randn(Nc, dI, generator=g, device=device).to(torch.bfloat16)
+            api.hcl_quant_mxfp4(x, kI_p[b], kI_s[b])
+            x = torch.randn(Nc, d, generator=g, device=device).to(torch.bfloat16)
+            api.hcl_quant_kv_fp8(x, c_n[b], c_s[b], c_r[b])
+            del x
+        ring = torch.randn(B, W, d, generator=g, device=device).to(torch.bfloat16)
+        r_n = torch.empty(B, W, d // 2, dtype=torch.uint8, device=device)
+        r_s = torch.empty(B, W, dtype=torch.float32, device=device)
+        r_r = torch.empty(B, W, d // 2, dtype=torch.bfloat16, device=device)
+        api.hcl_quant_kv_fp8(ring, r_n, r_s, r_r)
+        q = torch.randn(B, 1, cfg.H, d, generator=g, device=device).to(torch.bfloat16)
+        qI = torch.randn(B, 1, HI, dI, generator=g, device=device).to(torch.bfloat16)
+        w = torch.rand(B, 1, HI, generator=g, device=device)
+        pos = torch.full((B, 1), L - 1, dtype=torch.int32, device=device)
+        pipe = CsaDecode(q, qI, w, kI_p, KV(c_n, c_s, c_r), Nc, KV(r_n, r_s, r_r), L, W, pos,
+                         m=cfg.m, k=cfg.k, op_fmt=HCL_MXFP4, score_fmt=HCL_BF16, kI_sf=kI_s)
+        sets.append(pipe)
+    return sets
+
+
+def run_hcl(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from heavily_compressed_long_b200 import api
+    from heavily_compressed_long_b200._lib import lib
+    lib()                                               # fail loudly without libhcl.so
+    cfg = workload()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    B = cfg.B
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    per_set = B * cfg.Nc * (cfg.dI // 2 + cfg.dI // 32)
+    n_sets = max(2, -(-4 * l2 // per_set))              # streamed bytes per cycle >= 4 x L2
+    sets = build_inputs(cfg, B, rank, n_sets, device)
+    stream = torch.cuda.Stream(device)
+    torch.cuda.synchronize()
+
+    # eager warm-up (attributes, first-launch costs), then capture one graph per input set
+    with torch.cuda.stream(stream):
+        for p in sets:
+            p.step_parts(stream=stream)
+    torch.cuda.synchronize()
+    graphs = []
+    for p in sets:
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            p.step_parts(stream=stream)
+        graphs.append(gr)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def maxv(x):
+        if world > 1:
+            t = torch.tensor([x], dtype=torch.float64, device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            return float(t.item())
+        return x
+
+    K, Wm = args.steps, args.warmup
+    with torch.cuda.stream(stream):
+        for i in range(Wm):
+            graphs[i % n_sets].replay()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for i in range(K):
+            graphs[i % n_sets].replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    step_ms = maxv(e0.elapsed_time(e1) / K)
+
+    # dominant kernel alone: the indexer, back to back over the rotating sets
+    from heavily_compressed_long_b200.api import HCL_MXFP4
+    with torch.cuda.stream(stream):
+        for p in sets:
+            api.hcl_quant_mxfp4(p.qI, p.qI_packed, p.qI_sf, stream=stream)
+    torch.cuda.synchronize()
+    n_idx = max(50, min(K, 2000))
+
+    def run_indexer(i):
+        p = sets[i % n_sets]
+        api.hcl_csa_index_scores(HCL_MXFP4, p.qI_packed, p.w, p.kI, p.q_pos, p.m, p.scores,
+                                 Nc=p.Nc, qI_sf=p.qI_sf, kI_sf=p.kI_sf, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(2 * n_sets):
+            run_indexer(i)
+    i0, i1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    i0.record(stream)
+    with torch.cuda.stream(stream):
+        for i in range(n_idx):
+            run_indexer(i)
+    i1.record(stream)
+    torch.cuda.synchronize()
+    idx_ms = maxv(i0.elapsed_time(i1) / n_idx)
+
+    # end to end through the C ABI with host buffers: H2D of the step's queries, the fused
+    # decode-step call, D2H of the outputs -- every step
+    hq = [torch.empty_like(p.q, device="cpu").pin_memory() for p in sets]
+    hqi = [torch.empty_like(p.qI, device="cpu").pin_memory() for p in sets]
+    hw = [torch.empty_like(p.w, device="cpu").pin_memory() for p in sets]
+    hpos = [torch.empty_like(p.q_pos, device="cpu").pin_memory() for p in sets]
+    hout = [torch.empty_like(p.out, device="cpu").pin_memory() for p in sets]
+    for j, p in enumerate(sets):
+        hq[j].copy_(p.q)
+        hqi[j].copy_(p.qI)
+        hw[j].copy_(p.w)
+        hpos[j].copy_(p.q_pos)
+    h2d = hq[0].numel() * 2 + hqi[0].numel() * 2 + hw[0].numel() * 4 + hpos[0].numel() * 4
+    d2h = hout[0].numel() * 2
+
+    def e2e_step(i):
+        j = i % n_sets
+        p = sets[j]
+        p.q.copy_(hq[j], non_blocking=True)
+        p.qI.copy_(hqi[j], non_blocking=True)
+        p.w.copy_(hw[j], non_blocking=True)
+        p.q_pos.copy_(hpos[j], non_blocking=True)
+        p.step(stream=stream)
+        hout[j].copy_(p.out, non_blocking=True)
+
+    n_e2e = max(20, min(K, 2000))
+    with torch.cuda.stream(stream):
+        for i in range(max(Wm, n_sets)):
+            e2e_step(i)
+    torch.cuda.synchronize()
+    barrier()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    with torch.cuda.stream(stream):
+        for i in range(n_e2e):
+            e2e_step(i)
+    x1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = maxv(x0.elapsed_time(x1) / n_e2e)
+    clocks = sampler.stop() if sampler else None
+    status = int(sum(int(p.status.item()) for p in sets))
+
+    # CPU baseline: the oracle on the host cores, a bounded sample (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n, dt, f, n_keys = time_oracle(cfg, args.cpu_seconds, frac=args.cpu_frac)
+        cpu = {"value": n * f / dt, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"{n} decode queries, each over the first {n_keys} of {cfg.Nc} entries "
+                         f"(fraction {f:.3f}), full top-k and attention; scaled by the fraction"}
+
+    if rank == 0:
+        hbm, src = peaks()
+        q_per_step = B * world
+        value = q_per_step / (step_ms * 1e-3)
+        bpq = bytes_per_query(cfg)
+        step_gbs = B * bpq / (step_ms * 1e-3) / 1e9
+        idx_bytes = indexer_bytes_per_launch(cfg, B)
+        idx_gbs = idx_bytes / (idx_ms * 1e-3) / 1e9
+        launches = sets[0].launches_per_step()
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": Wm, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "mxfp4+e4m3+bf16 (fp32 accumulate)",
+            "data": "synthetic: seeded N(0,1) on device, MXFP4 / E4M3 quantised by libhcl",
+            "config": {"workload": cfg.name, "B_per_gpu": B, "L": cfg.L, "Nc": cfg.Nc, "H": cfg.H,
+                       "HI": cfg.HI, "dI": cfg.dI, "k": cfg.k, "W": cfg.W,
+                       "parallelism": f"dp{world} (sequences)",
+                       "l2": f"{n_sets} rotating input sets ({n_sets * per_set / 1e6:.0f} MB of index "
+                             f"keys streamed per cycle vs {l2 / 1e6:.0f} MB L2)",
+                       "timing": "CUDA graph per input set, CUDA events, max over ranks"},
+            "step_hbm_gbs": step_gbs,
+            "step_frac_of_hbm": step_gbs / hbm,
+            "bytes_per_query": bpq,
+            "roofline": {"bound": "hbm", "kernel": "indexer (tcgen05 kind::mxf4)",
+                         "achieved": idx_gbs, "peak": hbm, "unit": "GB/s", "frac": idx_gbs / hbm,
+                         "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback 6.65 TB/s",
+                         "bytes_per_launch": idx_bytes, "ms_per_launch": idx_ms,
+                         "share_of_step": idx_ms / step_ms, "traffic": None},
+            "e2e": {"value": q_per_step / (e2e_ms * 1e-3), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                    "path": "hcl_csa_decode_step (C ABI) + pinned H2D/D2H copies, no graph"},
+            "gpu_launches": K * launches,
+            "device_status": status,
+            "clocks": clocks,
+        }
+        if cpu:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    for gr in graphs:
+        del gr
+    graphs.clear()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="hcl", choices=["hcl", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-frac", type=float, default=1.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_hcl(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,167 @@
+"""Python binding of libhcl with the C ABI's names; torch tensors in, argument marshalling only.
+
+Every function takes CUDA tensors (device memory owned by the caller) and enqueues the
+corresponding libhcl call on the current torch stream (or `stream`).  No arithmetic of the
+method happens here.  Formats: HCL_BF16 / HCL_FP32 / HCL_FP8SPLIT / HCL_MXFP4.
+"""
+import ctypes
+import math
+
+import torch
+
+from . import _lib
+from ._lib import (HCL_BF16, HCL_FP32, HCL_FP8SPLIT, HCL_MXFP4, check, hcl_kv_t, lib)
+
+__all__ = ["KV", "hcl_csa_compress", "hcl_hca_compress", "hcl_quant_kv_fp8", "hcl_quant_mxfp4",
+           "hcl_csa_index_scores", "hcl_csa_topk", "hcl_csa_sparse_attn", "hcl_hca_dense_attn",
+           "hcl_csa_decode_step", "hcl_selftest_bounded_wait", "HCL_BF16", "HCL_FP32",
+           "HCL_FP8SPLIT", "HCL_MXFP4"]
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libhcl takes CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("libhcl takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class KV:
+    """A KV store (see hcl_kv_t): bf16 rows [B, cap, d], or split rows: e4m3 codes
+    [B, cap, d/2] (uint8), fp32 scale [B, cap], bf16 RoPE half [B, cap, d/2]."""
+
+    def __init__(self, data, scale=None, rope=None):
+        self.data, self.scale, self.rope = data, scale, rope
+        self.fmt = HCL_FP8SPLIT if scale is not None else HCL_BF16
+        self.cap = data.shape[1]
+        self._c = hcl_kv_t(self.fmt, self.cap, _ptr(data).value, None if scale is None else _ptr(scale).value,
+                           None if rope is None else _ptr(rope).value)
+
+    def ref(self):
+        return ctypes.byref(self._c)
+
+
+def _fmt_of(t):
+    return HCL_FP32 if t.dtype == torch.float32 else HCL_BF16
+
+
+def hcl_csa_compress(kv, gate, bias, m, out, entry_begin=0, entry_end=None, stream=None):
+    B, L, d = kv.shape
+    if entry_end is None:
+        entry_end = -(-L // m)
+    check(lib().hcl_csa_compress(_ptr(kv), _ptr(gate), _ptr(bias), B, L, d, m, entry_begin,
+                                 entry_end, _ptr(out), _fmt_of(out), out.shape[1], _stream(stream)))
+    return out
+
+
+def hcl_hca_compress(kv, gate, bias, m, out, entry_begin=0, entry_end=None, stream=None):
+    B, L, d = kv.shape
+    if entry_end is None:
+        entry_end = -(-L // m)
+    check(lib().hcl_hca_compress(_ptr(kv), _ptr(gate), _ptr(bias), B, L, d, m, entry_begin,
+                                 entry_end, _ptr(out), _fmt_of(out), out.shape[1], _stream(stream)))
+    return out
+
+
+def hcl_quant_kv_fp8(kv, nope, scale, rope, stream=None):
+    d = kv.shape[-1]
+    rows = kv.numel() // d
+    check(lib().hcl_quant_kv_fp8(_ptr(kv), rows, d, _ptr(nope), _ptr(scale), _ptr(rope),
+                                 _stream(stream)))
+
+
+def hcl_quant_mxfp4(x, packed, sf, stream=None):
+    cols = x.shape[-1]
+    rows = x.numel() // cols
+    check(lib().hcl_quant_mxfp4(_ptr(x), rows, cols, _ptr(packed), _ptr(sf), _stream(stream)))
+
+
+def hcl_csa_index_scores(op_fmt, qI, w, kI, q_pos, m, scores, Nc=None, qI_sf=None, kI_sf=None,
+                         status=None, stream=None):
+    B, Tq, HI = w.shape
+    dI = qI.shape[-1] * (2 if op_fmt == HCL_MXFP4 else 1)
+    cap = kI.shape[1]
+    Nc = cap if Nc is None else Nc
+    check(lib().hcl_csa_index_scores(op_fmt, _ptr(qI), _ptr(qI_sf), _ptr(w), _ptr(kI), _ptr(kI_sf),
+                                     B, Tq, HI, dI, Nc, cap, _ptr(q_pos), m, _ptr(scores),
+                                     _fmt_of(scores), _ptr(status), _stream(stream)))
+    return scores
+
+
+def hcl_csa_topk(scores, q_pos, m, k, idx, status=None, stream=None):
+    B, Tq, Nc = scores.shape
+    fmt = _fmt_of(scores)
+    wsb = lib().hcl_csa_topk_workspace_bytes(B, Tq, Nc, k, fmt)
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=scores.device) if wsb else None
+    check(lib().hcl_csa_topk(_ptr(scores), fmt, B, Tq, Nc, _ptr(q_pos), m, k, _ptr(idx), _ptr(ws),
+                             wsb, _ptr(status), _stream(stream)))
+    return idx
+
+
+def csa_sparse_attn_workspace_bytes(B, Tq, H, k, W):
+    return lib().hcl_csa_sparse_attn_workspace_bytes(B, Tq, H, k, W)
+
+
+def hcl_csa_sparse_attn(q, kvc: KV, Nc, idx, raw: KV, L, W, q_pos, out, lse=None, scale=None,
+                        sink=None, ws=None, status=None, stream=None):
+    B, Tq, H, d = q.shape
+    k = idx.shape[-1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    need = csa_sparse_attn_workspace_bytes(B, Tq, H, k, W)
+    if ws is None and need:
+        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    check(lib().hcl_csa_sparse_attn(_ptr(q), B, Tq, H, d, kvc.ref(), Nc, _ptr(idx), k, raw.ref(),
+                                    L, W, _ptr(q_pos), scale, _ptr(sink), _ptr(out), _ptr(lse),
+                                    _ptr(ws), 0 if ws is None else ws.numel(), _ptr(status),
+                                    _stream(stream)))
+    return out
+
+
+def hca_dense_attn_workspace_bytes(B, Tq, H, Nh, W):
+    return lib().hcl_hca_dense_attn_workspace_bytes(B, Tq, H, Nh, W)
+
+
+def hcl_hca_dense_attn(q, kvh: KV, Nh, mh, raw: KV, L, W, q_pos, out, lse=None, scale=None,
+                       sink=None, ws=None, status=None, stream=None):
+    B, Tq, H, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    need = hca_dense_attn_workspace_bytes(B, Tq, H, Nh, W)
+    if ws is None and need:
+        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    check(lib().hcl_hca_dense_attn(_ptr(q), B, Tq, H, d, kvh.ref(), Nh, mh, raw.ref(), L, W,
+                                   _ptr(q_pos), scale, _ptr(sink), _ptr(out), _ptr(lse), _ptr(ws),
+                                   0 if ws is None else ws.numel(), _ptr(status), _stream(stream)))
+    return out
+
+
+def decode_step_workspace_bytes(B, H, HI, Nc, k, W, op_fmt, score_fmt):
+    return lib().hcl_csa_decode_step_workspace_bytes(B, H, HI, Nc, k, W, op_fmt, score_fmt)
+
+
+def hcl_csa_decode_step(q, qI, w, op_fmt, kI, kvc: KV, Nc, m, k, raw: KV, L, W, q_pos, out,
+                        score_fmt=HCL_FP32, kI_sf=None, lse=None, idx_out=None, scale=None,
+                        sink=None, ws=None, status=None, stream=None):
+    """One CSA decode step (Tq = 1): MXFP4-quantise qI (MXFP4 keys only), score, top-k, attend."""
+    B, _, H, d = q.shape
+    HI, dI = qI.shape[-2], qI.shape[-1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    need = decode_step_workspace_bytes(B, H, HI, Nc, k, W, op_fmt, score_fmt)
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    check(lib().hcl_csa_decode_step(_ptr(q), _ptr(qI), _ptr(w), op_fmt, _ptr(kI), _ptr(kI_sf),
+                                    kI.shape[1], score_fmt, B, H, HI, dI, d, kvc.ref(), Nc, m, k,
+                                    raw.ref(), L, W, _ptr(q_pos), scale, _ptr(sink), _ptr(out),
+                                    _ptr(lse), _ptr(idx_out), _ptr(ws), ws.numel(), _ptr(status),
+                                    _stream(stream)))
+    return out
+
+
+def hcl_selftest_bounded_wait(status, limit_us=1000, stream=None):
+    check(lib().hcl_selftest_bounded_wait(_ptr(status), limit_us, _stream(stream)))

@@ -1,0 +1,349 @@
+// api.cu -- the extern "C" boundary of libhcl: argument validation, error reporting and the
+// composition of the hot-path steps.  Every entry point validates on the host and enqueues
+// nothing when it returns an error.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <mutex>
+
+#include "hcl_common.cuh"
+#include "hcl_internal.h"
+
+namespace hcl {
+
+static thread_local char g_err[512] = "";
+
+hcl_status_t fail(hcl_status_t code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+hcl_status_t check_cuda(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return HCL_OK;
+  return fail(HCL_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+hcl_status_t check_launch(const char* what) { return check_cuda(cudaGetLastError(), what); }
+
+static int current_device() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return dev;
+}
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = current_device();
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+static long long clock_khz() {
+  static long long cache[64] = {0};
+  int dev = current_device();
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cache[dev] == 0) {
+    int khz = 0;
+    cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev);
+    cache[dev] = khz > 0 ? khz : 2000000;
+  }
+  return cache[dev];
+}
+
+long long wait_limit_cycles() { return clock_khz() * 1000LL; }  // about one second
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+namespace {
+
+__global__ void selftest_wait_kernel(int32_t* status, long long limit) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // Nothing ever arrives on `bar`: the bounded wait must give up and report.
+  if (!mbar_wait(&bar, 0, limit, nullptr)) report(status, HCL_ERR_TIMEOUT);
+}
+
+}  // namespace
+
+hcl_status_t launch_selftest_wait(int32_t* status, int limit_us, cudaStream_t st) {
+  const long long limit = clock_khz() * (long long)limit_us / 1000LL;
+  selftest_wait_kernel<<<1, 32, 0, st>>>(status, limit);
+  return check_launch("selftest");
+}
+
+}  // namespace hcl
+
+using namespace hcl;
+
+#define HCL_REQUIRE(cond, ...)                                       \
+  do {                                                               \
+    if (!(cond)) return fail(HCL_ERR_INVALID_ARG, __VA_ARGS__);      \
+  } while (0)
+
+static cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+static hcl_status_t check_kv(const hcl_kv_t* kv, int d, const char* name) {
+  HCL_REQUIRE(kv != nullptr, "%s: descriptor is NULL", name);
+  HCL_REQUIRE(kv->cap > 0, "%s: cap must be positive", name);
+  HCL_REQUIRE(kv->data != nullptr && aligned16(kv->data), "%s: data must be 16-byte aligned", name);
+  if (kv->fmt == HCL_FP8SPLIT) {
+    HCL_REQUIRE(kv->scale != nullptr && kv->rope != nullptr && aligned16(kv->rope),
+                "%s: FP8SPLIT needs scale and 16-byte aligned rope", name);
+  } else {
+    HCL_REQUIRE(kv->fmt == HCL_BF16, "%s: fmt must be HCL_BF16 or HCL_FP8SPLIT", name);
+  }
+  (void)d;
+  return HCL_OK;
+}
+
+extern "C" {
+
+const char* hcl_version(void) { return "libhcl 0.1 (sm_100a)"; }
+const char* hcl_last_error(void) { return g_err; }
+
+static hcl_status_t compress_common(const void* kv, const void* gate, const float* bias, int B,
+                                    int L, int d, int m, int overlap, int e0, int e1, void* out,
+                                    int out_fmt, int out_cap, void* stream, int max_m) {
+  HCL_REQUIRE(B >= 0 && L >= 0, "B and L must be non-negative");
+  HCL_REQUIRE(d > 0 && d % 8 == 0 && d <= 1024, "d must be a positive multiple of 8, <= 1024");
+  HCL_REQUIRE(m >= 1 && m <= max_m, "m must be in [1, %d]", max_m);
+  const long long n_ent = (L + (long long)m - 1) / m;
+  HCL_REQUIRE(0 <= e0 && e0 <= e1 && e1 <= n_ent && e1 <= out_cap,
+              "need 0 <= entry_begin <= entry_end <= min(ceil(L/m)=%lld, out_cap=%d)", n_ent,
+              out_cap);
+  HCL_REQUIRE(out_fmt == HCL_FP32 || out_fmt == HCL_BF16, "out_fmt must be HCL_FP32 or HCL_BF16");
+  if (e1 == e0 || B == 0) return HCL_OK;
+  HCL_REQUIRE(kv && gate && bias && out, "NULL pointer");
+  HCL_REQUIRE(aligned16(kv) && aligned16(gate) && aligned16(out), "kv, gate, out must be 16-byte aligned");
+  return launch_compress(kv, gate, bias, B, L, d, m, overlap, e0, e1, out, out_fmt, out_cap,
+                         as_stream(stream));
+}
+
+hcl_status_t hcl_csa_compress(const void* kv, const void* gate, const float* bias, int B, int L,
+                              int d, int m, int entry_begin, int entry_end, void* out,
+                              int out_fmt, int out_cap, void* stream) {
+  return compress_common(kv, gate, bias, B, L, d, m, 1, entry_begin, entry_end, out, out_fmt,
+                         out_cap, stream, 64);
+}
+
+hcl_status_t hcl_hca_compress(const void* kv, const void* gate, const float* bias, int B, int L,
+                              int d, int m, int entry_begin, int entry_end, void* out,
+                              int out_fmt, int out_cap, void* stream) {
+  return compress_common(kv, gate, bias, B, L, d, m, 0, entry_begin, entry_end, out, out_fmt,
+                         out_cap, stream, 1024);
+}
+
+hcl_status_t hcl_quant_kv_fp8(const void* kv, int64_t rows, int d, void* nope, float* scale,
+                              void* rope, void* stream) {
+  HCL_REQUIRE(rows >= 0, "rows must be non-negative");
+  HCL_REQUIRE(d >= 16 && d <= 256 && (d & (d - 1)) == 0, "d must be a power of two in [16, 256]");
+  if (rows == 0) return HCL_OK;
+  HCL_REQUIRE(kv && nope && scale && rope, "NULL pointer");
+  HCL_REQUIRE(aligned16(kv) && aligned16(rope) && ((uintptr_t)nope & 7) == 0,
+              "kv, rope must be 16-byte aligned and nope 8-byte aligned");
+  return launch_quant_kv_fp8(kv, rows, d, nope, scale, rope, as_stream(stream));
+}
+
+hcl_status_t hcl_quant_mxfp4(const void* x, int64_t rows, int cols, void* packed, void* e8m0,
+                             void* stream) {
+  HCL_REQUIRE(rows >= 0, "rows must be non-negative");
+  HCL_REQUIRE(cols > 0 && cols % 32 == 0, "cols must be a positive multiple of 32");
+  if (rows == 0) return HCL_OK;
+  HCL_REQUIRE(x && packed && e8m0, "NULL pointer");
+  HCL_REQUIRE(aligned16(x) && aligned16(packed), "x and packed must be 16-byte aligned");
+  return launch_quant_mxfp4(x, rows, cols, packed, e8m0, as_stream(stream));
+}
+
+hcl_status_t hcl_csa_index_scores(int op_fmt, const void* qI, const void* qI_sf, const float* w,
+                                  const void* kI, const void* kI_sf, int B, int Tq, int HI,
+                                  int dI, int Nc, int kI_cap, const int32_t* q_pos, int m,
+                                  void* scores, int score_fmt, int32_t* status, void* stream) {
+  HCL_REQUIRE(op_fmt == HCL_BF16 || op_fmt == HCL_MXFP4, "op_fmt must be HCL_BF16 or HCL_MXFP4");
+  HCL_REQUIRE(score_fmt == HCL_FP32 || score_fmt == HCL_BF16, "score_fmt must be HCL_FP32 or HCL_BF16");
+  HCL_REQUIRE(B >= 0 && Tq >= 0 && Nc >= 0, "negative size");
+  if (dI != 64) return fail(HCL_ERR_UNSUPPORTED, "only dI == 64 is supported (got %d)", dI);
+  HCL_REQUIRE(HI >= 1 && HI <= 16, "HI must be in [1, 16]");
+  HCL_REQUIRE(m >= 1, "m must be >= 1");
+  HCL_REQUIRE(Nc <= kI_cap, "Nc must be <= kI_cap");
+  if (op_fmt == HCL_MXFP4) HCL_REQUIRE(kI_cap % 8 == 0, "MXFP4 keys need kI_cap % 8 == 0");
+  if ((long long)B * Tq * Nc == 0) return HCL_OK;
+  HCL_REQUIRE(qI && w && kI && q_pos && scores, "NULL pointer");
+  HCL_REQUIRE(aligned16(qI) && aligned16(kI), "qI and kI must be 16-byte aligned");
+  if (op_fmt == HCL_MXFP4) HCL_REQUIRE(qI_sf && kI_sf && aligned16(kI_sf), "MXFP4 needs 16-byte aligned scale arrays");
+  IndexerArgs a{op_fmt, qI, qI_sf, w, kI, kI_sf, B, Tq, HI, dI, Nc, kI_cap, q_pos, m, scores,
+                score_fmt, status};
+  return launch_indexer(a, as_stream(stream));
+}
+
+size_t hcl_csa_topk_workspace_bytes(int B, int Tq, int Nc, int k, int score_fmt) {
+  return topk_workspace_bytes(B, Tq, Nc, k, score_fmt);
+}
+
+hcl_status_t hcl_csa_topk(const void* scores, int score_fmt, int B, int Tq, int Nc,
+                          const int32_t* q_pos, int m, int k, int32_t* idx, void* ws,
+                          size_t ws_bytes, int32_t* status, void* stream) {
+  HCL_REQUIRE(score_fmt == HCL_FP32 || score_fmt == HCL_BF16, "score_fmt must be HCL_FP32 or HCL_BF16");
+  HCL_REQUIRE(B >= 0 && Tq >= 0 && Nc >= 0, "negative size");
+  HCL_REQUIRE(k >= 1 && k <= 4096, "k must be in [1, 4096]");
+  HCL_REQUIRE(Nc <= (1 << 22), "Nc must be <= 2^22");
+  HCL_REQUIRE(m >= 1, "m must be >= 1");
+  HCL_REQUIRE(ws_bytes >= topk_workspace_bytes(B, Tq, Nc, k, score_fmt), "workspace too small");
+  if ((long long)B * Tq == 0) return HCL_OK;
+  HCL_REQUIRE(q_pos && idx && (scores || Nc == 0), "NULL pointer");
+  TopkArgs a{scores, score_fmt, B, Tq, Nc, q_pos, m, k, idx, status};
+  return launch_topk(a, ws, ws_bytes, as_stream(stream));
+}
+
+static hcl_status_t attn_common(int mode, const void* q, int B, int Tq, int H, int d,
+                                const hcl_kv_t* comp, int n_comp, int mh, const int32_t* idx,
+                                int k, const hcl_kv_t* raw, int L, int W, const int32_t* q_pos,
+                                float scale, const float* sink, void* out, float* lse, void* ws,
+                                size_t ws_bytes, int32_t* status, void* stream) {
+  HCL_REQUIRE(B >= 0 && Tq >= 0, "negative size");
+  if (d != 128) return fail(HCL_ERR_UNSUPPORTED, "only d == 128 is supported (got %d)", d);
+  HCL_REQUIRE(H >= 1 && H <= 128, "H must be in [1, 128]");
+  HCL_REQUIRE(W >= 0 && n_comp >= 0 && L >= 0, "negative size");
+  if (mode == 0) HCL_REQUIRE(k >= 0 && (k == 0 || idx != nullptr), "k must be >= 0 with idx given");
+  else HCL_REQUIRE(mh >= 1, "mh must be >= 1");
+  if ((long long)B * Tq == 0) return HCL_OK;
+  HCL_REQUIRE(q && out && q_pos, "NULL pointer");
+  HCL_REQUIRE(aligned16(q) && aligned16(out), "q and out must be 16-byte aligned");
+  hcl_status_t e = check_kv(comp, d, mode == 0 ? "kvc" : "kvh");
+  if (e != HCL_OK) return e;
+  e = check_kv(raw, d, "raw");
+  if (e != HCL_OK) return e;
+  HCL_REQUIRE(comp->fmt == raw->fmt, "compressed and raw stores must share one format");
+  HCL_REQUIRE(comp->cap >= n_comp || mode == 0, "kvh cap must be >= Nh");
+  const int list = mode == 0 ? k + W : n_comp + W;
+  const size_t need = hcl::attn_workspace_bytes(mode, B, Tq, H, list, W);
+  HCL_REQUIRE(ws_bytes >= need, "workspace too small: need %zu bytes", need);
+  AttnArgs a;
+  a.mode = mode; a.q = q; a.B = B; a.Tq = Tq; a.H = H; a.d = d;
+  a.comp = *comp; a.n_comp = n_comp; a.mh = mh; a.idx = idx; a.k = k;
+  a.raw = *raw; a.L = L; a.W = W; a.q_pos = q_pos; a.scale = scale; a.sink = sink;
+  a.out = out; a.lse = lse; a.status = status;
+  return launch_attn(a, ws, ws_bytes, as_stream(stream));
+}
+
+size_t hcl_csa_sparse_attn_workspace_bytes(int B, int Tq, int H, int k, int W) {
+  return hcl::attn_workspace_bytes(0, B, Tq, H, k + W, W);
+}
+
+hcl_status_t hcl_csa_sparse_attn(const void* q, int B, int Tq, int H, int d, const hcl_kv_t* kvc,
+                                 int Nc, const int32_t* idx, int k, const hcl_kv_t* raw, int L,
+                                 int W, const int32_t* q_pos, float scale, const float* sink,
+                                 void* out, float* lse, void* ws, size_t ws_bytes,
+                                 int32_t* status, void* stream) {
+  return attn_common(0, q, B, Tq, H, d, kvc, Nc, 1, idx, k, raw, L, W, q_pos, scale, sink, out,
+                     lse, ws, ws_bytes, status, stream);
+}
+
+size_t hcl_hca_dense_attn_workspace_bytes(int B, int Tq, int H, int Nh, int W) {
+  return hcl::attn_workspace_bytes(1, B, Tq, H, Nh + W, W);
+}
+
+hcl_status_t hcl_hca_dense_attn(const void* q, int B, int Tq, int H, int d, const hcl_kv_t* kvh,
+                                int Nh, int mh, const hcl_kv_t* raw, int L, int W,
+                                const int32_t* q_pos, float scale, const float* sink, void* out,
+                                float* lse, void* ws, size_t ws_bytes, int32_t* status,
+                                void* stream) {
+  return attn_common(1, q, B, Tq, H, d, kvh, Nh, mh, nullptr, 0, raw, L, W, q_pos, scale, sink,
+                     out, lse, ws, ws_bytes, status, stream);
+}
+
+// ---- fused decode step -----------------------------------------------------------------
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct DecodeWs {
+  size_t q_packed, q_sf, scores, idx, attn, total;
+};
+
+static DecodeWs decode_ws_layout(int B, int H, int HI, int Nc, int k, int W, int op_fmt,
+                                 int score_fmt, int dI) {
+  DecodeWs l;
+  size_t off = 0;
+  l.q_packed = off;
+  if (op_fmt == HCL_MXFP4) off += align256((size_t)B * HI * dI / 2);
+  l.q_sf = off;
+  if (op_fmt == HCL_MXFP4) off += align256((size_t)B * HI * dI / 32);
+  l.scores = off;
+  off += align256((size_t)B * Nc * (score_fmt == HCL_BF16 ? 2 : 4));
+  l.idx = off;
+  off += align256((size_t)B * k * 4);
+  l.attn = off;
+  off += align256(hcl::attn_workspace_bytes(0, B, 1, H, k + W, W));
+  l.total = off;
+  return l;
+}
+
+size_t hcl_csa_decode_step_workspace_bytes(int B, int H, int HI, int Nc, int k, int W,
+                                           int op_fmt, int score_fmt) {
+  return decode_ws_layout(B, H, HI, Nc, k, W, op_fmt, score_fmt, 64).total;
+}
+
+hcl_status_t hcl_csa_decode_step(const void* q, const void* qI_bf16, const float* w, int op_fmt,
+                                 const void* kI, const void* kI_sf, int kI_cap, int score_fmt,
+                                 int B, int H, int HI, int dI, int d, const hcl_kv_t* kvc,
+                                 int Nc, int m, int k, const hcl_kv_t* raw, int L, int W,
+                                 const int32_t* q_pos, float scale, const float* sink,
+                                 void* out, float* lse, int32_t* idx_out, void* ws,
+                                 size_t ws_bytes, int32_t* status, void* stream) {
+  if (dI != 64) return fail(HCL_ERR_UNSUPPORTED, "only dI == 64 is supported");
+  const DecodeWs l = decode_ws_layout(B, H, HI, Nc, k, W, op_fmt, score_fmt, dI);
+  HCL_REQUIRE(ws != nullptr && aligned16(ws) && ws_bytes >= l.total,
+              "decode workspace too small: need %zu bytes", l.total);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  const void* qI = qI_bf16;
+  const void* qI_sf = nullptr;
+  hcl_status_t e;
+  if (op_fmt == HCL_MXFP4) {
+    e = hcl_quant_mxfp4(qI_bf16, (int64_t)B * HI, dI, wsb + l.q_packed, wsb + l.q_sf, stream);
+    if (e != HCL_OK) return e;
+    qI = wsb + l.q_packed;
+    qI_sf = wsb + l.q_sf;
+  }
+  void* scores = wsb + l.scores;
+  e = hcl_csa_index_scores(op_fmt, qI, qI_sf, w, kI, kI_sf, B, 1, HI, dI, Nc, kI_cap, q_pos, m,
+                           scores, score_fmt, status, stream);
+  if (e != HCL_OK) return e;
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(wsb + l.idx);
+  e = hcl_csa_topk(scores, score_fmt, B, 1, Nc, q_pos, m, k, idx, nullptr, 0, status, stream);
+  if (e != HCL_OK) return e;
+  return hcl_csa_sparse_attn(q, B, 1, H, d, kvc, Nc, idx, k, raw, L, W, q_pos, scale, sink, out,
+                             lse, wsb + l.attn, ws_bytes - l.attn, status, stream);
+}
+
+hcl_status_t hcl_selftest_bounded_wait(int32_t* status, int limit_us, void* stream) {
+  HCL_REQUIRE(status != nullptr, "status must be given");
+  HCL_REQUIRE(limit_us >= 1 && limit_us <= 10 * 1000 * 1000, "limit_us must be in [1, 1e7]");
+  return launch_selftest_wait(status, limit_us, as_stream(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,544 @@
+// attn.cu -- attention over compressed entries plus the raw sliding window.
+//
+// [Tripbot §3.1 step 2] CSA attends over the top-k selected compressed entries;
+// [Tripbot §3.2; CSDN §1.2] HCA attends densely over every compressed entry;
+// [Tripbot §3.3] both add a branch over the most recent W raw tokens and may add a learnable
+// sink that lets the weights sum to less than one.  Per query head h, over the row list J:
+//     z_j = scale * q_h . kv_j,   o_h = sum_j softmax(z)_j kv_j,   lse_h = log sum_j e^{z_j}
+// Each compressed or raw row serves as both key and value of the one shared KV head.
+//
+// Design (B200): one block per (sequence, query group, KV split).  A query group is G queries
+// x H heads = up to 128 (query, head) rows, 16 per warp; all rows of a group share one KV row
+// list (CSA: G = 1, the query's selected entries then its window; HCA: the G consecutive
+// queries share the visible-entry prefix and the union of their windows, with per-row
+// causal masks).  The list is processed in chunks of 64 rows, gathered with cp.async into a
+// double-buffered, XOR-swizzled shared tile (split FP8 rows are staged raw and widened to
+// bf16 in shared memory with their per-row scale); QK^T and PV run on tensor cores
+// (mma.sync m16n8k16 bf16, fp32 accumulation) with an online softmax in registers.  With
+// several KV splits each block writes a normalised partial (o, lse) to the caller's
+// workspace and a merge kernel combines them by log-sum-exp.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "hcl_common.cuh"
+#include "hcl_internal.h"
+
+namespace hcl {
+namespace {
+
+constexpr int D = 128;
+constexpr int KVB = 64;
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LN2 = 0.6931471805599453f;
+
+struct AttnParams {
+  const __nv_bfloat16* q;
+  int B, Tq, H;
+  hcl_kv_t comp;
+  int n_comp, mh;
+  const int32_t* idx;
+  int k;
+  hcl_kv_t raw;
+  int W;
+  const int32_t* q_pos;
+  float scale_log2;
+  const float* sink;
+  __nv_bfloat16* out;
+  float* lse;
+  float* ws_o;
+  float* ws_lse;
+  int G, n_groups, splits, cps, rows_pad;
+  int32_t* status;
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// byte offset of 16-byte chunk `c` (0..15) of tile row `r` (256-byte rows, XOR swizzle)
+__device__ __forceinline__ uint32_t tile_off(int r, int c) {
+  return uint32_t(r) * 256u + (uint32_t(c ^ (r & 7)) << 4);
+}
+
+// Two E4M3 codes -> two bf16 values times `scale` (exact widening, one rounding).
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t codes, float scale) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(codes));
+  __half2 hv = *reinterpret_cast<__half2*>(&h2);
+  float2 f = __half22float2(hv);
+  return pack_bf16(f.x * scale, f.y * scale);
+}
+
+struct RowSrc {
+  long long slot;  // row slot in the store (-1: invalid)
+  int from_raw;
+};
+
+template <int KVFMT, int MODE, int NW>
+__global__ void __launch_bounds__(NW * 32)
+    attn_kernel(AttnParams p) {
+  constexpr int NT = NW * 32;
+  extern __shared__ __align__(128) uint8_t at_smem[];
+  uint8_t* tiles = at_smem;                              // [2][64][256 B] bf16
+  uint8_t* stage = at_smem + 2 * KVB * 256;              // fp8: [2][64][64 B] codes
+  float* sscale = reinterpret_cast<float*>(stage + 2 * KVB * 64);  // fp8: [2][64]
+  RowSrc* rsrc = reinterpret_cast<RowSrc*>(sscale + 2 * KVB);      // [2][64]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int bid = blockIdx.x;
+  const int split = bid % p.splits;
+  bid /= p.splits;
+  const int grp = bid % p.n_groups;
+  const int b = bid / p.n_groups;
+  const int t0 = grp * p.G;
+  const int gq = min(p.G, p.Tq - t0);  // queries in this group
+
+  // positions of the group's queries
+  int pmin = 0x7fffffff, pmax = -1;
+  for (int q = 0; q < gq; q++) {
+    int pp = p.q_pos[(size_t)b * p.Tq + t0 + q];
+    pmin = min(pmin, pp);
+    pmax = max(pmax, pp);
+  }
+  // row list: [list_a entries] ++ [raw tokens raw_lo .. raw_lo + n_raw - 1]
+  int n_a, raw_lo, n_raw;
+  if (MODE == 0) {
+    n_a = p.k;
+    raw_lo = pmax - p.W + 1;  // CSA: G == 1, window of the one query (may start < 0)
+    n_raw = p.W;
+  } else {
+    n_a = pmax < 0 ? 0 : min(p.n_comp, (pmax + 1) / p.mh);
+    raw_lo = pmin - p.W + 1;
+    n_raw = p.W > 0 ? max(0, pmax - raw_lo + 1) : 0;
+  }
+  const int total = n_a + n_raw;
+  const int n_chunks = (total + KVB - 1) / KVB;
+  const int c_begin = split * p.cps;
+  const int c_end = min(n_chunks, c_begin + p.cps);
+
+  // this thread's two rows (g, g+8 of the warp's 16) -> query, head, position, visibility
+  const int g = lane >> 2, tq = lane & 3;
+  int row_q[2], row_h[2], row_p[2], row_nv[2];
+  bool row_ok[2];
+#pragma unroll
+  for (int i = 0; i < 2; i++) {
+    const int r = warp * 16 + g + 8 * i;
+    const int q = r / p.H;
+    row_q[i] = q;
+    row_h[i] = r % p.H;
+    row_ok[i] = q < gq;
+    row_p[i] = row_ok[i] ? p.q_pos[(size_t)b * p.Tq + t0 + q] : -1;
+    row_nv[i] = row_p[i] < 0 ? 0 : min(p.n_comp, (row_p[i] + 1) / max(1, p.mh));
+  }
+
+  // Q fragments (A operand, 16 rows x 128 dims = 8 k-steps)
+  uint32_t qa[8][4];
+  {
+    const __nv_bfloat16* qrow[2];
+#pragma unroll
+    for (int i = 0; i < 2; i++)
+      qrow[i] = row_ok[i] ? p.q + (((size_t)b * p.Tq + t0 + row_q[i]) * p.H + row_h[i]) * D
+                          : nullptr;
+#pragma unroll
+    for (int kk = 0; kk < 8; kk++) {
+      const int c0 = kk * 16 + tq * 2;
+      qa[kk][0] = qrow[0] ? *reinterpret_cast<const uint32_t*>(qrow[0] + c0) : 0u;
+      qa[kk][1] = qrow[1] ? *reinterpret_cast<const uint32_t*>(qrow[1] + c0) : 0u;
+      qa[kk][2] = qrow[0] ? *reinterpret_cast<const uint32_t*>(qrow[0] + c0 + 8) : 0u;
+      qa[kk][3] = qrow[1] ? *reinterpret_cast<const uint32_t*>(qrow[1] + c0 + 8) : 0u;
+    }
+  }
+
+  float o[16][4];
+#pragma unroll
+  for (int n = 0; n < 16; n++) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
+
+  // ---- gather of one chunk into buffer `buf` ----
+  auto resolve = [&](int chunk, int buf) {
+    for (int j = tid; j < KVB; j += NT) {
+      const int e = chunk * KVB + j;
+      RowSrc rs{-1, 0};
+      if (e < n_a) {
+        long long ent;
+        if (MODE == 0) {
+          ent = p.idx[((size_t)b * p.Tq + t0) * p.k + e];
+          if (ent < -1 || ent >= p.n_comp) {
+            report(p.status, HCL_ERR_DEVICE_FAULT);
+            ent = -1;
+          }
+        } else {
+          ent = e;
+        }
+        if (ent >= 0) rs.slot = (long long)b * p.comp.cap + (ent % p.comp.cap);
+      } else if (e < total) {
+        const long long u = (long long)raw_lo + (e - n_a);
+        if (u >= 0) { rs.slot = (long long)b * p.raw.cap + (u % p.raw.cap); rs.from_raw = 1; }
+      }
+      rsrc[buf * KVB + j] = rs;
+    }
+  };
+  auto issue = [&](int buf) {
+    uint8_t* tile = tiles + buf * KVB * 256;
+    if (KVFMT == HCL_BF16) {
+      for (int u = tid; u < KVB * 16; u += NT) {
+        const int r = u >> 4, c = u & 15;
+        const RowSrc rs = rsrc[buf * KVB + r];
+        uint8_t* dst = tile + tile_off(r, c);
+        if (rs.slot >= 0) {
+          const hcl_kv_t& st = rs.from_raw ? p.raw : p.comp;
+          cp_async16(dst, static_cast<const uint8_t*>(st.data) + rs.slot * 256 + c * 16);
+        } else {
+          *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+        }
+      }
+    } else {
+      // rope half straight into tile columns 64..127; codes and scale into staging
+      for (int u = tid; u < KVB * 13; u += NT) {
+        const int r = u / 13, c = u % 13;
+        const RowSrc rs = rsrc[buf * KVB + r];
+        const hcl_kv_t& st = rs.from_raw ? p.raw : p.comp;
+        if (c < 8) {
+          uint8_t* dst = tile + tile_off(r, 8 + c);
+          if (rs.slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.rope) + rs.slot * 128 + c * 16);
+          else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+        } else if (c < 12) {
+          uint8_t* dst = stage + (buf * KVB + r) * 64 + (c - 8) * 16;
+          if (rs.slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.data) + rs.slot * 64 + (c - 8) * 16);
+          else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+        } else {
+          float* dst = sscale + buf * KVB + r;
+          if (rs.slot >= 0)
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)),
+                         "l"(st.scale + rs.slot)
+                         : "memory");
+          else *dst = 0.f;
+        }
+      }
+    }
+    cp_async_commit();
+  };
+  auto widen = [&](int buf) {  // FP8 staging -> bf16 tile columns 0..63
+    uint8_t* tile = tiles + buf * KVB * 256;
+    for (int u = tid; u < KVB * 8; u += NT) {
+      const int r = u >> 3, c = u & 7;  // 8 codes -> one 16-byte bf16 chunk
+      const uint2 codes = *reinterpret_cast<const uint2*>(stage + (buf * KVB + r) * 64 + c * 8);
+      const float sc = sscale[buf * KVB + r];
+      uint4 v;
+      v.x = e4m3x2_to_bf16x2(uint16_t(codes.x & 0xffff), sc);
+      v.y = e4m3x2_to_bf16x2(uint16_t(codes.x >> 16), sc);
+      v.z = e4m3x2_to_bf16x2(uint16_t(codes.y & 0xffff), sc);
+      v.w = e4m3x2_to_bf16x2(uint16_t(codes.y >> 16), sc);
+      *reinterpret_cast<uint4*>(tile + tile_off(r, c)) = v;
+    }
+  };
+
+  if (c_begin < c_end) {
+    resolve(c_begin, 0);
+    __syncthreads();
+    issue(0);
+  }
+  for (int c = c_begin; c < c_end; c++) {
+    const int buf = (c - c_begin) & 1;
+    if (c + 1 < c_end) {
+      resolve(c + 1, buf ^ 1);
+      __syncthreads();
+      issue(buf ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    if (KVFMT == HCL_FP8SPLIT) {
+      widen(buf);
+      __syncthreads();
+    }
+    const uint32_t tbase = smem_u32(tiles + buf * KVB * 256);
+
+    // S = Q K^T for this warp's 16 rows x 64 kv rows
+    float s[8][4];
+#pragma unroll
+    for (int n = 0; n < 8; n++) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+#pragma unroll
+    for (int n = 0; n < 8; n++) {
+#pragma unroll
+      for (int kk = 0; kk < 8; kk += 2) {
+        const int mi = lane >> 3, ri = lane & 7;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(tbase + tile_off(n * 8 + ri, kk * 2 + mi), b0, b1, b2, b3);
+        mma_bf16(s[n], qa[kk], b0, b1);
+        mma_bf16(s[n], qa[kk + 1], b2, b3);
+      }
+    }
+    // mask, scale (log2 domain), online softmax
+    float cmax[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int n = 0; n < 8; n++) {
+#pragma unroll
+      for (int e2 = 0; e2 < 4; e2++) {
+        const int i = e2 >> 1;
+        const int j = n * 8 + tq * 2 + (e2 & 1);
+        const RowSrc rs = rsrc[buf * KVB + j];
+        const int e = c * KVB + j;
+        bool vis = rs.slot >= 0 && row_ok[i];
+        if (MODE == 1 && vis) {
+          if (e < n_a) vis = e < row_nv[i];
+          else {
+            const int u = raw_lo + (e - n_a);
+            vis = u <= row_p[i] && u > row_p[i] - p.W;
+          }
+        }
+        const float z = vis ? s[n][e2] * p.scale_log2 : -INFINITY;
+        s[n][e2] = z;
+        cmax[i] = fmaxf(cmax[i], z);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 2; i++) {
+      cmax[i] = fmaxf(cmax[i], __shfl_xor_sync(0xffffffffu, cmax[i], 1));
+      cmax[i] = fmaxf(cmax[i], __shfl_xor_sync(0xffffffffu, cmax[i], 2));
+    }
+    float corr[2], muse[2];
+#pragma unroll
+    for (int i = 0; i < 2; i++) {
+      const float mnew = fmaxf(mrow[i], cmax[i]);
+      muse[i] = mnew == -INFINITY ? 0.f : mnew;
+      corr[i] = exp2f(mrow[i] - muse[i]);
+      mrow[i] = mnew;
+    }
+    float rsum[2] = {0.f, 0.f};
+    uint32_t pa[4][4];
+#pragma unroll
+    for (int n = 0; n < 8; n++) {
+      const float p0 = exp2f(s[n][0] - muse[0]), p1 = exp2f(s[n][1] - muse[0]);
+      const float p2 = exp2f(s[n][2] - muse[1]), p3 = exp2f(s[n][3] - muse[1]);
+      rsum[0] += p0 + p1;
+      rsum[1] += p2 + p3;
+      const int kk = n >> 1, hi = n & 1;
+      pa[kk][hi * 2 + 0] = pack_bf16(p0, p1);
+      pa[kk][hi * 2 + 1] = pack_bf16(p2, p3);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; i++) lrow[i] = lrow[i] * corr[i] + rsum[i];
+#pragma unroll
+    for (int n = 0; n < 16; n++) {
+      o[n][0] *= corr[0]; o[n][1] *= corr[0];
+      o[n][2] *= corr[1]; o[n][3] *= corr[1];
+    }
+    // O += P V
+#pragma unroll
+    for (int kk = 0; kk < 4; kk++) {
+#pragma unroll
+      for (int n = 0; n < 16; n += 2) {
+        const int mi = lane >> 3, ri = lane & 7;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(tbase + tile_off(kk * 16 + (mi & 1) * 8 + ri, n + (mi >> 1)), b0, b1, b2, b3);
+        mma_bf16(o[n], pa[kk], b0, b1);
+        mma_bf16(o[n + 1], pa[kk], b2, b3);
+      }
+    }
+    __syncthreads();
+  }
+
+  // row sums across the 4 threads of a row
+#pragma unroll
+  for (int i = 0; i < 2; i++) {
+    lrow[i] += __shfl_xor_sync(0xffffffffu, lrow[i], 1);
+    lrow[i] += __shfl_xor_sync(0xffffffffu, lrow[i], 2);
+  }
+  const size_t item = (size_t)blockIdx.x;
+#pragma unroll
+  for (int i = 0; i < 2; i++) {
+    if (!row_ok[i]) continue;
+    const int r = warp * 16 + g + 8 * i;
+    float m2 = mrow[i], l2 = lrow[i], f = 1.f;
+    if (p.splits == 1) {
+      if (p.sink) {
+        const float s2 = p.sink[row_h[i]] * LOG2E;
+        const float mm = fmaxf(m2, s2);
+        f = (l2 > 0.f) ? exp2f(m2 - mm) : 0.f;
+        l2 = l2 * f + exp2f(s2 - mm);
+        m2 = mm;
+      }
+      const float inv = l2 > 0.f ? f / l2 : 0.f;
+      const size_t orow = ((size_t)b * p.Tq + t0 + row_q[i]) * p.H + row_h[i];
+      __nv_bfloat16* dst = p.out + orow * D;
+#pragma unroll
+      for (int n = 0; n < 16; n++) {
+        const int col = n * 8 + tq * 2;
+        *reinterpret_cast<uint32_t*>(dst + col) = pack_bf16(o[n][2 * i] * inv, o[n][2 * i + 1] * inv);
+      }
+      if (p.lse && tq == 0) p.lse[orow] = l2 > 0.f ? (m2 + log2f(l2)) * LN2 : -INFINITY;
+    } else {
+      const float inv = l2 > 0.f ? 1.f / l2 : 0.f;
+      float* dst = p.ws_o + (item * p.rows_pad + r) * D;
+#pragma unroll
+      for (int n = 0; n < 16; n++) {
+        const int col = n * 8 + tq * 2;
+        *reinterpret_cast<float2*>(dst + col) = make_float2(o[n][2 * i] * inv, o[n][2 * i + 1] * inv);
+      }
+      if (tq == 0) p.ws_lse[item * p.rows_pad + r] = l2 > 0.f ? m2 + log2f(l2) : -INFINITY;
+    }
+  }
+}
+
+// Combine the KV splits of every (query, head) row by log-sum-exp (log2 domain partials).
+__global__ void attn_merge_kernel(AttnParams p) {
+  const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long nrows = (long long)p.B * p.Tq * p.H;
+  if (gw >= nrows) return;
+  const int h = int(gw % p.H);
+  const long long bt = gw / p.H;
+  const int t = int(bt % p.Tq);
+  const int b = int(bt / p.Tq);
+  const int grp = t / p.G;
+  const int r = (t - grp * p.G) * p.H + h;
+  const size_t item0 = ((size_t)b * p.n_groups + grp) * p.splits;
+  float M = -INFINITY;
+  for (int s = 0; s < p.splits; s++) M = fmaxf(M, p.ws_lse[(item0 + s) * p.rows_pad + r]);
+  float s2 = -INFINITY;
+  if (p.sink) {
+    s2 = p.sink[h] * LOG2E;
+    M = fmaxf(M, s2);
+  }
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float den = 0.f;
+  if (M > -INFINITY) {
+    for (int s = 0; s < p.splits; s++) {
+      const float ls = p.ws_lse[(item0 + s) * p.rows_pad + r];
+      if (ls == -INFINITY) continue;
+      const float wgt = exp2f(ls - M);
+      den += wgt;
+      const float4 v = reinterpret_cast<const float4*>(p.ws_o + ((item0 + s) * p.rows_pad + r) * D)[lane];
+      acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
+    }
+    if (p.sink) den += exp2f(s2 - M);
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  __nv_bfloat16* dst = p.out + gw * D + lane * 4;
+  reinterpret_cast<uint2*>(dst)[0] = make_uint2(pack_bf16(acc.x * inv, acc.y * inv),
+                                                pack_bf16(acc.z * inv, acc.w * inv));
+  if (p.lse && lane == 0) p.lse[gw] = den > 0.f ? (M + log2f(den)) * LN2 : -INFINITY;
+}
+
+struct Plan {
+  int G, NW, n_groups, splits, cps, rows_pad, n_chunks_max;
+};
+
+Plan make_plan(int mode, int B, int Tq, int H, int list_max) {
+  Plan pl;
+  pl.G = mode == 0 ? 1 : std::max(1, 128 / H);
+  pl.G = std::min(pl.G, Tq);
+  const int rows = pl.G * H;
+  pl.NW = rows <= 16 ? 1 : rows <= 32 ? 2 : rows <= 64 ? 4 : 8;
+  pl.rows_pad = pl.NW * 16;
+  pl.n_groups = (Tq + pl.G - 1) / pl.G;
+  pl.n_chunks_max = std::max(1, (list_max + KVB - 1) / KVB);
+  const long long blocks = (long long)B * pl.n_groups;
+  const long long target = 2LL * num_sms();
+  int splits = (int)std::max(1LL, std::min<long long>(pl.n_chunks_max, (target + blocks - 1) / blocks));
+  pl.cps = (pl.n_chunks_max + splits - 1) / splits;
+  pl.splits = (pl.n_chunks_max + pl.cps - 1) / pl.cps;
+  return pl;
+}
+
+template <int KVFMT, int MODE, int NW>
+hcl_status_t launch_t(const AttnParams& p, cudaStream_t st, long long grid) {
+  const size_t smem = 2 * KVB * 256 + 2 * KVB * 64 + 2 * KVB * 4 + 2 * KVB * sizeof(RowSrc);
+  attn_kernel<KVFMT, MODE, NW><<<(unsigned)grid, NW * 32, smem, st>>>(p);
+  return check_launch("attention");
+}
+
+template <int KVFMT, int MODE>
+hcl_status_t launch_nw(const AttnParams& p, int NW, cudaStream_t st, long long grid) {
+  switch (NW) {
+    case 1: return launch_t<KVFMT, MODE, 1>(p, st, grid);
+    case 2: return launch_t<KVFMT, MODE, 2>(p, st, grid);
+    case 4: return launch_t<KVFMT, MODE, 4>(p, st, grid);
+    default: return launch_t<KVFMT, MODE, 8>(p, st, grid);
+  }
+}
+
+int list_max_of(const AttnArgs& a) {
+  if (a.mode == 0) return a.k + std::max(0, a.W);
+  // HCA: visible entries (at most n_comp) plus the union of the group's windows
+  const Plan pl = make_plan(1, a.B, a.Tq, a.H, 0);
+  return a.n_comp + (a.W > 0 ? a.W + pl.G - 1 : 0);
+}
+
+}  // namespace
+
+size_t attn_workspace_bytes(int mode, int B, int Tq, int H, int list_len, int W) {
+  (void)W;
+  const Plan pl = make_plan(mode, B, Tq, H, list_len);
+  if (pl.splits <= 1) return 0;
+  const size_t items = (size_t)B * pl.n_groups * pl.splits;
+  return items * pl.rows_pad * (D + 1) * sizeof(float);
+}
+
+hcl_status_t launch_attn(const AttnArgs& a, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if ((long long)a.B * a.Tq == 0) return HCL_OK;
+  const int list_max = list_max_of(a);
+  const Plan pl = make_plan(a.mode, a.B, a.Tq, a.H, list_max);
+  AttnParams p;
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.B = a.B; p.Tq = a.Tq; p.H = a.H;
+  p.comp = a.comp; p.n_comp = a.n_comp; p.mh = a.mode == 0 ? 1 : a.mh;
+  p.idx = a.idx; p.k = a.k;
+  p.raw = a.raw; p.W = a.W;
+  p.q_pos = a.q_pos;
+  p.scale_log2 = a.scale * LOG2E;
+  p.sink = a.sink;
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.lse = a.lse;
+  p.G = pl.G; p.n_groups = pl.n_groups; p.splits = pl.splits; p.cps = pl.cps;
+  p.rows_pad = pl.rows_pad;
+  p.status = a.status;
+  p.ws_o = nullptr;
+  p.ws_lse = nullptr;
+  if (pl.splits > 1) {
+    const size_t items = (size_t)a.B * pl.n_groups * pl.splits;
+    const size_t need = items * pl.rows_pad * (D + 1) * sizeof(float);
+    if (ws == nullptr || ws_bytes < need)
+      return fail(HCL_ERR_INVALID_ARG, "attention workspace too small: need %zu bytes, got %zu",
+                  need, ws_bytes);
+    p.ws_o = static_cast<float*>(ws);
+    p.ws_lse = p.ws_o + items * pl.rows_pad * D;
+  }
+  const long long grid = (long long)a.B * pl.n_groups * pl.splits;
+  hcl_status_t e;
+  const bool fp8 = a.comp.fmt == HCL_FP8SPLIT;
+  if (a.mode == 0) e = fp8 ? launch_nw<HCL_FP8SPLIT, 0>(p, pl.NW, st, grid)
+                           : launch_nw<HCL_BF16, 0>(p, pl.NW, st, grid);
+  else e = fp8 ? launch_nw<HCL_FP8SPLIT, 1>(p, pl.NW, st, grid)
+               : launch_nw<HCL_BF16, 1>(p, pl.NW, st, grid);
+  if (e != HCL_OK || pl.splits == 1) return e;
+  const long long threads = (long long)a.B * a.Tq * a.H * 32;
+  attn_merge_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(p);
+  return check_launch("attention merge");
+}
+
+}  // namespace hcl

@@ -1,0 +1,96 @@
+// hcl_internal.h -- host-side declarations shared by the libhcl translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/hcl.h"
+
+namespace hcl {
+
+// Thread-local error message of the last failing call; returns `code`.
+hcl_status_t fail(hcl_status_t code, const char* fmt, ...);
+// Maps a pending launch / runtime error to HCL_ERR_CUDA with a message.
+hcl_status_t check_cuda(cudaError_t e, const char* what);
+hcl_status_t check_launch(const char* what);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Number of SMs of the current device (cached per device).
+int num_sms();
+// Bounded-wait budget for device spin loops, in SM clock cycles (about one second).
+long long wait_limit_cycles();
+
+// cuTensorMapEncodeTiled obtained from the driver at run time (no libcuda link).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled();
+
+// ---- launchers (each validates nothing; the extern "C" layer does) ----
+
+hcl_status_t launch_compress(const void* kv, const void* gate, const float* bias, int B, int L,
+                             int d, int m, int overlap, int e0, int e1, void* out, int out_fmt,
+                             int out_cap, cudaStream_t st);
+
+hcl_status_t launch_quant_kv_fp8(const void* kv, int64_t rows, int d, void* nope, float* scale,
+                                 void* rope, cudaStream_t st);
+hcl_status_t launch_quant_mxfp4(const void* x, int64_t rows, int cols, void* packed, void* sf,
+                                cudaStream_t st);
+
+struct IndexerArgs {
+  int op_fmt;
+  const void* qI;
+  const void* qI_sf;
+  const float* w;
+  const void* kI;
+  const void* kI_sf;
+  int B, Tq, HI, dI, Nc, kI_cap;
+  const int32_t* q_pos;
+  int m;
+  void* scores;
+  int score_fmt;
+  int32_t* status;
+};
+hcl_status_t launch_indexer(const IndexerArgs& a, cudaStream_t st);
+
+struct TopkArgs {
+  const void* scores;
+  int score_fmt;
+  int B, Tq, Nc;
+  const int32_t* q_pos;
+  int m, k;
+  int32_t* idx;
+  int32_t* status;
+};
+size_t topk_workspace_bytes(int B, int Tq, int Nc, int k, int score_fmt);
+hcl_status_t launch_topk(const TopkArgs& a, void* ws, size_t ws_bytes, cudaStream_t st);
+
+// One attention launch: CSA (selected entries + window) or HCA (visible entries + window).
+struct AttnArgs {
+  int mode;  // 0 = CSA, 1 = HCA
+  const void* q;
+  int B, Tq, H, d;
+  hcl_kv_t comp;  // compressed entries
+  int n_comp;     // CSA: Nc; HCA: Nh
+  int mh;         // HCA ratio
+  const int32_t* idx;
+  int k;
+  hcl_kv_t raw;
+  int L, W;
+  const int32_t* q_pos;
+  float scale;
+  const float* sink;
+  void* out;
+  float* lse;
+  int32_t* status;
+};
+size_t attn_workspace_bytes(int mode, int B, int Tq, int H, int list_len, int W);
+hcl_status_t launch_attn(const AttnArgs& a, void* ws, size_t ws_bytes, cudaStream_t st);
+
+hcl_status_t launch_selftest_wait(int32_t* status, int limit_us, cudaStream_t st);
+
+}  // namespace hcl

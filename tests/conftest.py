@@ -18,3 +18,14 @@ def orc():
     import oracle
     oracle.lib()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def hcl():
+    """The CUDA library; GPU tests skip without a device and fail loudly without libhcl.so."""
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from heavily_compressed_long_b200 import api, _lib
+    _lib.lib()  # raises if libhcl.so is missing
+    return api
