@@ -431,8 +431,60 @@ def run_hcl(args, rank, world, local_rank):
     graphs.clear()
 
 
+def run_kernel_micro(args, local_rank):
+    """One kernel alone on one input set of `--batch` sequences (indexer: larger than L2),
+    for profiling: times back-to-back launches with CUDA events and prints a JSON line."""
+    import torch
+    from heavily_compressed_long_b200 import api
+    from heavily_compressed_long_b200.api import HCL_MXFP4
+    cfg = workload()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    B = args.batch
+    (p,) = build_inputs(cfg, B, 0, 1, device)
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        api.hcl_quant_mxfp4(p.qI, p.qI_packed, p.qI_sf, stream=stream)
+        p.step_parts(stream=stream)
+    torch.cuda.synchronize()
+
+    def launch():
+        if args.kernel == "indexer":
+            api.hcl_csa_index_scores(HCL_MXFP4, p.qI_packed, p.w, p.kI, p.q_pos, p.m, p.scores,
+                                     Nc=p.Nc, qI_sf=p.qI_sf, kI_sf=p.kI_sf, stream=stream)
+        elif args.kernel == "topk":
+            api.hcl_csa_topk(p.scores, p.q_pos, p.m, p.k, p.idx, stream=stream)
+        else:
+            api.hcl_csa_sparse_attn(p.q, p.kvc, p.Nc, p.idx, p.raw, p.L, p.W, p.q_pos, p.out,
+                                    lse=p.lse, ws=p.attn_ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            launch()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            launch()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    hbm, src = peaks()
+    nbytes = indexer_bytes_per_launch(cfg, B) if args.kernel == "indexer" else None
+    line = {"kernel": args.kernel, "workload": f"{cfg.name} with B={B}", "ms_per_launch": ms,
+            "launches": args.steps}
+    if nbytes:
+        line.update({"bytes_per_launch": nbytes, "achieved_gbs": nbytes / ms / 1e6,
+                     "peak_gbs": hbm, "frac": nbytes / ms / 1e6 / hbm, "peak_source": src})
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--kernel", default=None, choices=["indexer", "topk", "attn"],
+                    help="time one kernel alone (profiling aid) instead of the whole step")
+    ap.add_argument("--batch", type=int, default=16, help="sequences for --kernel")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=20)
@@ -448,6 +500,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.kernel:
+        run_kernel_micro(args, local_rank)
         return
     import torch
     import torch.distributed as dist

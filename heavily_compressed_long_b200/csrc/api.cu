@@ -240,8 +240,7 @@ static hcl_status_t attn_common(int mode, const void* q, int B, int Tq, int H, i
   if (e != HCL_OK) return e;
   HCL_REQUIRE(comp->fmt == raw->fmt, "compressed and raw stores must share one format");
   HCL_REQUIRE(comp->cap >= n_comp || mode == 0, "kvh cap must be >= Nh");
-  const int list = mode == 0 ? k + W : n_comp + W;
-  const size_t need = hcl::attn_workspace_bytes(mode, B, Tq, H, list, W);
+  const size_t need = hcl::attn_workspace_bytes(mode, B, Tq, H, mode == 0 ? k : n_comp, W);
   HCL_REQUIRE(ws_bytes >= need, "workspace too small: need %zu bytes", need);
   AttnArgs a;
   a.mode = mode; a.q = q; a.B = B; a.Tq = Tq; a.H = H; a.d = d;
@@ -252,7 +251,7 @@ static hcl_status_t attn_common(int mode, const void* q, int B, int Tq, int H, i
 }
 
 size_t hcl_csa_sparse_attn_workspace_bytes(int B, int Tq, int H, int k, int W) {
-  return hcl::attn_workspace_bytes(0, B, Tq, H, k + W, W);
+  return hcl::attn_workspace_bytes(0, B, Tq, H, k, W);
 }
 
 hcl_status_t hcl_csa_sparse_attn(const void* q, int B, int Tq, int H, int d, const hcl_kv_t* kvc,
@@ -265,7 +264,7 @@ hcl_status_t hcl_csa_sparse_attn(const void* q, int B, int Tq, int H, int d, con
 }
 
 size_t hcl_hca_dense_attn_workspace_bytes(int B, int Tq, int H, int Nh, int W) {
-  return hcl::attn_workspace_bytes(1, B, Tq, H, Nh + W, W);
+  return hcl::attn_workspace_bytes(1, B, Tq, H, Nh, W);
 }
 
 hcl_status_t hcl_hca_dense_attn(const void* q, int B, int Tq, int H, int d, const hcl_kv_t* kvh,
@@ -298,7 +297,7 @@ static DecodeWs decode_ws_layout(int B, int H, int HI, int Nc, int k, int W, int
   l.idx = off;
   off += align256((size_t)B * k * 4);
   l.attn = off;
-  off += align256(hcl::attn_workspace_bytes(0, B, 1, H, k + W, W));
+  off += align256(hcl::attn_workspace_bytes(0, B, 1, H, k, W));
   l.total = off;
   return l;
 }

@@ -136,7 +136,9 @@ __global__ void __launch_bounds__(NW * 32)
   const int total = n_a + n_raw;
   const int n_chunks = (total + KVB - 1) / KVB;
   const int c_begin = split * p.cps;
-  const int c_end = min(n_chunks, c_begin + p.cps);
+  // the last split takes every remaining chunk (query groups whose positions are not
+  // consecutive may have longer lists than the host planned for)
+  const int c_end = split == p.splits - 1 ? n_chunks : min(n_chunks, c_begin + p.cps);
 
   // this thread's two rows (g, g+8 of the warp's 16) -> query, head, position, visibility
   const int g = lane >> 2, tq = lane & 3;
@@ -482,18 +484,19 @@ hcl_status_t launch_nw(const AttnParams& p, int NW, cudaStream_t st, long long g
   }
 }
 
-int list_max_of(const AttnArgs& a) {
-  if (a.mode == 0) return a.k + std::max(0, a.W);
-  // HCA: visible entries (at most n_comp) plus the union of the group's windows
-  const Plan pl = make_plan(1, a.B, a.Tq, a.H, 0);
-  return a.n_comp + (a.W > 0 ? a.W + pl.G - 1 : 0);
+// Longest row list a block may process: CSA k selected entries + W window rows; HCA every
+// entry (n = Nh) plus the union of the G windows of a query group.  The workspace query and
+// the launch both plan from this one number.
+int list_max_for(int mode, int B, int Tq, int H, int n, int W) {
+  if (mode == 0) return n + std::max(0, W);
+  const Plan pl = make_plan(1, B, Tq, H, 0);
+  return n + (W > 0 ? W + pl.G - 1 : 0);
 }
 
 }  // namespace
 
-size_t attn_workspace_bytes(int mode, int B, int Tq, int H, int list_len, int W) {
-  (void)W;
-  const Plan pl = make_plan(mode, B, Tq, H, list_len);
+size_t attn_workspace_bytes(int mode, int B, int Tq, int H, int n, int W) {
+  const Plan pl = make_plan(mode, B, Tq, H, list_max_for(mode, B, Tq, H, n, W));
   if (pl.splits <= 1) return 0;
   const size_t items = (size_t)B * pl.n_groups * pl.splits;
   return items * pl.rows_pad * (D + 1) * sizeof(float);
@@ -501,7 +504,7 @@ size_t attn_workspace_bytes(int mode, int B, int Tq, int H, int list_len, int W)
 
 hcl_status_t launch_attn(const AttnArgs& a, void* ws, size_t ws_bytes, cudaStream_t st) {
   if ((long long)a.B * a.Tq == 0) return HCL_OK;
-  const int list_max = list_max_of(a);
+  const int list_max = list_max_for(a.mode, a.B, a.Tq, a.H, a.mode == 0 ? a.k : a.n_comp, a.W);
   const Plan pl = make_plan(a.mode, a.B, a.Tq, a.H, list_max);
   AttnParams p;
   p.q = static_cast<const __nv_bfloat16*>(a.q);

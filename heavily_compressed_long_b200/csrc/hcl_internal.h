@@ -88,7 +88,8 @@ struct AttnArgs {
   float* lse;
   int32_t* status;
 };
-size_t attn_workspace_bytes(int mode, int B, int Tq, int H, int list_len, int W);
+// n = k (CSA) or Nh (HCA)
+size_t attn_workspace_bytes(int mode, int B, int Tq, int H, int n, int W);
 hcl_status_t launch_attn(const AttnArgs& a, void* ws, size_t ws_bytes, cudaStream_t st);
 
 hcl_status_t launch_selftest_wait(int32_t* status, int limit_us, cudaStream_t st);

@@ -32,6 +32,23 @@ def bf16_ulp(x):
     return 2.0 ** (np.maximum(e, -126) - 7)
 
 
+def bf16_out_ratio(gpu, ref, rel=1e-3):
+    """Worst ratio of |gpu - ref| to the bf16-output allowance: the benchmark spec's fp32
+    tolerance (rel, norm-wise per row) plus one bf16 ulp of ref for the output rounding.
+    <= 1 passes.  -inf entries must match exactly."""
+    g = np.asarray(gpu, np.float64)
+    r = np.asarray(ref, np.float64)
+    g = g.reshape(-1, g.shape[-1])
+    r = r.reshape(-1, r.shape[-1])
+    fin = np.isfinite(r)
+    if not np.array_equal(fin, np.isfinite(g)):
+        return float("inf")
+    rz = np.where(fin, r, 0.0)
+    gz = np.where(fin, g, 0.0)
+    allow = bf16_ulp(rz) + rel * np.abs(rz).max(1, keepdims=True)
+    return float((np.abs(gz - rz) / allow).max()) if rz.size else 0.0
+
+
 def within_bf16_ulp(gpu, ref, n_ulp=1.0):
     g = np.asarray(gpu, np.float64)
     r = np.asarray(ref, np.float64)

@@ -9,7 +9,7 @@ import torch
 
 import oracle
 from synth import gen
-from tests.helpers import as_f64, check_topk_band, cuda, rel_rowwise, within_bf16_ulp
+from tests.helpers import as_f64, bf16_out_ratio, check_topk_band, cuda, rel_rowwise
 
 pytestmark = pytest.mark.gpu
 RNG = np.random.default_rng(20261202)
@@ -79,7 +79,7 @@ def test_compress(hcl, B, L, m, overlap):
     torch.cuda.synchronize()
     assert rel_rowwise(as_f64(out32[:, :n]), ref) <= 1e-3
     assert torch.isnan(out32[:, n:]).all()              # nothing written past the entries
-    assert within_bf16_ulp(as_f64(out16), ref, 1.0)
+    assert bf16_out_ratio(as_f64(out16), ref) <= 1.0
 
 
 def test_compress_entry_range(hcl):
@@ -137,7 +137,7 @@ def test_index_scores_mxfp4_bf16_scores(hcl, B, Tq, Nc, cap):
     hcl.hcl_csa_index_scores(hcl.HCL_MXFP4, t(qp), cuda(w), t(kp), cuda(pos), 4, out, Nc=Nc,
                              qI_sf=t(qs), kI_sf=t(ks))
     torch.cuda.synchronize()
-    assert within_bf16_ulp(as_f64(out), ref, 1.0)
+    assert bf16_out_ratio(as_f64(out), ref) <= 1.0
 
 
 def test_index_scores_deterministic(hcl):
