@@ -39,6 +39,7 @@ SIGNATURES = {
     "hcl_csa_topk": (I, [P, I, I, I, I, P, I, I, P, P, SZ, P, P]),
     "hcl_csa_sparse_attn_workspace_bytes": (SZ, [I, I, I, I, I]),
     "hcl_csa_sparse_attn": (I, [P, I, I, I, I, KVP, I, P, I, KVP, I, I, P, F, P, P, P, P, SZ, P, P]),
+    "hcl_csa_sparse_attn_noalloc": (I, [P, I, I, I, I, KVP, I, P, I, KVP, I, I, P, F, P, P, P, P, P]),
     "hcl_hca_dense_attn_workspace_bytes": (SZ, [I, I, I, I, I]),
     "hcl_hca_dense_attn": (I, [P, I, I, I, I, KVP, I, I, KVP, I, I, P, F, P, P, P, P, SZ, P, P]),
     "hcl_csa_decode_step_workspace_bytes": (SZ, [I, I, I, I, I, I, I, I]),

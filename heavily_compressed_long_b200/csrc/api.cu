@@ -263,6 +263,29 @@ hcl_status_t hcl_csa_sparse_attn(const void* q, int B, int Tq, int H, int d, con
                      lse, ws, ws_bytes, status, stream);
 }
 
+// The CSA attention with its split-KV partials in the library's fixed scratch array instead
+// of a caller workspace, for callers that may not allocate device memory (see hcl.h).
+hcl_status_t hcl_csa_sparse_attn_noalloc(const void* q, int B, int Tq, int H, int d,
+                                         const hcl_kv_t* kvc, int Nc, const int32_t* idx, int k,
+                                         const hcl_kv_t* raw, int L, int W,
+                                         const int32_t* q_pos, float scale, const float* sink,
+                                         void* out, float* lse, int32_t* status, void* stream) {
+  static_assert(HCL_NOALLOC_SCRATCH_BYTES == hcl::NOALLOC_SCRATCH_BYTES, "scratch size");
+  HCL_REQUIRE(B >= 0 && Tq >= 0 && H >= 1 && k >= 0 && W >= 0, "invalid size");
+  const size_t need = hcl::attn_workspace_bytes(0, B, Tq, H, k, W);
+  HCL_REQUIRE(need <= hcl::NOALLOC_SCRATCH_BYTES,
+              "hcl_csa_sparse_attn_noalloc: this problem needs %zu bytes of split-KV scratch, "
+              "more than the library's fixed %zu bytes; use hcl_csa_sparse_attn with a workspace",
+              need, hcl::NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  if (need > 0) {
+    hcl_status_t e = hcl::noalloc_scratch(&scratch);
+    if (e != HCL_OK) return e;
+  }
+  return attn_common(0, q, B, Tq, H, d, kvc, Nc, 1, idx, k, raw, L, W, q_pos, scale, sink, out,
+                     lse, scratch, need > 0 ? hcl::NOALLOC_SCRATCH_BYTES : 0, status, stream);
+}
+
 size_t hcl_hca_dense_attn_workspace_bytes(int B, int Tq, int H, int Nh, int W) {
   return hcl::attn_workspace_bytes(1, B, Tq, H, Nh, W);
 }

@@ -20,6 +20,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "hcl_common.cuh"
 #include "hcl_internal.h"
@@ -542,6 +543,35 @@ hcl_status_t launch_attn(const AttnArgs& a, void* ws, size_t ws_bytes, cudaStrea
   const long long threads = (long long)a.B * a.Tq * a.H * 32;
   attn_merge_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(p);
   return check_launch("attention merge");
+}
+
+// ---------------------------------------------------------------------------------------
+// Scratch for hcl_csa_sparse_attn_noalloc: a fixed device array in this module, so callers
+// that may not allocate device memory still get the split-KV attention.  Every GPU that loads
+// the library holds these NOALLOC_SCRATCH_BYTES until the process exits.  All calls share it:
+// calls that overlap on the GPU race on it.  Nothing in it has to start at zero -- each
+// partial (o, lse) slot the merge reads is written earlier in the same call.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+// Device address of the scratch array on the current device.  The array's name is only a
+// host-side stand-in in host code, so the address is looked up once per device (with that
+// device current) by cudaGetSymbolAddress and cached.
+hcl_status_t noalloc_scratch(void** ptr) {
+  static std::mutex mu;
+  static void* cache[64] = {};
+  int dev = 0;
+  hcl_status_t e = check_cuda(cudaGetDevice(&dev), "cudaGetDevice");
+  if (e != HCL_OK) return e;
+  if (dev < 0 || dev >= 64) return fail(HCL_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == nullptr) {
+    void* p = nullptr;
+    e = check_cuda(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
+    if (e != HCL_OK) return e;
+    cache[dev] = p;
+  }
+  *ptr = cache[dev];
+  return HCL_OK;
 }
 
 }  // namespace hcl

@@ -92,6 +92,11 @@ struct AttnArgs {
 size_t attn_workspace_bytes(int mode, int B, int Tq, int H, int n, int W);
 hcl_status_t launch_attn(const AttnArgs& a, void* ws, size_t ws_bytes, cudaStream_t st);
 
+// Fixed device scratch of hcl_csa_sparse_attn_noalloc (split-KV partials), and its device
+// address on the current device (looked up once per device).
+constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(16) << 20;
+hcl_status_t noalloc_scratch(void** ptr);
+
 hcl_status_t launch_selftest_wait(int32_t* status, int limit_us, cudaStream_t st);
 
 }  // namespace hcl

@@ -178,6 +178,30 @@ HCL_API hcl_status_t hcl_csa_sparse_attn(const void* q, int B, int Tq, int H, in
                                  int32_t* status, void* stream);
 
 /* ---------------------------------------------------------------------------------------
+ * hcl_csa_sparse_attn_noalloc -- the CSA attention above for callers that cannot allocate
+ * device memory.  (The paper has no counterpart; this is a deployment variant.)
+ * Some callers may not call cudaMalloc at all: serving runtimes that reserve the device's
+ * memory up front for their own pool and forbid allocation on the request path (cudaMalloc
+ * can synchronise the device and fail once the pool owns the memory), and plugin hosts that
+ * hand a kernel only its inputs and outputs.  This entry point takes the same arguments as
+ * hcl_csa_sparse_attn minus the workspace and allocates nothing: the split-KV partial results
+ * live in a fixed array inside the library, HCL_NOALLOC_SCRATCH_BYTES (16 MiB) on every GPU
+ * that loads the library, held until the process exits.  A problem whose partials need more
+ * (hcl_csa_sparse_attn_workspace_bytes() > 16 MiB) is rejected with HCL_ERR_INVALID_ARG and
+ * a message naming the limit.  The first call on a device looks the array's device address
+ * up (cudaGetSymbolAddress); make that first call before any stream capture.  All calls
+ * share the array and leave their partials in it; calls that overlap on the GPU (different
+ * streams, or threads) race on it, so serialise them.  Nothing in the array needs clearing:
+ * each call writes every slot it later reads.
+ */
+#define HCL_NOALLOC_SCRATCH_BYTES (16u << 20)
+HCL_API hcl_status_t hcl_csa_sparse_attn_noalloc(const void* q, int B, int Tq, int H, int d,
+                                         const hcl_kv_t* kvc, int Nc, const int32_t* idx, int k,
+                                         const hcl_kv_t* raw, int L, int W,
+                                         const int32_t* q_pos, float scale, const float* sink,
+                                         void* out, float* lse, int32_t* status, void* stream);
+
+/* ---------------------------------------------------------------------------------------
  * a7 -- HCA attention [Tripbot §3.2, §3.3; CSDN §1.2].  As a6 with J = { kvh entry i :
  * 0 <= i < Nh, mh*(i+1) - 1 <= p } followed by the window: dense, no selection.
  *   kvh: [B, cap, d] rows (cap >= Nh).  d == 128, 1 <= H <= 128.

@@ -1,0 +1,106 @@
+"""hcl_csa_sparse_attn_noalloc: the CSA attention for callers that may not allocate device
+memory (serving runtimes that own the device's memory pool and forbid cudaMalloc on the
+request path; plugin hosts that pass a kernel only its inputs and outputs).  Its split-KV
+partials live in a fixed 16 MiB array inside the library instead of a caller workspace.
+
+Checked through the C ABI against hcl_csa_sparse_attn (the workspace entry point) on two
+calls in a row with different inputs, within the attention tolerance the other tests use
+(5e-2 max abs for FP8 KV rows, 2e-2 for bf16); and a problem needing more scratch than the
+fixed array is refused with a message naming the limit.  This file is collected last so a
+run that stops at the first failure has already run every other test."""
+import ctypes
+import math
+
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+
+def _kv_struct(_lib, data, scale=None, rope=None):
+    fmt = _lib.HCL_FP8SPLIT if scale is not None else _lib.HCL_BF16
+    return _lib.hcl_kv_t(fmt, data.shape[1], data.data_ptr(),
+                         None if scale is None else scale.data_ptr(),
+                         None if rope is None else rope.data_ptr())
+
+
+def _problem(seed, B, H, Nc, k, W, fp8):
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    d, L = 128, 4 * Nc
+    q = torch.randn(B, 1, H, d, generator=g, device="cuda").to(torch.bfloat16)
+    idx = torch.stack([torch.randperm(Nc, generator=g, device="cuda")[:k].sort().values
+                       for _ in range(B)]).view(B, 1, k).to(torch.int32).contiguous()
+    pos = torch.full((B, 1), L - 1, dtype=torch.int32, device="cuda")
+    ent = torch.randn(B, Nc, d, generator=g, device="cuda").to(torch.bfloat16)
+    raw = torch.randn(B, W, d, generator=g, device="cuda").to(torch.bfloat16)
+    if not fp8:
+        return q, idx, pos, (ent,), (raw,), L
+    from heavily_compressed_long_b200 import api
+    out = []
+    for t in (ent, raw):
+        n = torch.empty(t.shape[0], t.shape[1], 64, dtype=torch.uint8, device="cuda")
+        s = torch.empty(t.shape[0], t.shape[1], dtype=torch.float32, device="cuda")
+        r = torch.empty(t.shape[0], t.shape[1], 64, dtype=torch.bfloat16, device="cuda")
+        api.hcl_quant_kv_fp8(t, n, s, r)
+        out.append((n, s, r))
+    return q, idx, pos, out[0], out[1], L
+
+
+def _call_both(hcl, _lib, L_, B, H, Nc, k, W, fp8, seed):
+    q, idx, pos, kvc_t, raw_t, L = _problem(seed, B, H, Nc, k, W, fp8)
+    kvc = _kv_struct(_lib, *kvc_t)
+    raw = _kv_struct(_lib, *raw_t)
+    scale = 1.0 / math.sqrt(128)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    # the workspace entry point
+    need = L_.hcl_csa_sparse_attn_workspace_bytes(B, 1, H, k, W)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device="cuda")
+    out_ref = torch.empty(B, 1, H, 128, dtype=torch.bfloat16, device="cuda")
+    lse_ref = torch.empty(B, 1, H, dtype=torch.float32, device="cuda")
+    _lib.check(L_.hcl_csa_sparse_attn(q.data_ptr(), B, 1, H, 128, ctypes.byref(kvc), Nc,
+                                      idx.data_ptr(), k, ctypes.byref(raw), L, W, pos.data_ptr(),
+                                      scale, None, out_ref.data_ptr(), lse_ref.data_ptr(),
+                                      ws.data_ptr(), ws.numel(), status.data_ptr(), stream))
+    # the allocation-free entry point
+    out = torch.empty_like(out_ref)
+    lse = torch.empty_like(lse_ref)
+    _lib.check(L_.hcl_csa_sparse_attn_noalloc(q.data_ptr(), B, 1, H, 128, ctypes.byref(kvc), Nc,
+                                              idx.data_ptr(), k, ctypes.byref(raw), L, W,
+                                              pos.data_ptr(), scale, None, out.data_ptr(),
+                                              lse.data_ptr(), status.data_ptr(), stream))
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    return need, out, out_ref, lse, lse_ref
+
+
+@pytest.mark.parametrize("fp8", [True, False])
+def test_noalloc_matches_workspace_entry_point_twice(hcl, fp8):
+    from heavily_compressed_long_b200 import _lib
+    L_ = _lib.lib()
+    tol = 5e-2 if fp8 else 2e-2
+    # 1M-context decode shape (8 sequences, 128 heads, top-1024 + 128 window): splits the KV
+    # list, so the partials go through the fixed scratch array; then a second, different call
+    for seed, (B, H, Nc, k, W) in [(11, (8, 128, 20000, 1024, 128)), (12, (3, 64, 9000, 512, 128))]:
+        need, out, out_ref, lse, lse_ref = _call_both(hcl, _lib, L_, B, H, Nc, k, W, fp8, seed)
+        assert 0 < need <= (16 << 20)               # the partials go through the scratch
+        assert (out.float() - out_ref.float()).abs().max().item() <= tol
+        assert (lse - lse_ref).abs().max().item() <= tol
+
+
+def test_noalloc_rejects_problems_beyond_the_fixed_scratch(hcl):
+    from heavily_compressed_long_b200 import _lib
+    L_ = _lib.lib()
+    B, H, k, W = 64, 128, 4096, 128
+    need = L_.hcl_csa_sparse_attn_workspace_bytes(B, 1, H, k, W)
+    assert need > (16 << 20)
+    fake = ctypes.c_void_p(1 << 30)
+    kv = _lib.hcl_kv_t(_lib.HCL_BF16, 8192, fake.value, None, None)
+    rc = L_.hcl_csa_sparse_attn_noalloc(fake, B, 1, H, 128, ctypes.byref(kv), 8192, fake, k,
+                                        ctypes.byref(kv), 32768, W, fake, 0.1, None, fake, None,
+                                        None, None)
+    assert rc == _lib.HCL_ERR_INVALID_ARG
+    msg = L_.hcl_last_error().decode()
+    assert "fixed" in msg and str(16 << 20) in msg
