@@ -268,13 +268,13 @@ def run_hcl(args, rank, world, local_rank):
     # eager warm-up (attributes, first-launch costs), then capture one graph per input set
     with torch.cuda.stream(stream):
         for p in sets:
-            p.step_parts(stream=stream)
+            p.step(stream=stream)
     torch.cuda.synchronize()
     graphs = []
     for p in sets:
         gr = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr, stream=stream):
-            p.step_parts(stream=stream)
+            p.step(stream=stream)
         graphs.append(gr)
     torch.cuda.synchronize()
 
@@ -462,14 +462,21 @@ def run_kernel_micro(args, local_rank):
         for _ in range(args.warmup):
             launch()
     torch.cuda.synchronize()
+    # the launches are replayed from a CUDA graph so host-side call overhead does not leave
+    # the device idle between them (device time per launch)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for _ in range(args.steps):
+            launch()
+    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     with torch.cuda.stream(stream):
-        for _ in range(args.steps):
-            launch()
+        graph.replay()
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
+    del graph
     hbm, src = peaks()
     nbytes = indexer_bytes_per_launch(cfg, B) if args.kernel == "indexer" else None
     line = {"kernel": args.kernel, "workload": f"{cfg.name} with B={B}", "ms_per_launch": ms,

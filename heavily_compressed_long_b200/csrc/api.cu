@@ -180,10 +180,13 @@ hcl_status_t hcl_quant_mxfp4(const void* x, int64_t rows, int cols, void* packed
   return launch_quant_mxfp4(x, rows, cols, packed, e8m0, as_stream(stream));
 }
 
-hcl_status_t hcl_csa_index_scores(int op_fmt, const void* qI, const void* qI_sf, const float* w,
-                                  const void* kI, const void* kI_sf, int B, int Tq, int HI,
-                                  int dI, int Nc, int kI_cap, const int32_t* q_pos, int m,
-                                  void* scores, int score_fmt, int32_t* status, void* stream) {
+// Validation + launch of the indexer.  qI_bf16 (MXFP4 keys only): the bf16 index query, to be
+// quantised inside the indexer instead of taking pre-quantised qI / qI_sf.
+static hcl_status_t index_scores_impl(int op_fmt, const void* qI, const void* qI_sf,
+                                      const void* qI_bf16, const float* w, const void* kI,
+                                      const void* kI_sf, int B, int Tq, int HI, int dI, int Nc,
+                                      int kI_cap, const int32_t* q_pos, int m, void* scores,
+                                      int score_fmt, int32_t* status, void* stream) {
   HCL_REQUIRE(op_fmt == HCL_BF16 || op_fmt == HCL_MXFP4, "op_fmt must be HCL_BF16 or HCL_MXFP4");
   HCL_REQUIRE(score_fmt == HCL_FP32 || score_fmt == HCL_BF16, "score_fmt must be HCL_FP32 or HCL_BF16");
   HCL_REQUIRE(B >= 0 && Tq >= 0 && Nc >= 0, "negative size");
@@ -193,12 +196,23 @@ hcl_status_t hcl_csa_index_scores(int op_fmt, const void* qI, const void* qI_sf,
   HCL_REQUIRE(Nc <= kI_cap, "Nc must be <= kI_cap");
   if (op_fmt == HCL_MXFP4) HCL_REQUIRE(kI_cap % 8 == 0, "MXFP4 keys need kI_cap % 8 == 0");
   if ((long long)B * Tq * Nc == 0) return HCL_OK;
-  HCL_REQUIRE(qI && w && kI && q_pos && scores, "NULL pointer");
-  HCL_REQUIRE(aligned16(qI) && aligned16(kI), "qI and kI must be 16-byte aligned");
-  if (op_fmt == HCL_MXFP4) HCL_REQUIRE(qI_sf && kI_sf && aligned16(kI_sf), "MXFP4 needs 16-byte aligned scale arrays");
+  const void* q_any = qI_bf16 ? qI_bf16 : qI;
+  HCL_REQUIRE(q_any && w && kI && q_pos && scores, "NULL pointer");
+  HCL_REQUIRE(aligned16(q_any) && aligned16(kI), "qI and kI must be 16-byte aligned");
+  if (op_fmt == HCL_MXFP4)
+    HCL_REQUIRE((qI_bf16 || qI_sf) && kI_sf && aligned16(kI_sf),
+                "MXFP4 needs 16-byte aligned scale arrays");
   IndexerArgs a{op_fmt, qI, qI_sf, w, kI, kI_sf, B, Tq, HI, dI, Nc, kI_cap, q_pos, m, scores,
                 score_fmt, status};
-  return launch_indexer(a, as_stream(stream));
+  return launch_indexer_q(a, qI_bf16, as_stream(stream));
+}
+
+hcl_status_t hcl_csa_index_scores(int op_fmt, const void* qI, const void* qI_sf, const float* w,
+                                  const void* kI, const void* kI_sf, int B, int Tq, int HI,
+                                  int dI, int Nc, int kI_cap, const int32_t* q_pos, int m,
+                                  void* scores, int score_fmt, int32_t* status, void* stream) {
+  return index_scores_impl(op_fmt, qI, qI_sf, nullptr, w, kI, kI_sf, B, Tq, HI, dI, Nc, kI_cap,
+                           q_pos, m, scores, score_fmt, status, stream);
 }
 
 size_t hcl_csa_topk_workspace_bytes(int B, int Tq, int Nc, int k, int score_fmt) {
@@ -342,18 +356,15 @@ hcl_status_t hcl_csa_decode_step(const void* q, const void* qI_bf16, const float
   HCL_REQUIRE(ws != nullptr && aligned16(ws) && ws_bytes >= l.total,
               "decode workspace too small: need %zu bytes", l.total);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
-  const void* qI = qI_bf16;
-  const void* qI_sf = nullptr;
   hcl_status_t e;
-  if (op_fmt == HCL_MXFP4) {
-    e = hcl_quant_mxfp4(qI_bf16, (int64_t)B * HI, dI, wsb + l.q_packed, wsb + l.q_sf, stream);
-    if (e != HCL_OK) return e;
-    qI = wsb + l.q_packed;
-    qI_sf = wsb + l.q_sf;
-  }
+  // MXFP4 keys: the bf16 index query is quantised inside the indexer (no separate launch)
   void* scores = wsb + l.scores;
-  e = hcl_csa_index_scores(op_fmt, qI, qI_sf, w, kI, kI_sf, B, 1, HI, dI, Nc, kI_cap, q_pos, m,
-                           scores, score_fmt, status, stream);
+  if (op_fmt == HCL_MXFP4)
+    e = index_scores_impl(op_fmt, nullptr, nullptr, qI_bf16, w, kI, kI_sf, B, 1, HI, dI, Nc,
+                          kI_cap, q_pos, m, scores, score_fmt, status, stream);
+  else
+    e = index_scores_impl(op_fmt, qI_bf16, nullptr, nullptr, w, kI, kI_sf, B, 1, HI, dI, Nc,
+                          kI_cap, q_pos, m, scores, score_fmt, status, stream);
   if (e != HCL_OK) return e;
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(wsb + l.idx);
   e = hcl_csa_topk(scores, score_fmt, B, 1, Nc, q_pos, m, k, idx, nullptr, 0, status, stream);

@@ -17,6 +17,7 @@
 // (mma.sync m16n8k16 bf16, fp32 accumulation) with an online softmax in registers.  With
 // several KV splits each block writes a normalised partial (o, lse) to the caller's
 // workspace and a merge kernel combines them by log-sum-exp.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -25,11 +26,14 @@
 #include "hcl_common.cuh"
 #include "hcl_internal.h"
 
+namespace cg = cooperative_groups;
+
 namespace hcl {
 namespace {
 
 constexpr int D = 128;
 constexpr int KVB = 64;
+constexpr int MAX_CLUSTER_ROWS = 16;   // largest cluster of splits merged through DSMEM
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
@@ -50,6 +54,8 @@ struct AttnParams {
   float* ws_o;
   float* ws_lse;
   int G, n_groups, splits, cps, rows_pad;
+  int cmerge;  // 1: the splits of a group form one cluster and merge through DSMEM
+  int hsplit;  // blocks sharing one group's (query, head) rows (cluster merge only)
   int32_t* status;
 };
 
@@ -100,17 +106,23 @@ struct RowSrc {
 template <int KVFMT, int MODE, int NW>
 __global__ void __launch_bounds__(NW * 32)
     attn_kernel(AttnParams p) {
+  pdl_enter();
   constexpr int NT = NW * 32;
   extern __shared__ __align__(128) uint8_t at_smem[];
   uint8_t* tiles = at_smem;                              // [2][64][256 B] bf16
   uint8_t* stage = at_smem + 2 * KVB * 256;              // fp8: [2][64][64 B] codes
   float* sscale = reinterpret_cast<float*>(stage + 2 * KVB * 64);  // fp8: [2][64]
   RowSrc* rsrc = reinterpret_cast<RowSrc*>(sscale + 2 * KVB);      // [2][64]
+  float* part = reinterpret_cast<float*>(rsrc + 2 * KVB);         // cluster merge: [16*NW][D]
+  float* plse = part + NW * 16 * D;                                // cluster merge: [16*NW]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int bid = blockIdx.x;
   const int split = bid % p.splits;
   bid /= p.splits;
+  const int hpart = bid % p.hsplit;   // which slice of the group's (query, head) rows
+  bid /= p.hsplit;
+  const int row_base = hpart * NW * 16;
   const int grp = bid % p.n_groups;
   const int b = bid / p.n_groups;
   const int t0 = grp * p.G;
@@ -147,7 +159,7 @@ __global__ void __launch_bounds__(NW * 32)
   bool row_ok[2];
 #pragma unroll
   for (int i = 0; i < 2; i++) {
-    const int r = warp * 16 + g + 8 * i;
+    const int r = row_base + warp * 16 + g + 8 * i;
     const int q = r / p.H;
     row_q[i] = q;
     row_h[i] = r % p.H;
@@ -258,21 +270,19 @@ __global__ void __launch_bounds__(NW * 32)
     }
   };
 
+  // Both buffers are filled up front (their index loads and row gathers overlap); afterwards
+  // each buffer is refilled with the chunk two ahead as soon as it has been consumed.
   if (c_begin < c_end) {
     resolve(c_begin, 0);
+    if (c_begin + 1 < c_end) resolve(c_begin + 1, 1);
     __syncthreads();
     issue(0);
+    if (c_begin + 1 < c_end) issue(1);
   }
   for (int c = c_begin; c < c_end; c++) {
     const int buf = (c - c_begin) & 1;
-    if (c + 1 < c_end) {
-      resolve(c + 1, buf ^ 1);
-      __syncthreads();
-      issue(buf ^ 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
+    if (c + 1 < c_end) cp_async_wait<1>();   // chunk c landed; chunk c+1 may be in flight
+    else cp_async_wait<0>();
     __syncthreads();
     if (KVFMT == HCL_FP8SPLIT) {
       widen(buf);
@@ -363,6 +373,11 @@ __global__ void __launch_bounds__(NW * 32)
       }
     }
     __syncthreads();
+    if (c + 2 < c_end) {   // this buffer is free: start the chunk two ahead
+      resolve(c + 2, buf);
+      __syncthreads();
+      issue(buf);
+    }
   }
 
   // row sums across the 4 threads of a row
@@ -395,20 +410,73 @@ __global__ void __launch_bounds__(NW * 32)
       }
       if (p.lse && tq == 0) p.lse[orow] = l2 > 0.f ? (m2 + log2f(l2)) * LN2 : -INFINITY;
     } else {
+      // normalised partial and its log2-domain LSE: to this block's shared memory (cluster
+      // merge) or to the caller's workspace (merge kernel)
       const float inv = l2 > 0.f ? 1.f / l2 : 0.f;
-      float* dst = p.ws_o + (item * p.rows_pad + r) * D;
+      float* dst = p.cmerge ? part + r * D : p.ws_o + (item * p.rows_pad + r) * D;
 #pragma unroll
       for (int n = 0; n < 16; n++) {
         const int col = n * 8 + tq * 2;
         *reinterpret_cast<float2*>(dst + col) = make_float2(o[n][2 * i] * inv, o[n][2 * i + 1] * inv);
       }
-      if (tq == 0) p.ws_lse[item * p.rows_pad + r] = l2 > 0.f ? m2 + log2f(l2) : -INFINITY;
+      const float ls = l2 > 0.f ? m2 + log2f(l2) : -INFINITY;
+      if (tq == 0) {
+        if (p.cmerge) plse[r] = ls;
+        else p.ws_lse[item * p.rows_pad + r] = ls;
+      }
     }
+  }
+  if (p.cmerge) {
+    // The splits of this query group are the blocks of one cluster: after the barrier, block
+    // `split` merges rows split, split + S, ... by log-sum-exp, reading every block's partial
+    // through distributed shared memory.
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    const int S = p.splits;
+    const int rows_valid = gq * p.H;
+    // r: row within this block's slice (index into every block's partials); rg: in the group
+    for (int r = split + S * warp; r < NW * 16; r += S * NW) {
+      const int rg = row_base + r;
+      if (rg >= rows_valid) break;
+      const float ls = lane < S ? cluster.map_shared_rank(plse, lane)[r] : -INFINITY;
+      float M = ls;
+#pragma unroll
+      for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
+      const int h = rg % p.H;
+      float s2 = -INFINITY;
+      if (p.sink) {
+        s2 = p.sink[h] * LOG2E;
+        M = fmaxf(M, s2);
+      }
+      const float wl = (ls == -INFINITY || M == -INFINITY) ? 0.f : exp2f(ls - M);
+      float den = wl;
+#pragma unroll
+      for (int o2 = 16; o2 > 0; o2 >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o2);
+      if (p.sink && M > -INFINITY) den += exp2f(s2 - M);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      // unrolled so every split's (remote) partial row is in flight at once
+#pragma unroll
+      for (int s = 0; s < MAX_CLUSTER_ROWS; s++) {
+        const float wgt = __shfl_sync(0xffffffffu, wl, s);
+        if (s < S && wgt != 0.f) {
+          const float4 v =
+              reinterpret_cast<const float4*>(cluster.map_shared_rank(part, s) + r * D)[lane];
+          acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
+        }
+      }
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+      const size_t orow = ((size_t)b * p.Tq + t0 + rg / p.H) * p.H + h;
+      reinterpret_cast<uint2*>(p.out + orow * D)[lane] =
+          make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
+      if (p.lse && lane == 0) p.lse[orow] = den > 0.f ? (M + log2f(den)) * LN2 : -INFINITY;
+    }
+    cluster.sync();  // no block leaves while another may still read its partial
   }
 }
 
 // Combine the KV splits of every (query, head) row by log-sum-exp (log2 domain partials).
 __global__ void attn_merge_kernel(AttnParams p) {
+  pdl_enter();
   const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const long long nrows = (long long)p.B * p.Tq * p.H;
@@ -420,8 +488,15 @@ __global__ void attn_merge_kernel(AttnParams p) {
   const int grp = t / p.G;
   const int r = (t - grp * p.G) * p.H + h;
   const size_t item0 = ((size_t)b * p.n_groups + grp) * p.splits;
+  // split LSEs: one per lane (32 at a time), reduced with shuffles -- no dependent loads
   float M = -INFINITY;
-  for (int s = 0; s < p.splits; s++) M = fmaxf(M, p.ws_lse[(item0 + s) * p.rows_pad + r]);
+  for (int s0 = 0; s0 < p.splits; s0 += 32) {
+    const int s = s0 + lane;
+    const float ls = s < p.splits ? p.ws_lse[(item0 + s) * p.rows_pad + r] : -INFINITY;
+    M = fmaxf(M, ls);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float s2 = -INFINITY;
   if (p.sink) {
     s2 = p.sink[h] * LOG2E;
@@ -430,13 +505,23 @@ __global__ void attn_merge_kernel(AttnParams p) {
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float den = 0.f;
   if (M > -INFINITY) {
-    for (int s = 0; s < p.splits; s++) {
-      const float ls = p.ws_lse[(item0 + s) * p.rows_pad + r];
-      if (ls == -INFINITY) continue;
-      const float wgt = exp2f(ls - M);
-      den += wgt;
-      const float4 v = reinterpret_cast<const float4*>(p.ws_o + ((item0 + s) * p.rows_pad + r) * D)[lane];
-      acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
+    for (int s0 = 0; s0 < p.splits; s0 += 32) {
+      const int s = s0 + lane;
+      const float ls = s < p.splits ? p.ws_lse[(item0 + s) * p.rows_pad + r] : -INFINITY;
+      const float wl = ls == -INFINITY ? 0.f : exp2f(ls - M);    // this lane's split weight
+      float dsum = wl;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+      den += dsum;
+      const int ns = min(32, p.splits - s0);
+#pragma unroll 4
+      for (int j = 0; j < ns; j++) {
+        const float wgt = __shfl_sync(0xffffffffu, wl, j);
+        if (wgt == 0.f) continue;
+        const float4 v = __ldg(reinterpret_cast<const float4*>(
+                                   p.ws_o + ((item0 + s0 + j) * p.rows_pad + r) * D) + lane);
+        acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
+      }
     }
     if (p.sink) den += exp2f(s2 - M);
   }
@@ -448,9 +533,15 @@ __global__ void attn_merge_kernel(AttnParams p) {
 }
 
 struct Plan {
-  int G, NW, n_groups, splits, cps, rows_pad, n_chunks_max;
+  int G, NW, n_groups, splits, cps, rows_pad, n_chunks_max, cmerge, hsplit;
 };
 
+constexpr int MAX_CLUSTER = 16;
+
+// Blocks: one per (sequence, query group, split).  Splits spread a long row list over the
+// SMs when there are few groups; when the splits of a group fit one cluster (<= 16 blocks)
+// and there are enough groups for ~half the SMs, they merge through DSMEM (no workspace, no
+// merge launch); otherwise through the caller's workspace and a merge kernel.
 Plan make_plan(int mode, int B, int Tq, int H, int list_max) {
   Plan pl;
   pl.G = mode == 0 ? 1 : std::max(1, 128 / H);
@@ -463,16 +554,59 @@ Plan make_plan(int mode, int B, int Tq, int H, int list_max) {
   const long long blocks = (long long)B * pl.n_groups;
   const long long target = 2LL * num_sms();
   int splits = (int)std::max(1LL, std::min<long long>(pl.n_chunks_max, (target + blocks - 1) / blocks));
+  pl.cmerge = 0;
+  if (splits > 1 && (splits <= MAX_CLUSTER || blocks * MAX_CLUSTER * 2 >= num_sms())) {
+    splits = std::min(splits, MAX_CLUSTER);
+    pl.cmerge = 1;
+  }
   pl.cps = (pl.n_chunks_max + splits - 1) / splits;
   pl.splits = (pl.n_chunks_max + pl.cps - 1) / pl.cps;
+  if (pl.splits == 1) pl.cmerge = 0;
+  // few clusters of 8-warp blocks leave SMs idle: halve the rows per block instead
+  pl.hsplit = 1;
+  if (pl.cmerge && pl.NW == 8 && blocks * pl.splits * 2 <= num_sms()) {
+    pl.hsplit = 2;
+    pl.NW = 4;
+    pl.rows_pad = 64;
+  }
   return pl;
 }
 
 template <int KVFMT, int MODE, int NW>
 hcl_status_t launch_t(const AttnParams& p, cudaStream_t st, long long grid) {
-  const size_t smem = 2 * KVB * 256 + 2 * KVB * 64 + 2 * KVB * 4 + 2 * KVB * sizeof(RowSrc);
-  attn_kernel<KVFMT, MODE, NW><<<(unsigned)grid, NW * 32, smem, st>>>(p);
-  return check_launch("attention");
+  auto kern = attn_kernel<KVFMT, MODE, NW>;
+  size_t smem = 2 * KVB * 256 + 2 * KVB * 64 + 2 * KVB * 4 + 2 * KVB * sizeof(RowSrc);
+  if (!p.cmerge) {
+    return check_cuda(launch_pdl(kern, dim3((unsigned)grid), dim3(NW * 32), smem, st, 1, p),
+                      "attention launch");
+  }
+  smem += (size_t)NW * 16 * (D + 1) * sizeof(float);
+  static bool attr_done = false;  // per instantiation, set once
+  if (!attr_done) {
+    hcl_status_t e = check_cuda(
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
+        "attention smem attribute");
+    if (e != HCL_OK) return e;
+    e = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1),
+                   "attention cluster attribute");
+    if (e != HCL_OK) return e;
+    attr_done = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(NW * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return check_cuda(cudaLaunchKernelEx(&cfg, kern, p), "attention launch");
 }
 
 template <int KVFMT, int MODE>
@@ -498,7 +632,7 @@ int list_max_for(int mode, int B, int Tq, int H, int n, int W) {
 
 size_t attn_workspace_bytes(int mode, int B, int Tq, int H, int n, int W) {
   const Plan pl = make_plan(mode, B, Tq, H, list_max_for(mode, B, Tq, H, n, W));
-  if (pl.splits <= 1) return 0;
+  if (pl.splits <= 1 || pl.cmerge) return 0;
   const size_t items = (size_t)B * pl.n_groups * pl.splits;
   return items * pl.rows_pad * (D + 1) * sizeof(float);
 }
@@ -520,10 +654,12 @@ hcl_status_t launch_attn(const AttnArgs& a, void* ws, size_t ws_bytes, cudaStrea
   p.lse = a.lse;
   p.G = pl.G; p.n_groups = pl.n_groups; p.splits = pl.splits; p.cps = pl.cps;
   p.rows_pad = pl.rows_pad;
+  p.cmerge = pl.cmerge;
+  p.hsplit = pl.hsplit;
   p.status = a.status;
   p.ws_o = nullptr;
   p.ws_lse = nullptr;
-  if (pl.splits > 1) {
+  if (pl.splits > 1 && !pl.cmerge) {
     const size_t items = (size_t)a.B * pl.n_groups * pl.splits;
     const size_t need = items * pl.rows_pad * (D + 1) * sizeof(float);
     if (ws == nullptr || ws_bytes < need)
@@ -532,17 +668,18 @@ hcl_status_t launch_attn(const AttnArgs& a, void* ws, size_t ws_bytes, cudaStrea
     p.ws_o = static_cast<float*>(ws);
     p.ws_lse = p.ws_o + items * pl.rows_pad * D;
   }
-  const long long grid = (long long)a.B * pl.n_groups * pl.splits;
+  const long long grid = (long long)a.B * pl.n_groups * pl.hsplit * pl.splits;
   hcl_status_t e;
   const bool fp8 = a.comp.fmt == HCL_FP8SPLIT;
   if (a.mode == 0) e = fp8 ? launch_nw<HCL_FP8SPLIT, 0>(p, pl.NW, st, grid)
                            : launch_nw<HCL_BF16, 0>(p, pl.NW, st, grid);
   else e = fp8 ? launch_nw<HCL_FP8SPLIT, 1>(p, pl.NW, st, grid)
                : launch_nw<HCL_BF16, 1>(p, pl.NW, st, grid);
-  if (e != HCL_OK || pl.splits == 1) return e;
+  if (e != HCL_OK || pl.splits == 1 || pl.cmerge) return e;
   const long long threads = (long long)a.B * a.Tq * a.H * 32;
-  attn_merge_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(p);
-  return check_launch("attention merge");
+  return check_cuda(launch_pdl(attn_merge_kernel, dim3((unsigned)((threads + 255) / 256)),
+                               dim3(256), 0, st, 1, p),
+                    "attention merge launch");
 }
 
 // ---------------------------------------------------------------------------------------

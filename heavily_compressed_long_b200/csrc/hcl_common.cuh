@@ -205,6 +205,22 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 
 // ---------------------------------------------------------------------------------------
+// Programmatic dependent launch.  Every libhcl kernel is launched so that it may start while
+// the previous kernel in the stream finishes; it calls pdl_wait() before touching global
+// memory (this returns once every prerequisite grid has completed and its writes are
+// visible), then pdl_trigger() so that its own successor may be scheduled.  Because a kernel
+// triggers only after its wait, ordering stays transitive along the stream.
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_enter() {
+  pdl_wait();
+  pdl_trigger();
+}
+
+// ---------------------------------------------------------------------------------------
 // cp.async (Ampere-style 16-byte async copies, used by the gather kernels)
 
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/hcl.h"
 
 namespace hcl {
@@ -17,6 +19,33 @@ hcl_status_t check_cuda(cudaError_t e, const char* what);
 hcl_status_t check_launch(const char* what);
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Launches `kern` with programmatic dependent launch allowed (the kernel must begin with
+// pdl_enter() / pdl_wait()), and as clusters of `cluster_x` blocks when cluster_x > 1.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  n++;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    n++;
+  }
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Number of SMs of the current device (cached per device).
 int num_sms();
@@ -56,6 +85,9 @@ struct IndexerArgs {
   int32_t* status;
 };
 hcl_status_t launch_indexer(const IndexerArgs& a, cudaStream_t st);
+// MXFP4 keys with the bf16 index query [B, Tq, HI, 64] quantised inside the indexer's prologue
+// (bit-identical to hcl_quant_mxfp4); a.qI / a.qI_sf are then unused.
+hcl_status_t launch_indexer_q(const IndexerArgs& a, const void* qI_bf16, cudaStream_t st);
 
 struct TopkArgs {
   const void* scores;

@@ -9,6 +9,7 @@
 
 #include "hcl_common.cuh"
 #include "hcl_internal.h"
+#include "mxfp4.cuh"
 
 namespace hcl {
 namespace {
@@ -56,24 +57,6 @@ __global__ void quant_kv_fp8_kernel(const __nv_bfloat16* __restrict__ kv, long l
   }
 }
 
-// E2M1 code of |q| by comparison against the midpoints of 0, .5, 1, 1.5, 2, 3, 4, 6; a value
-// exactly on a midpoint goes to the even code; beyond 6 saturates to code 7.
-__device__ __forceinline__ uint32_t e2m1_code(float q) {
-  float a = fabsf(q);
-  uint32_t c = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) +
-               (a >= 3.5f) + (a > 5.0f);
-  return c | (signbit(q) ? 8u : 0u);
-}
-
-// floor(log2(a)) for a finite a > 0 (normal or subnormal binary32).
-__device__ __forceinline__ int floor_log2(float a) {
-  uint32_t b = __float_as_uint(a);
-  int e = int(b >> 23);
-  if (e > 0) return e - 127;
-  uint32_t mant = b & 0x7FFFFFu;
-  return (31 - __clz(mant)) - 149;
-}
-
 // One thread per block of 32 values.
 __global__ void quant_mxfp4_kernel(const __nv_bfloat16* __restrict__ x, long long rows, int cols,
                                    uint8_t* __restrict__ packed, uint8_t* __restrict__ sf) {
@@ -86,25 +69,9 @@ __global__ void quant_mxfp4_kernel(const __nv_bfloat16* __restrict__ x, long lon
   uint4 v[4];
 #pragma unroll
   for (int i = 0; i < 4; i++) v[i] = __ldg(src + i);
-  const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(v);
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(bf2f(e[i])));
-  int code = 127;
-  if (amax > 0.f) {
-    code = floor_log2(amax) - 2 + 127;
-    code = code < 0 ? 0 : (code > 254 ? 254 : code);
-  }
-  const float X = code >= 1 ? __uint_as_float(uint32_t(code) << 23) : __uint_as_float(0x00400000u);
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 4; i++) {
-    uint32_t acc = 0;
-#pragma unroll
-    for (int k = 0; k < 8; k++) acc |= e2m1_code(__fdiv_rn(bf2f(e[i * 8 + k]), X)) << (4 * k);
-    w[i] = acc;
-  }
-  *reinterpret_cast<uint4*>(packed + r * (cols / 2) + j * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+  uint4 pk;
+  const int code = mxfp4_encode32(v, pk);
+  *reinterpret_cast<uint4*>(packed + r * (cols / 2) + j * 16) = pk;
   sf[r * nb + j] = uint8_t(code);
 }
 

@@ -39,9 +39,11 @@ class CsaDecode:
         self.step_ws = torch.empty(max(n, 16), dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
 
-    def launches_per_step(self):
-        n = 3 + (1 if self.op_fmt == HCL_MXFP4 else 0)
-        # the attention adds a merge launch when it splits the KV list
+    def launches_per_step(self, fused=True):
+        """Kernels one step launches: indexer, top-k, attention (+ split merge), and with
+        step_parts() a separate q_I quantisation for MXFP4 keys (fused into the indexer by
+        the C-ABI decode step)."""
+        n = 3 + (1 if (self.op_fmt == HCL_MXFP4 and not fused) else 0)
         need = api.csa_sparse_attn_workspace_bytes(self.B, 1, self.H, self.k, self.W)
         return n + (1 if need else 0)
 

@@ -192,6 +192,12 @@ def test_cfg4_csa_1m_mxfp4_fp8(hcl):
             assert np.abs(as_f64(pipe.out[sl]) - o_ref).max() <= 5e-2
             assert np.abs(as_f64(pipe.lse[sl]) - l_ref).max() <= 5e-2
     assert pipe.status.item() == 0
+    # the fused C-ABI decode step (q_I quantised inside the indexer) gives the same bits
+    out1, idx1, sc1 = pipe.out.clone(), pipe.idx.clone(), pipe.scores.clone()
+    pipe.step()
+    torch.cuda.synchronize()
+    assert torch.equal(idx1, pipe.idx) and torch.equal(out1, pipe.out)
+    assert pipe.status.item() == 0
 
 
 # =========================================================================================

@@ -216,6 +216,7 @@ def hcl_kv(data, scale=None, rope=None):
     (2, 1, 128, 9000, 1024, 128, True, False),  # cfg-4 shape, FP8 split rows
     (1, 3, 16, 700, 100, 37, False, False),     # ragged list, several queries
     (2, 2, 128, 3000, 64, 0, True, True),       # no window
+    (1, 1, 128, 9000, 4096, 128, True, True),   # long list: splits merged via the workspace
 ])
 def test_csa_attn(hcl, B, Tq, H, Nc, k, W, fp8, sink):
     d, L = 128, 4 * Nc + 11

@@ -81,9 +81,10 @@ def test_noalloc_matches_workspace_entry_point_twice(hcl, fp8):
     from heavily_compressed_long_b200 import _lib
     L_ = _lib.lib()
     tol = 5e-2 if fp8 else 2e-2
-    # 1M-context decode shape (8 sequences, 128 heads, top-1024 + 128 window): splits the KV
-    # list, so the partials go through the fixed scratch array; then a second, different call
-    for seed, (B, H, Nc, k, W) in [(11, (8, 128, 20000, 1024, 128)), (12, (3, 64, 9000, 512, 128))]:
+    # few sequences with long selections (top-4096 / top-2048 + 128 window): the KV list is
+    # split over more blocks than one cluster holds, so the split partials go through the
+    # fixed scratch array; then a second, different call
+    for seed, (B, H, Nc, k, W) in [(11, (1, 128, 20000, 4096, 128)), (12, (2, 64, 9000, 2048, 128))]:
         need, out, out_ref, lse, lse_ref = _call_both(hcl, _lib, L_, B, H, Nc, k, W, fp8, seed)
         assert 0 < need <= (16 << 20)               # the partials go through the scratch
         assert (out.float() - out_ref.float()).abs().max().item() <= tol
@@ -93,7 +94,7 @@ def test_noalloc_matches_workspace_entry_point_twice(hcl, fp8):
 def test_noalloc_rejects_problems_beyond_the_fixed_scratch(hcl):
     from heavily_compressed_long_b200 import _lib
     L_ = _lib.lib()
-    B, H, k, W = 64, 128, 4096, 128
+    B, H, k, W = 4, 128, 4096, 128          # 4 long selections: 264 split partials > 16 MiB
     need = L_.hcl_csa_sparse_attn_workspace_bytes(B, 1, H, k, W)
     assert need > (16 << 20)
     fake = ctypes.c_void_p(1 << 30)
