@@ -51,6 +51,23 @@ def bytes_per_query(cfg):
     return kI + rows + qo
 
 
+def rank_sequences(n_per_rank, rank):
+    """Global ids of the sequences rank `rank` decodes (weak scaling: a fixed number per
+    rank, disjoint across ranks, no data-path exchange)."""
+    return list(range(rank * n_per_rank, (rank + 1) * n_per_rank))
+
+
+def max_over_ranks(x, world, device):
+    """The slowest rank's value (a device-side all-reduce MAX); x itself when world == 1."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def indexer_bytes_per_launch(cfg, B):
     """Algorithmic bytes of one indexer launch: MXFP4 keys read + bf16 scores written."""
     return B * cfg.Nc * (cfg.dI // 2 + cfg.dI // 32 + 2)
@@ -283,11 +300,7 @@ def run_hcl(args, rank, world, local_rank):
             dist.barrier()
 
     def maxv(x):
-        if world > 1:
-            t = torch.tensor([x], dtype=torch.float64, device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            return float(t.item())
-        return x
+        return max_over_ranks(x, world, device)
 
     K, Wm = args.steps, args.warmup
     with torch.cuda.stream(stream):
@@ -431,12 +444,63 @@ def run_hcl(args, rank, world, local_rank):
     graphs.clear()
 
 
+def run_prefill_indexer(args, local_rank):
+    """The lightning indexer on the chunked-prefill shape (4096 new queries x 16 heads x 64
+    against 66560 compressed entries, bf16 operands, bf16 scores, entry-causal): a dense
+    tensor-core contraction.  Prints TFLOP/s against the measured bf16 dense peak."""
+    import torch
+    from heavily_compressed_long_b200 import api
+    from heavily_compressed_long_b200.api import HCL_BF16
+    from synth.configs import PAIR_PREFILL as cfg
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    g = torch.Generator(device=device)
+    g.manual_seed(cfg.seed)
+    Tq, HI, dI, Nc = cfg.Tq, cfg.HI, cfg.dI, cfg.Nc
+    qI = torch.randn(1, Tq, HI, dI, generator=g, device=device).to(torch.bfloat16)
+    kI = torch.randn(1, Nc, dI, generator=g, device=device).to(torch.bfloat16)
+    w = torch.rand(1, Tq, HI, generator=g, device=device)
+    pos = torch.arange(cfg.first_pos, cfg.first_pos + Tq, dtype=torch.int32,
+                       device=device).unsqueeze(0).contiguous()
+    scores = torch.empty(1, Tq, Nc, dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.Stream(device)
+
+    def launch():
+        api.hcl_csa_index_scores(HCL_BF16, qI, w, kI, pos, cfg.m, scores, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, args.warmup)):
+            launch()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            launch()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = 2.0 * Tq * HI * dI * Nc                # dense contraction incl. masked tiles
+    peak = 1662.1
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            peak = float(json.load(f)["bf16_tflops"])
+    print(json.dumps({"kernel": "indexer_prefill", "workload": f"{cfg.name} indexer",
+                      "ms_per_launch": ms, "flops_per_launch": flops,
+                      "achieved_tflops": flops / ms / 1e9, "peak_tflops": peak,
+                      "frac": flops / ms / 1e9 / peak,
+                      "scores_bytes": Tq * Nc * 2}), flush=True)
+
+
 def run_kernel_micro(args, local_rank):
     """One kernel alone on one input set of `--batch` sequences (indexer: larger than L2),
     for profiling: times back-to-back launches with CUDA events and prints a JSON line."""
     import torch
     from heavily_compressed_long_b200 import api
     from heavily_compressed_long_b200.api import HCL_MXFP4
+    if args.kernel == "indexer_prefill":
+        return run_prefill_indexer(args, local_rank)
     cfg = workload()
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
@@ -489,7 +553,7 @@ def run_kernel_micro(args, local_rank):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kernel", default=None, choices=["indexer", "topk", "attn"],
+    ap.add_argument("--kernel", default=None, choices=["indexer", "topk", "attn", "indexer_prefill"],
                     help="time one kernel alone (profiling aid) instead of the whole step")
     ap.add_argument("--batch", type=int, default=16, help="sequences for --kernel")
     ap.add_argument("--gpus", type=int, default=1)
