@@ -96,6 +96,17 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
 }
 
 // 3-D tiled TMA load into shared memory, completing on `bar` (transaction bytes).
+// Untiled bulk copy global -> this CTA's shared memory, completing `bytes` on `bar`.  Both
+// addresses 16-byte aligned, bytes a multiple of 16 (no multicast).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int x,
                                             int y, int z) {
   asm volatile(

@@ -41,12 +41,14 @@ constexpr int HP = 16;     // heads per query, padded = UMMA N per query
 struct IdxParams {
   const uint8_t* qI;          // pre-quantised / bf16 operand rows
   const uint8_t* qI_sf;       // MXFP4 scales of qI (when pre-quantised)
+  const uint8_t* kI_sf;       // MXFP4 key scales [B, cap, 2] (packed-row decode path)
   const __nv_bfloat16* qI_bf16;  // bf16 index queries to quantise in-kernel (MXFP4 keys), or null
   const float* w;
   const int32_t* q_pos;
   void* scores;
   int score_fmt;
-  int B, Tq, HI, Nc, m;
+  int B, Tq, HI, Nc, m, cap;
+  int vec_ok;                 // Nc % 4 == 0 and scores 16-byte aligned: vector score stores
   int n_qt, n_kt, n_kc, kt_per_chunk;
   int32_t* status;
   long long limit;
@@ -58,21 +60,29 @@ __host__ __device__ constexpr uint32_t tmem_cols_for(uint32_t need) {
   return c;
 }
 
+// Operand kinds: 0 = bf16 (one key per 128-byte K-row, SW128); 1 = MXFP4 (one key per 32-byte
+// K-row, SW32); 2 = MXFP4 packed rows (decode): four consecutive keys form one 128-byte K-row
+// (K = 256 = 4 keys x 64), loaded with SW128 as one 16 KB box of 512 keys.  The query operand
+// is block-diagonal (row (j, h) holds q_h in K-segment j), so UMMA k-step j (K = 64) yields
+// key 4r+j against every head in accumulator columns j*16 .. j*16+15 of lane r.
 template <int KIND, int QT, int TPS, int STAGES, int NACC, int EPI>
 struct IdxLayout {
-  static constexpr int N = QT * HP;
-  static constexpr int ROWB = KIND == 0 ? 128 : 32;       // bytes per K-row of an operand
+  static constexpr int KPR = KIND == 2 ? 4 : 1;            // keys per operand row
+  static constexpr int TK = KEYS * KPR;                     // keys per tile
+  static constexpr int N = QT * HP * KPR;
+  static constexpr int ROWB = KIND == 1 ? 32 : 128;         // bytes per K-row of an operand
   static constexpr int A_TILE = KEYS * ROWB;
   static constexpr int A_STAGE = TPS * A_TILE;
-  static constexpr int SF_TILE = KIND == 1 ? KEYS * 2 : 0;
+  static constexpr int SF_TILE = KIND == 0 ? 0 : TK * 2;    // raw E8M0 bytes per tile
+  static constexpr int SF_BLOCKS = KIND == 0 ? 0 : KPR;     // 512-byte tcgen05.cp blocks per tile
   static constexpr int BOX_ROWS = (TPS * KEYS) < 256 ? (TPS * KEYS) : 256;
   static constexpr int B_BYTES = ((N * ROWB + 1023) / 1024) * 1024;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
   static constexpr int OFF_SFRAW = OFF_B + B_BYTES;
-  static constexpr int OFF_SFEXP = OFF_SFRAW + (KIND == 1 ? STAGES * TPS * 256 : 0);
-  static constexpr int OFF_SFB = OFF_SFEXP + (KIND == 1 ? STAGES * TPS * 512 : 0);
-  static constexpr int OFF_W = OFF_SFB + (KIND == 1 ? 512 : 0);
+  static constexpr int OFF_SFEXP = OFF_SFRAW + STAGES * TPS * SF_TILE;
+  static constexpr int OFF_SFB = OFF_SFEXP + STAGES * TPS * SF_BLOCKS * 512;
+  static constexpr int OFF_W = OFF_SFB + (KIND != 0 ? 512 : 0);
   static constexpr int OFF_NVIS = OFF_W + QT * HP * 4;
   static constexpr int OFF_BAR = ((OFF_NVIS + QT * 4 + 7) / 8) * 8;
   static constexpr int NBAR = 2 * STAGES + 2 * NACC + 1;
@@ -80,18 +90,16 @@ struct IdxLayout {
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int NT = 64 + 32 * EPI;
   static constexpr int ACC_COLS = NACC * TPS * N;
-  static constexpr uint32_t TMEM_COLS = tmem_cols_for(ACC_COLS + (KIND == 1 ? 4 * TPS + 4 : 0));
+  static constexpr uint32_t TMEM_COLS =
+      tmem_cols_for(ACC_COLS + (KIND != 0 ? 4 * SF_BLOCKS * TPS + 4 : 0));
 };
-
-__device__ __forceinline__ void epi_bar(int nthreads) {
-  asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
-}
 
 template <int KIND, int QT, int TPS, int STAGES, int NACC, int EPI>
 __global__ void __launch_bounds__(64 + 32 * EPI, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmSF,
                    IdxParams p) {
   using Lay = IdxLayout<KIND, QT, TPS, STAGES, NACC, EPI>;
+  static_assert(KIND != 2 || (QT == 1 && EPI == 4), "packed rows: one query, 128 epilogue threads");
   constexpr int N = Lay::N;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -139,8 +147,12 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
     prefetch_tmap(&tmK);
     if (KIND == 1) prefetch_tmap(&tmSF);
   }
+  __syncthreads();  // barriers initialised, TMEM allocated
+  tc_fence_after();
   // everything above touches no global memory; the rest may read what the previous kernel
-  // in the stream wrote
+  // in the stream wrote.  The producer starts streaming keys as soon as the epilogue warps
+  // have issued their few prologue loads (named barrier 3); the MMA warp waits (named
+  // barrier 2) until those warps have built the query operand.
   pdl_enter();
   if (threadIdx.x >= 64) {
     // Query operand tile (K-major, swizzled as the UMMA descriptor expects), head weights,
@@ -157,61 +169,154 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
               p.qI + (((size_t)b * p.Tq + t) * p.HI + h) * 128 + c * 16));
         *reinterpret_cast<uint4*>(sB + (n >> 3) * 1024 + (n & 7) * 128 + ((c ^ (n & 7)) << 4)) = v;
       }
-    } else {
-      for (int u = et; u < 128; u += ne) reinterpret_cast<uint32_t*>(sSFB)[u] = 0u;
-      epi_bar(ne);
-      for (int n = et; n < N; n += ne) {
-        const int q = n / HP, h = n % HP, t = t0 + q;
-        uint4 pk0 = make_uint4(0, 0, 0, 0), pk1 = pk0;
-        uint32_t s0 = 0, s1 = 0;
-        if (t < p.Tq && h < p.HI) {
-          const size_t row = ((size_t)b * p.Tq + t) * p.HI + h;
-          if (p.qI_bf16 != nullptr) {
-            const uint4* src = reinterpret_cast<const uint4*>(p.qI_bf16 + row * 64);
-            uint4 v0[4], v1[4];
+    } else if (KIND == 2) {
+      // Packed rows, one query (EPI = 4: 128 threads).  Thread et holds 8 values of head
+      // h = et/8, scale block half = (et/4)&1, part c = et&3; the four threads of a block share
+      // its amax by shuffles (max is exact, so the scale matches hcl_quant_mxfp4 bit for bit).
+      // Its packed word goes to rows (seg, h) of the block-diagonal operand, chunk 2*seg+half.
+      // All global loads are issued before the producer may start (named barrier 3).
+      const int h = et >> 3, half = (et >> 2) & 1, c = et & 3;
+      const bool valid = t0 < p.Tq && h < p.HI;
+      const bool quant = p.qI_bf16 != nullptr;
+      const size_t row = ((size_t)b * p.Tq + t0) * p.HI + h;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      uint32_t word = 0;
+      int code = 0;
+      if (valid) {
+        if (quant) {
+          v = __ldg(reinterpret_cast<const uint4*>(p.qI_bf16 + row * 64 + half * 32 + c * 8));
+        } else {
+          word = __ldg(reinterpret_cast<const uint32_t*>(p.qI + row * 32 + half * 16 + c * 4));
+          code = __ldg(p.qI_sf + row * 2 + half);
+        }
+      }
+      float wv = 0.f;
+      if (et < HP && t0 < p.Tq && et < p.HI) wv = __ldg(p.w + ((size_t)b * p.Tq + t0) * p.HI + et);
+      int pos = -1;
+      if (et == 0 && t0 < p.Tq) pos = __ldg(p.q_pos + (size_t)b * p.Tq + t0);
+      asm volatile("bar.arrive 3, %0;" ::"r"(32 + 32 * EPI) : "memory");
+      if (quant) {
+        float amax = bf16x8_amax(v);
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        code = mxfp4_scale_code(amax);
+        word = mxfp4_encode8(v, e8m0_value(code));
+        if (!valid) { word = 0; code = 0; }
+      }
+      const int code_other = __shfl_xor_sync(0xffffffffu, code, 4);
 #pragma unroll
-            for (int i = 0; i < 4; i++) { v0[i] = __ldg(src + i); v1[i] = __ldg(src + 4 + i); }
-            s0 = (uint32_t)mxfp4_encode32(v0, pk0);
-            s1 = (uint32_t)mxfp4_encode32(v1, pk1);
-          } else {
-            const uint4* src = reinterpret_cast<const uint4*>(p.qI + row * 32);
-            pk0 = __ldg(src);
-            pk1 = __ldg(src + 1);
-            s0 = p.qI_sf[row * 2];
-            s1 = p.qI_sf[row * 2 + 1];
+      for (int seg = 0; seg < 4; seg++) {
+        const int n = seg * HP + h;
+        const int cc = 2 * seg + half;
+        *reinterpret_cast<uint32_t*>(sB + (n >> 3) * 1024 + (n & 7) * 128 +
+                                     ((cc ^ (n & 7)) << 4) + c * 4) = word;
+      }
+      // the six zero chunks of each of the 64 rows
+      for (int it = et; it < N * 6; it += ne) {
+        const int n = it / 6, j = it % 6, seg = n / HP;
+        const int cc = j < 2 * seg ? j : j + 2;
+        *reinterpret_cast<uint4*>(sB + (n >> 3) * 1024 + (n & 7) * 128 + ((cc ^ (n & 7)) << 4)) =
+            make_uint4(0, 0, 0, 0);
+      }
+      // query scales: word (n%32)*4 + n/32 of row n = (seg, h) holds (s_half0, s_half1);
+      // the words of rows 64..127 are zero
+      if (half == 0 && c == 0) {
+#pragma unroll
+        for (int seg = 0; seg < 4; seg++) {
+          const int n = seg * HP + h;
+          reinterpret_cast<uint32_t*>(sSFB)[(n & 31) * 4 + (n >> 5)] =
+              uint32_t(code) | (uint32_t(code_other) << 8);
+        }
+      }
+      if (et < 64) reinterpret_cast<uint32_t*>(sSFB)[4 * (et >> 1) + 2 + (et & 1)] = 0u;
+      if (et < HP) sW[et] = wv;
+      if (et == 0) sNvis[0] = pos < 0 ? 0 : min(p.Nc, (pos + 1) / p.m);
+    } else {
+      // Thread et owns the query-scale word et of the tcgen05.cp block (line et/4, word et%4),
+      // i.e. operand row n = et/4 + 32*(et%4), and builds that row.  Every global load is
+      // issued before the producer may start (named barrier 3), so these few loads are not
+      // queued behind the key stream.
+      const int n = (et >> 2) + 32 * (et & 3);
+      const int seg = KIND == 2 ? n / HP : 0;   // packed rows: K-segment of this B row
+      const int q = KIND == 2 ? 0 : n / HP, h = n % HP, t = t0 + q;
+      const bool valid = et < 128 && n < N && t < p.Tq && h < p.HI;
+      const bool quant = p.qI_bf16 != nullptr;
+      const size_t row = ((size_t)b * p.Tq + t) * p.HI + h;
+      uint4 v0[4], v1[4];
+      uint4 pk0 = make_uint4(0, 0, 0, 0), pk1 = pk0;
+      uint32_t s0 = 0, s1 = 0;
+      if (valid) {
+        if (quant) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.qI_bf16 + row * 64);
+#pragma unroll
+          for (int i = 0; i < 4; i++) { v0[i] = __ldg(src + i); v1[i] = __ldg(src + 4 + i); }
+        } else {
+          const uint4* src = reinterpret_cast<const uint4*>(p.qI + row * 32);
+          pk0 = __ldg(src);
+          pk1 = __ldg(src + 1);
+          s0 = p.qI_sf[row * 2];
+          s1 = p.qI_sf[row * 2 + 1];
+        }
+      }
+      float wv = 0.f;
+      if (et < QT * HP) {
+        const int qw = et / HP, hw = et % HP, tw = t0 + qw;
+        if (tw < p.Tq && hw < p.HI) wv = __ldg(p.w + ((size_t)b * p.Tq + tw) * p.HI + hw);
+      }
+      int pos = -1;
+      if (et < QT && t0 + et < p.Tq) pos = __ldg(p.q_pos + (size_t)b * p.Tq + t0 + et);
+      asm volatile("bar.arrive 3, %0;" ::"r"(32 + 32 * EPI) : "memory");
+      if (valid && quant) {
+        s0 = (uint32_t)mxfp4_encode32(v0, pk0);
+        s1 = (uint32_t)mxfp4_encode32(v1, pk1);
+      }
+      if (et < 128 && n < N) {
+        if (KIND == 1) {
+          const int sw = (n & 7) >> 2;
+          uint8_t* rowp = sB + (n >> 3) * 256 + (n & 7) * 32;
+          *reinterpret_cast<uint4*>(rowp + ((0 ^ sw) << 4)) = pk0;
+          *reinterpret_cast<uint4*>(rowp + ((1 ^ sw) << 4)) = pk1;
+        } else {
+          // 128-byte SW128 row: q_h's 32 bytes in chunks 2*seg, 2*seg+1, zeros elsewhere
+          uint8_t* rowp = sB + (n >> 3) * 1024 + (n & 7) * 128;
+#pragma unroll
+          for (int c = 0; c < 8; c++) {
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(rowp + ((c ^ (n & 7)) << 4)) =
+                c == 2 * seg ? pk0 : (c == 2 * seg + 1 ? pk1 : z);
           }
         }
-        const int sw = (n & 7) >> 2;
-        uint8_t* rowp = sB + (n >> 3) * 256 + (n & 7) * 32;
-        *reinterpret_cast<uint4*>(rowp + ((0 ^ sw) << 4)) = pk0;
-        *reinterpret_cast<uint4*>(rowp + ((1 ^ sw) << 4)) = pk1;
-        sSFB[(n & 31) * 16 + (n >> 5) * 4 + 0] = uint8_t(s0);
-        sSFB[(n & 31) * 16 + (n >> 5) * 4 + 1] = uint8_t(s1);
       }
+      if (et < 128) reinterpret_cast<uint32_t*>(sSFB)[et] = s0 | (s1 << 8);
+      if (et < QT * HP) sW[et] = wv;
+      if (et < QT) sNvis[et] = pos < 0 ? 0 : min(p.Nc, (pos + 1) / p.m);
     }
-    for (int u = et; u < QT * HP; u += ne) {
-      const int q = u / HP, h = u % HP, t = t0 + q;
-      sW[u] = (t < p.Tq && h < p.HI) ? p.w[((size_t)b * p.Tq + t) * p.HI + h] : 0.f;
-    }
-    for (int q = et; q < QT; q += ne) {
-      const int t = t0 + q;
-      int nv = 0;
-      if (t < p.Tq) {
-        const int pos = p.q_pos[(size_t)b * p.Tq + t];
-        nv = pos < 0 ? 0 : min(p.Nc, (pos + 1) / p.m);
+    if (KIND == 0) {
+      for (int u = et; u < QT * HP; u += ne) {
+        const int q = u / HP, h = u % HP, t = t0 + q;
+        sW[u] = (t < p.Tq && h < p.HI) ? p.w[((size_t)b * p.Tq + t) * p.HI + h] : 0.f;
       }
-      sNvis[q] = nv;
+      for (int q = et; q < QT; q += ne) {
+        const int t = t0 + q;
+        int nv = 0;
+        if (t < p.Tq) {
+          const int pos = p.q_pos[(size_t)b * p.Tq + t];
+          nv = pos < 0 ? 0 : min(p.Nc, (pos + 1) / p.m);
+        }
+        sNvis[q] = nv;
+      }
+      asm volatile("bar.arrive 3, %0;" ::"r"(32 + 32 * EPI) : "memory");
     }
     fence_proxy_async_smem();
   }
-  __syncthreads();
-  tc_fence_after();
+  if (warp >= 1) asm volatile("bar.sync 2, %0;" ::"r"(32 + 32 * EPI) : "memory");
   const uint32_t tbase = *sTmem;
   const uint32_t sfa_t = tbase + Lay::ACC_COLS;
-  const uint32_t sfb_t = tbase + Lay::ACC_COLS + 4 * TPS;
+  const uint32_t sfb_t = tbase + Lay::ACC_COLS + 4 * Lay::SF_BLOCKS * TPS;
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
+    asm volatile("bar.sync 3, %0;" ::"r"(32 + 32 * EPI) : "memory");  // prologue loads issued
     if (lane == 0) {
       int issued = 0;
       for (int i = 0; i < nstages; i++) {
@@ -222,13 +327,21 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
           report(p.status, HCL_ERR_TIMEOUT);
           break;
         }
-        mbar_arrive_expect_tx(&full[s], TPS * (Lay::A_TILE + Lay::SF_TILE));
-        const int row0 = (kt0 + i * TPS) * KEYS;
+        const int key0 = (kt0 + i * TPS) * Lay::TK;
+        // packed rows: the stage's key scales are one contiguous run, copied untiled (its
+        // length stops at the buffer's capacity; cap % 8 == 0 keeps it a multiple of 16 B)
+        const uint32_t sf_bytes =
+            KIND == 2 ? 2u * (uint32_t)min(TPS * Lay::TK, p.cap - key0) : TPS * Lay::SF_TILE;
+        mbar_arrive_expect_tx(&full[s], TPS * Lay::A_TILE + sf_bytes);
 #pragma unroll
         for (int r = 0; r < TPS * KEYS; r += Lay::BOX_ROWS)
-          tma_load_3d(sA + s * Lay::A_STAGE + r * Lay::ROWB, &tmK, &full[s], 0, row0 + r, b);
+          tma_load_3d(sA + s * Lay::A_STAGE + r * Lay::ROWB, &tmK, &full[s], 0,
+                      key0 / Lay::KPR + r, b);
         if (KIND == 1)
-          tma_load_3d(sSFraw + s * TPS * 256, &tmSF, &full[s], 0, row0 / 8, b);
+          tma_load_3d(sSFraw + s * TPS * 256, &tmSF, &full[s], 0, key0 / 8, b);
+        if (KIND == 2)
+          bulk_load(sSFraw + s * TPS * Lay::SF_TILE, p.kI_sf + ((size_t)b * p.cap + key0) * 2,
+                    sf_bytes, &full[s]);
         issued++;
       }
       // Drain: every issued copy has landed before the block may exit.
@@ -237,7 +350,7 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
-    if (KIND == 1 && lane == 0)
+    if (KIND != 0 && lane == 0)
       tmem_cp_32x128b_x4(sfb_t, make_sdesc(smem_u32(sSFB), 16, 128, SMEM_SWIZZLE_NONE));
     for (int i = 0; i < nstages; i++) {
       const int s = i % STAGES;
@@ -262,6 +375,23 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
         fence_proxy_async_smem();
         __syncwarp();
       }
+      if (KIND == 2) {
+        // packed rows: row r of a tile holds keys 4r..4r+3; k-step j needs key 4r+j's two
+        // scales at (line r%32, word r/32) -- raw u16 index 4r+j
+#pragma unroll
+        for (int t = 0; t < TPS; t++) {
+          const uint16_t* raw =
+              reinterpret_cast<const uint16_t*>(sSFraw + (s * TPS + t) * Lay::SF_TILE);
+#pragma unroll
+          for (int j = 0; j < 4; j++) {
+            const uint4 v = make_uint4(raw[4 * lane + j], raw[4 * (lane + 32) + j],
+                                       raw[4 * (lane + 64) + j], raw[4 * (lane + 96) + j]);
+            *reinterpret_cast<uint4*>(sSFexp + ((s * TPS + t) * 4 + j) * 512 + lane * 16) = v;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
       if (lane == 0) {
         const uint32_t aB = smem_u32(sB);
 #pragma unroll
@@ -274,6 +404,16 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
               umma_bf16(d, make_sdesc(aA + 32 * k, 16, 1024, SMEM_SWIZZLE_128B),
                         make_sdesc(aB + 32 * k, 16, 1024, SMEM_SWIZZLE_128B), idesc_bf16(KEYS, N),
                         k > 0 ? 1u : 0u);
+          } else if (KIND == 2) {
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+              tmem_cp_32x128b_x4(sfa_t + 4 * (t * 4 + j),
+                                 make_sdesc(smem_u32(sSFexp + ((s * TPS + t) * 4 + j) * 512), 16,
+                                            128, SMEM_SWIZZLE_NONE));
+              umma_mxf4(d, make_sdesc(aA + 32 * j, 16, 1024, SMEM_SWIZZLE_128B),
+                        make_sdesc(aB + 32 * j, 16, 1024, SMEM_SWIZZLE_128B), idesc_mxf4(KEYS, N),
+                        sfa_t + 4 * (t * 4 + j), sfb_t, j > 0 ? 1u : 0u);
+            }
           } else {
             tmem_cp_32x128b_x4(sfa_t + 4 * t, make_sdesc(smem_u32(sSFexp + (s * TPS + t) * 512),
                                                          16, 128, SMEM_SWIZZLE_NONE));
@@ -314,6 +454,42 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
       }
     };
 
+    // packed rows (one query): lane r of the tile holds keys 4r..4r+3, stored as one vector
+    auto emit4 = [&](int tile, const uint32_t (&r)[4][16]) {
+      const int key = tile * Lay::TK + (quarter * 32 + lane) * 4;
+      const int nv = sNvis[0];
+      float v[4];
+#pragma unroll
+      for (int j = 0; j < 4; j++) {
+        float s = 0.f;
+#pragma unroll
+        for (int h = 0; h < HP; h++) s = fmaf(sW[h], fmaxf(__uint_as_float(r[j][h]), 0.f), s);
+        v[j] = key + j < nv ? s : -INFINITY;
+      }
+      if (t0 >= p.Tq) return;
+      const size_t o = ((size_t)b * p.Tq + t0) * p.Nc + key;
+      if (p.vec_ok && key + 3 < p.Nc) {
+        if (p.score_fmt == HCL_FP32) {
+          *reinterpret_cast<float4*>(static_cast<float*>(p.scores) + o) =
+              make_float4(v[0], v[1], v[2], v[3]);
+        } else {
+          __nv_bfloat162 lo = __floats2bfloat162_rn(v[0], v[1]);
+          __nv_bfloat162 hi = __floats2bfloat162_rn(v[2], v[3]);
+          uint2 u;
+          u.x = *reinterpret_cast<uint32_t*>(&lo);
+          u.y = *reinterpret_cast<uint32_t*>(&hi);
+          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.scores) + o) = u;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+          if (key + j >= p.Nc) break;
+          if (p.score_fmt == HCL_FP32) static_cast<float*>(p.scores)[o + j] = v[j];
+          else static_cast<__nv_bfloat16*>(p.scores)[o + j] = __float2bfloat16_rn(v[j]);
+        }
+      }
+    };
+
     for (int i = 0; i < nstages; i++) {
       const int a = i % NACC;
       bool ok = mbar_wait(&accf[a], (i / NACC) & 1, p.limit, sAbort);
@@ -325,7 +501,18 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
       tc_fence_after();
       const int tile0 = kt0 + i * TPS;
       const uint32_t tacc = tbase + lane_off + a * TPS * N;
-      if (ALL_AT_ONCE) {
+      if constexpr (KIND == 2) {
+        uint32_t r[TPS][4][16];
+#pragma unroll
+        for (int t = 0; t < TPS; t++)
+#pragma unroll
+          for (int j = 0; j < 4; j++) tmem_ld16(tacc + t * N + j * HP, r[t][j]);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&acce[a]);
+#pragma unroll
+        for (int t = 0; t < TPS; t++) emit4(tile0 + t, r[t]);
+      } else if (ALL_AT_ONCE) {
         uint32_t r[TPS * QPER][16];
 #pragma unroll
         for (int t = 0; t < TPS; t++)
@@ -401,13 +588,17 @@ hcl_status_t run(const IndexerArgs& a, const void* qI_bf16, const CUtensorMap& t
   p.q_pos = a.q_pos;
   p.scores = a.scores;
   p.score_fmt = a.score_fmt;
-  p.B = a.B; p.Tq = a.Tq; p.HI = a.HI; p.Nc = a.Nc; p.m = a.m;
+  p.kI_sf = static_cast<const uint8_t*>(a.kI_sf);
+  p.B = a.B; p.Tq = a.Tq; p.HI = a.HI; p.Nc = a.Nc; p.m = a.m; p.cap = a.kI_cap;
+  p.vec_ok = (a.Nc % 4 == 0) && (reinterpret_cast<uintptr_t>(a.scores) % 16 == 0);
   p.n_qt = (a.Tq + QT - 1) / QT;
-  p.n_kt = (a.Nc + KEYS - 1) / KEYS;
+  p.n_kt = (a.Nc + Lay::TK - 1) / Lay::TK;
+  // key chunks per (sequence, query tile): as many as fill the co-resident slots without
+  // spilling into a second wave
   const long long target = (long long)num_sms() * per_sm;
   const long long base = (long long)a.B * p.n_qt;
   const int n_stages_total = (p.n_kt + TPS - 1) / TPS;
-  int n_kc = (int)std::max(1LL, std::min<long long>(n_stages_total, (target + base - 1) / base));
+  int n_kc = (int)std::max(1LL, std::min<long long>(n_stages_total, target / base));
   const int st_per_chunk = (n_stages_total + n_kc - 1) / n_kc;
   p.kt_per_chunk = st_per_chunk * TPS;
   p.n_kc = (p.n_kt + p.kt_per_chunk - 1) / p.kt_per_chunk;
@@ -437,7 +628,7 @@ hcl_status_t make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, 
 }
 
 // Decode configurations: stage = TPS tiles; box rows = min(256, TPS*128).
-constexpr int DEC_BF16_TPS = 2, DEC_MX_TPS = 4;
+constexpr int DEC_BF16_TPS = 2;
 
 }  // namespace
 
@@ -456,15 +647,20 @@ hcl_status_t launch_indexer_q(const IndexerArgs& a, const void* qI_bf16, cudaStr
     if (decode) return run<0, 1, DEC_BF16_TPS, 3, 3, 4>(a, nullptr, tmK, tmSF, st, 0);
     return run<0, 16, 1, 4, 2, 8>(a, nullptr, tmK, tmSF, st, 120 * 1024);
   }
-  const int tps = decode ? DEC_MX_TPS : 1;
-  const cuuint32_t rows = std::min(256, tps * KEYS);
+  if (decode) {
+    // packed rows: [B, cap/4, 128 B] (four keys per row), 16 KB boxes with SW128; the key
+    // scales are fetched by untiled bulk copies
+    e = make_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.kI, 128, a.kI_cap / 4, a.B, 128,
+                 (cuuint64_t)a.kI_cap * 32, 128, KEYS, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != HCL_OK) return e;
+    return run<2, 1, 1, 5, 3, 4>(a, qI_bf16, tmK, tmSF, st, 0);
+  }
   e = make_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.kI, 32, a.kI_cap, a.B, 32,
-               (cuuint64_t)a.kI_cap * 32, 32, rows, CU_TENSOR_MAP_SWIZZLE_32B);
+               (cuuint64_t)a.kI_cap * 32, 32, KEYS, CU_TENSOR_MAP_SWIZZLE_32B);
   if (e != HCL_OK) return e;
   e = make_map(&tmSF, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.kI_sf, 16, a.kI_cap / 8, a.B, 16,
-               (cuuint64_t)a.kI_cap * 2, 16, tps * KEYS / 8, CU_TENSOR_MAP_SWIZZLE_NONE);
+               (cuuint64_t)a.kI_cap * 2, 16, KEYS / 8, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (e != HCL_OK) return e;
-  if (decode) return run<1, 1, DEC_MX_TPS, 5, 3, 4>(a, qI_bf16, tmK, tmSF, st, 0);
   return run<1, 8, 1, 8, 2, 8>(a, qI_bf16, tmK, tmSF, st, 120 * 1024);
 }
 

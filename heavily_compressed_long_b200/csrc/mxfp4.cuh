@@ -40,25 +40,35 @@ __device__ __forceinline__ float e8m0_value(int code) {
   return code >= 1 ? __uint_as_float(uint32_t(code) << 23) : __uint_as_float(0x00400000u);
 }
 
-// Encode 32 bf16 values (four 16-byte vectors) into 16 packed bytes (element 2j in the low
-// nibble of byte j) and return the E8M0 scale code.
-__device__ __forceinline__ int mxfp4_encode32(const uint4 (&v)[4], uint4& packed) {
-  const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(v);
+// Largest magnitude among 8 bf16 values (one 16-byte vector).
+__device__ __forceinline__ float bf16x8_amax(const uint4& v) {
+  const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&v);
   float amax = 0.f;
 #pragma unroll
-  for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(__bfloat162float(e[i])));
+  for (int i = 0; i < 8; i++) amax = fmaxf(amax, fabsf(__bfloat162float(e[i])));
+  return amax;
+}
+
+// E2M1 codes of 8 bf16 values divided by the block scale X, packed into 4 bytes (element 2j in
+// the low nibble of byte j).
+__device__ __forceinline__ uint32_t mxfp4_encode8(const uint4& v, float X) {
+  const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&v);
+  uint32_t acc = 0;
+#pragma unroll
+  for (int k = 0; k < 8; k++) acc |= e2m1_code(__fdiv_rn(__bfloat162float(e[k]), X)) << (4 * k);
+  return acc;
+}
+
+// Encode 32 bf16 values (four 16-byte vectors) into 16 packed bytes and return the E8M0 scale
+// code.
+__device__ __forceinline__ int mxfp4_encode32(const uint4 (&v)[4], uint4& packed) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; i++) amax = fmaxf(amax, bf16x8_amax(v[i]));
   const int code = mxfp4_scale_code(amax);
   const float X = e8m0_value(code);
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 4; i++) {
-    uint32_t acc = 0;
-#pragma unroll
-    for (int k = 0; k < 8; k++)
-      acc |= e2m1_code(__fdiv_rn(__bfloat162float(e[i * 8 + k]), X)) << (4 * k);
-    w[i] = acc;
-  }
-  packed = make_uint4(w[0], w[1], w[2], w[3]);
+  packed = make_uint4(mxfp4_encode8(v[0], X), mxfp4_encode8(v[1], X), mxfp4_encode8(v[2], X),
+                      mxfp4_encode8(v[3], X));
   return code;
 }
 

@@ -89,8 +89,10 @@ def test_host_validation_without_device(libhcl):
 
 def test_workspace_queries(libhcl):
     L = libhcl.lib()
-    # decode at B = 8, H = 128, k + W = 1152 splits the KV list -> needs a workspace
-    assert L.hcl_csa_sparse_attn_workspace_bytes(8, 1, 128, 1024, 128) > 0
+    # decode at B = 8, H = 128, k + W = 1152: the splits merge inside a cluster, no workspace
+    assert L.hcl_csa_sparse_attn_workspace_bytes(8, 1, 128, 1024, 128) == 0
+    # one sequence with k = 4096 splits into more pieces than a cluster holds -> workspace
+    assert L.hcl_csa_sparse_attn_workspace_bytes(1, 1, 128, 4096, 128) > 0
     # a prefill chunk with many queries does not split
     assert L.hcl_csa_sparse_attn_workspace_bytes(1, 4096, 64, 1024, 128) == 0
     assert L.hcl_csa_decode_step_workspace_bytes(8, 128, 16, 262144, 1024, 128,

@@ -140,6 +140,38 @@ def test_index_scores_mxfp4_bf16_scores(hcl, B, Tq, Nc, cap):
     assert bf16_out_ratio(as_f64(out), ref) <= 1.0
 
 
+@pytest.mark.parametrize("B,Nc,cap,nvis,fp32", [
+    (3, 5000, 5008, (5000, 1237, 0), True),     # vector fp32 stores, visibility inside a row
+    (3, 5000, 5008, (4999, 1, 2050), False),    # vector bf16 stores, ragged visibility
+    (1, 70001, 70008, (70001,), False),         # many blocks per row, scalar tail stores
+    (2, 512, 512, (512, 511), True),            # exactly one 512-key tile
+    (1, 3, 8, (3,), True),                      # fewer keys than one packed row group
+])
+def test_index_scores_mxfp4_decode(hcl, B, Nc, cap, nvis, fp32):
+    """Decode (one query) with MXFP4 operands: keys packed four to a 128-byte row.  Covers
+    partial tiles, rows whose visible prefix ends inside a four-key group and both score
+    formats (the in-kernel quantisation of bf16 index queries is covered by the fused decode
+    step's bitwise comparison with the separate calls)."""
+    HI = 16
+    qb, kb = rbf16(B, 1, HI, 64), rbf16(B, cap, 64)
+    qp, qs = oracle.quant_mxfp4(qb)
+    kp, ks = oracle.quant_mxfp4(kb)
+    w = torch.from_numpy(RNG.random((B, 1, HI)).astype(np.float32))
+    pos = torch.tensor([[4 * v - 1 if v > 0 else 2] for v in nvis], dtype=torch.int32)
+    ref = oracle.index_scores(oracle.FMT_MXFP4, qp, w, kp[:, :Nc], pos, 4, qI_sf=qs,
+                              kI_sf=ks[:, :Nc], bf16_scores=not fp32)
+    t = lambda a: cuda(torch.from_numpy(np.ascontiguousarray(a)))
+    dt = torch.float32 if fp32 else torch.bfloat16
+    out = torch.empty(B, 1, Nc, dtype=dt, device="cuda")
+    hcl.hcl_csa_index_scores(hcl.HCL_MXFP4, t(qp), cuda(w), t(kp), cuda(pos), 4, out, Nc=Nc,
+                             qI_sf=t(qs), kI_sf=t(ks))
+    torch.cuda.synchronize()
+    if fp32:
+        assert rel_rowwise(as_f64(out), ref) <= 1e-3
+    else:
+        assert bf16_out_ratio(as_f64(out), ref) <= 1.0
+
+
 def test_index_scores_deterministic(hcl):
     qI, kI = cuda(rbf16(2, 1, 16, 64)), cuda(rbf16(2, 5000, 64))
     w = cuda(torch.rand(2, 1, 16))
