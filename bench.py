@@ -68,6 +68,21 @@ def max_over_ranks(x, world, device):
     return float(t.item())
 
 
+# DRAM traffic of one indexer launch as measured once with ncu (dram__bytes_read.sum +
+# dram__bytes_write.sum over 16 sequences; profiles/indexer_mxfp4_decode_B16.md), per sequence.
+# It is reported only while the indexer source is the one that was profiled.
+INDEXER_TRAFFIC = {"source_sha256_16": "b2c672a212a5db8a",
+                   "bytes_per_seq": (142.650624e6 + 6.076160e6) / 16}
+
+
+def indexer_traffic(B):
+    import hashlib
+    src = os.path.join(ROOT, "heavily_compressed_long_b200", "csrc", "indexer.cu")
+    with open(src, "rb") as fh:
+        h = hashlib.sha256(fh.read()).hexdigest()[:16]
+    return B * INDEXER_TRAFFIC["bytes_per_seq"] if h == INDEXER_TRAFFIC["source_sha256_16"] else None
+
+
 def indexer_bytes_per_launch(cfg, B):
     """Algorithmic bytes of one indexer launch: MXFP4 keys read + bf16 scores written."""
     return B * cfg.Nc * (cfg.dI // 2 + cfg.dI // 32 + 2)
@@ -428,7 +443,8 @@ def run_hcl(args, rank, world, local_rank):
                          "achieved": idx_gbs, "peak": hbm, "unit": "GB/s", "frac": idx_gbs / hbm,
                          "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback 6.65 TB/s",
                          "bytes_per_launch": idx_bytes, "ms_per_launch": idx_ms,
-                         "share_of_step": idx_ms / step_ms, "traffic": None},
+                         "share_of_step": idx_ms / step_ms, "traffic": indexer_traffic(B),
+                         "traffic_source": "ncu capture at 16 sequences, scaled per sequence"},
             "e2e": {"value": q_per_step / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                     "path": "hcl_csa_decode_step (C ABI) + pinned H2D/D2H copies, no graph"},

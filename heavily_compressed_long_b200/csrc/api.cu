@@ -186,7 +186,8 @@ static hcl_status_t index_scores_impl(int op_fmt, const void* qI, const void* qI
                                       const void* qI_bf16, const float* w, const void* kI,
                                       const void* kI_sf, int B, int Tq, int HI, int dI, int Nc,
                                       int kI_cap, const int32_t* q_pos, int m, void* scores,
-                                      int score_fmt, int32_t* status, void* stream) {
+                                      int score_fmt, int32_t* status, void* stream,
+                                      uint16_t* gmax = nullptr) {
   HCL_REQUIRE(op_fmt == HCL_BF16 || op_fmt == HCL_MXFP4, "op_fmt must be HCL_BF16 or HCL_MXFP4");
   HCL_REQUIRE(score_fmt == HCL_FP32 || score_fmt == HCL_BF16, "score_fmt must be HCL_FP32 or HCL_BF16");
   HCL_REQUIRE(B >= 0 && Tq >= 0 && Nc >= 0, "negative size");
@@ -203,7 +204,7 @@ static hcl_status_t index_scores_impl(int op_fmt, const void* qI, const void* qI
     HCL_REQUIRE((qI_bf16 || qI_sf) && kI_sf && aligned16(kI_sf),
                 "MXFP4 needs 16-byte aligned scale arrays");
   IndexerArgs a{op_fmt, qI, qI_sf, w, kI, kI_sf, B, Tq, HI, dI, Nc, kI_cap, q_pos, m, scores,
-                score_fmt, status};
+                score_fmt, status, gmax};
   return launch_indexer_q(a, qI_bf16, as_stream(stream));
 }
 
@@ -219,9 +220,9 @@ size_t hcl_csa_topk_workspace_bytes(int B, int Tq, int Nc, int k, int score_fmt)
   return topk_workspace_bytes(B, Tq, Nc, k, score_fmt);
 }
 
-hcl_status_t hcl_csa_topk(const void* scores, int score_fmt, int B, int Tq, int Nc,
-                          const int32_t* q_pos, int m, int k, int32_t* idx, void* ws,
-                          size_t ws_bytes, int32_t* status, void* stream) {
+static hcl_status_t topk_common(const void* scores, int score_fmt, int B, int Tq, int Nc,
+                               const int32_t* q_pos, int m, int k, int32_t* idx, void* ws,
+                               size_t ws_bytes, int32_t* status, void* stream, int prewait) {
   HCL_REQUIRE(score_fmt == HCL_FP32 || score_fmt == HCL_BF16, "score_fmt must be HCL_FP32 or HCL_BF16");
   HCL_REQUIRE(B >= 0 && Tq >= 0 && Nc >= 0, "negative size");
   HCL_REQUIRE(k >= 1 && k <= 4096, "k must be in [1, 4096]");
@@ -230,15 +231,23 @@ hcl_status_t hcl_csa_topk(const void* scores, int score_fmt, int B, int Tq, int 
   HCL_REQUIRE(ws_bytes >= topk_workspace_bytes(B, Tq, Nc, k, score_fmt), "workspace too small");
   if ((long long)B * Tq == 0) return HCL_OK;
   HCL_REQUIRE(q_pos && idx && (scores || Nc == 0), "NULL pointer");
-  TopkArgs a{scores, score_fmt, B, Tq, Nc, q_pos, m, k, idx, status};
+  TopkArgs a{scores, score_fmt, B, Tq, Nc, q_pos, m, k, idx, status, prewait};
   return launch_topk(a, ws, ws_bytes, as_stream(stream));
+}
+
+hcl_status_t hcl_csa_topk(const void* scores, int score_fmt, int B, int Tq, int Nc,
+                          const int32_t* q_pos, int m, int k, int32_t* idx, void* ws,
+                          size_t ws_bytes, int32_t* status, void* stream) {
+  return topk_common(scores, score_fmt, B, Tq, Nc, q_pos, m, k, idx, ws, ws_bytes, status, stream,
+                     0);
 }
 
 static hcl_status_t attn_common(int mode, const void* q, int B, int Tq, int H, int d,
                                 const hcl_kv_t* comp, int n_comp, int mh, const int32_t* idx,
                                 int k, const hcl_kv_t* raw, int L, int W, const int32_t* q_pos,
                                 float scale, const float* sink, void* out, float* lse, void* ws,
-                                size_t ws_bytes, int32_t* status, void* stream) {
+                                size_t ws_bytes, int32_t* status, void* stream,
+                                int prewait = 0) {
   HCL_REQUIRE(B >= 0 && Tq >= 0, "negative size");
   if (d != 128) return fail(HCL_ERR_UNSUPPORTED, "only d == 128 is supported (got %d)", d);
   HCL_REQUIRE(H >= 1 && H <= 128, "H must be in [1, 128]");
@@ -260,7 +269,7 @@ static hcl_status_t attn_common(int mode, const void* q, int B, int Tq, int H, i
   a.mode = mode; a.q = q; a.B = B; a.Tq = Tq; a.H = H; a.d = d;
   a.comp = *comp; a.n_comp = n_comp; a.mh = mh; a.idx = idx; a.k = k;
   a.raw = *raw; a.L = L; a.W = W; a.q_pos = q_pos; a.scale = scale; a.sink = sink;
-  a.out = out; a.lse = lse; a.status = status;
+  a.out = out; a.lse = lse; a.status = status; a.prewait = prewait;
   return launch_attn(a, ws, ws_bytes, as_stream(stream));
 }
 
@@ -318,8 +327,14 @@ hcl_status_t hcl_hca_dense_attn(const void* q, int B, int Tq, int H, int d, cons
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct DecodeWs {
-  size_t q_packed, q_sf, scores, idx, attn, total;
+  size_t q_packed, q_sf, scores, gmax, idx, attn, total;
 };
+
+// The decode step selects from the indexer's per-16-entry maxima when the keys are MXFP4 and
+// the scores bf16 (the indexer's packed-row decode path writes them).
+static bool decode_uses_gmax(int op_fmt, int score_fmt, int Nc) {
+  return op_fmt == HCL_MXFP4 && score_fmt == HCL_BF16 && hcl::topk_gmax_supported(Nc);
+}
 
 static DecodeWs decode_ws_layout(int B, int H, int HI, int Nc, int k, int W, int op_fmt,
                                  int score_fmt, int dI) {
@@ -331,6 +346,8 @@ static DecodeWs decode_ws_layout(int B, int H, int HI, int Nc, int k, int W, int
   if (op_fmt == HCL_MXFP4) off += align256((size_t)B * HI * dI / 32);
   l.scores = off;
   off += align256((size_t)B * Nc * (score_fmt == HCL_BF16 ? 2 : 4));
+  l.gmax = off;
+  if (decode_uses_gmax(op_fmt, score_fmt, Nc)) off += align256((size_t)B * hcl::gmax_row_stride(Nc) * 2);
   l.idx = off;
   off += align256((size_t)B * k * 4);
   l.attn = off;
@@ -359,18 +376,29 @@ hcl_status_t hcl_csa_decode_step(const void* q, const void* qI_bf16, const float
   hcl_status_t e;
   // MXFP4 keys: the bf16 index query is quantised inside the indexer (no separate launch)
   void* scores = wsb + l.scores;
+  uint16_t* gmax =
+      decode_uses_gmax(op_fmt, score_fmt, Nc) ? reinterpret_cast<uint16_t*>(wsb + l.gmax) : nullptr;
   if (op_fmt == HCL_MXFP4)
     e = index_scores_impl(op_fmt, nullptr, nullptr, qI_bf16, w, kI, kI_sf, B, 1, HI, dI, Nc,
-                          kI_cap, q_pos, m, scores, score_fmt, status, stream);
+                          kI_cap, q_pos, m, scores, score_fmt, status, stream, gmax);
   else
     e = index_scores_impl(op_fmt, qI_bf16, nullptr, nullptr, w, kI, kI_sf, B, 1, HI, dI, Nc,
                           kI_cap, q_pos, m, scores, score_fmt, status, stream);
   if (e != HCL_OK) return e;
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(wsb + l.idx);
-  e = hcl_csa_topk(scores, score_fmt, B, 1, Nc, q_pos, m, k, idx, nullptr, 0, status, stream);
+  // the top-k's predecessor is the indexer above, which does not write q_pos
+  if (gmax != nullptr) {
+    HCL_REQUIRE(k >= 1 && k <= 4096, "k must be in [1, 4096]");
+    TopkArgs ta{scores, score_fmt, B, 1, Nc, q_pos, m, k, idx, status, 1};
+    e = launch_topk_gmax(ta, gmax, as_stream(stream));
+  } else {
+    e = topk_common(scores, score_fmt, B, 1, Nc, q_pos, m, k, idx, nullptr, 0, status, stream, 1);
+  }
   if (e != HCL_OK) return e;
-  return hcl_csa_sparse_attn(q, B, 1, H, d, kvc, Nc, idx, k, raw, L, W, q_pos, scale, sink, out,
-                             lse, wsb + l.attn, ws_bytes - l.attn, status, stream);
+  // the attention's predecessor is the top-k above, which writes neither q nor q_pos: the
+  // attention may load its queries before waiting for it
+  return attn_common(0, q, B, 1, H, d, kvc, Nc, 1, idx, k, raw, L, W, q_pos, scale, sink, out,
+                     lse, wsb + l.attn, ws_bytes - l.attn, status, stream, 1);
 }
 
 hcl_status_t hcl_selftest_bounded_wait(int32_t* status, int limit_us, void* stream) {

@@ -56,6 +56,8 @@ struct AttnParams {
   int G, n_groups, splits, cps, rows_pad;
   int cmerge;  // 1: the splits of a group form one cluster and merge through DSMEM
   int hsplit;  // blocks sharing one group's (query, head) rows (cluster merge only)
+  int prewait; // 1: q, q_pos are not written by the previous kernel in the stream, so they may
+               // be read before waiting for it (set only inside the fused decode step)
   int32_t* status;
 };
 
@@ -106,15 +108,20 @@ struct RowSrc {
 template <int KVFMT, int MODE, int NW>
 __global__ void __launch_bounds__(NW * 32)
     attn_kernel(AttnParams p) {
-  pdl_enter();
+  // Wait for the previous kernel before the first global read -- or, when q and q_pos are
+  // known not to come from it, only before reading the selected indices.
+  if (!p.prewait) pdl_enter();
   constexpr int NT = NW * 32;
   extern __shared__ __align__(128) uint8_t at_smem[];
   uint8_t* tiles = at_smem;                              // [2][64][256 B] bf16
   uint8_t* stage = at_smem + 2 * KVB * 256;              // fp8: [2][64][64 B] codes
   float* sscale = reinterpret_cast<float*>(stage + 2 * KVB * 64);  // fp8: [2][64]
   RowSrc* rsrc = reinterpret_cast<RowSrc*>(sscale + 2 * KVB);      // [2][64]
-  float* part = reinterpret_cast<float*>(rsrc + 2 * KVB);         // cluster merge: [16*NW][D]
-  float* plse = part + NW * 16 * D;                                // cluster merge: [16*NW]
+  // cluster merge: the partials of the rows this block merges, pushed here by every split:
+  // recv[slot][split][D] and recv_lse[slot][split], slot = row / splits
+  float* recv = reinterpret_cast<float*>(rsrc + 2 * KVB);
+  const int rpo = (NW * 16 + p.splits - 1) / p.splits;            // rows merged per block
+  float* recv_lse = recv + (size_t)rpo * p.splits * D;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int bid = blockIdx.x;
@@ -186,14 +193,16 @@ __global__ void __launch_bounds__(NW * 32)
     }
   }
 
+  if (p.prewait) pdl_enter();
+
   float o[16][4];
 #pragma unroll
   for (int n = 0; n < 16; n++) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
   float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
 
   // ---- gather of one chunk into buffer `buf` ----
-  auto resolve = [&](int chunk, int buf) {
-    for (int j = tid; j < KVB; j += NT) {
+  auto resolve_row = [&](int chunk, int buf, int j) {
+    {
       const int e = chunk * KVB + j;
       RowSrc rs{-1, 0};
       if (e < n_a) {
@@ -214,6 +223,9 @@ __global__ void __launch_bounds__(NW * 32)
       }
       rsrc[buf * KVB + j] = rs;
     }
+  };
+  auto resolve = [&](int chunk, int buf) {
+    for (int j = tid; j < KVB; j += NT) resolve_row(chunk, buf, j);
   };
   auto issue = [&](int buf) {
     uint8_t* tile = tiles + buf * KVB * 256;
@@ -273,8 +285,16 @@ __global__ void __launch_bounds__(NW * 32)
   // Both buffers are filled up front (their index loads and row gathers overlap); afterwards
   // each buffer is refilled with the chunk two ahead as soon as it has been consumed.
   if (c_begin < c_end) {
-    resolve(c_begin, 0);
-    if (c_begin + 1 < c_end) resolve(c_begin + 1, 1);
+    if (NT >= 2 * KVB) {
+      // both chunks' index loads in flight together: threads [0, 64) and [64, 128)
+      if (tid < 2 * KVB) {
+        const int ch = c_begin + tid / KVB;
+        if (ch < c_end) resolve_row(ch, tid / KVB, tid % KVB);
+      }
+    } else {
+      resolve(c_begin, 0);
+      if (c_begin + 1 < c_end) resolve(c_begin + 1, 1);
+    }
     __syncthreads();
     issue(0);
     if (c_begin + 1 < c_end) issue(1);
@@ -410,35 +430,52 @@ __global__ void __launch_bounds__(NW * 32)
       }
       if (p.lse && tq == 0) p.lse[orow] = l2 > 0.f ? (m2 + log2f(l2)) * LN2 : -INFINITY;
     } else {
-      // normalised partial and its log2-domain LSE: to this block's shared memory (cluster
-      // merge) or to the caller's workspace (merge kernel)
+      // normalised partial and its log2-domain LSE: pushed into the shared memory of the
+      // block that merges row r (cluster merge: block r % splits, slot r / splits), or to
+      // the caller's workspace (merge kernel)
       const float inv = l2 > 0.f ? 1.f / l2 : 0.f;
-      float* dst = p.cmerge ? part + r * D : p.ws_o + (item * p.rows_pad + r) * D;
+      const float ls = l2 > 0.f ? m2 + log2f(l2) : -INFINITY;
+      float* dst;
+      float* dst_lse;
+      if (p.cmerge) {
+        cg::cluster_group cluster = cg::this_cluster();
+        const int owner = r % p.splits, slot = r / p.splits;
+        dst = cluster.map_shared_rank(recv, owner) + ((size_t)slot * p.splits + split) * D;
+        dst_lse = cluster.map_shared_rank(recv_lse, owner) + slot * p.splits + split;
+      } else {
+        dst = p.ws_o + (item * p.rows_pad + r) * D;
+        dst_lse = p.ws_lse + item * p.rows_pad + r;
+      }
+      // 16-byte stores: the two threads of a column pair swap halves, and for column block n
+      // the even (n even) or odd (n odd) thread of each pair writes four columns.  Both
+      // threads of a pair hold the same row, so they skip rows together.
+      const unsigned pm = 3u << (lane & ~1);
 #pragma unroll
       for (int n = 0; n < 16; n++) {
-        const int col = n * 8 + tq * 2;
-        *reinterpret_cast<float2*>(dst + col) = make_float2(o[n][2 * i] * inv, o[n][2 * i + 1] * inv);
+        const float mx = o[n][2 * i] * inv, my = o[n][2 * i + 1] * inv;
+        const float ox = __shfl_xor_sync(pm, mx, 1), oy = __shfl_xor_sync(pm, my, 1);
+        if ((tq & 1) == (n & 1)) {
+          const float4 v = (tq & 1) ? make_float4(ox, oy, mx, my) : make_float4(mx, my, ox, oy);
+          *reinterpret_cast<float4*>(dst + n * 8 + (tq >> 1) * 4) = v;
+        }
       }
-      const float ls = l2 > 0.f ? m2 + log2f(l2) : -INFINITY;
-      if (tq == 0) {
-        if (p.cmerge) plse[r] = ls;
-        else p.ws_lse[item * p.rows_pad + r] = ls;
-      }
+      if (tq == 0) *dst_lse = ls;
     }
   }
   if (p.cmerge) {
-    // The splits of this query group are the blocks of one cluster: after the barrier, block
-    // `split` merges rows split, split + S, ... by log-sum-exp, reading every block's partial
-    // through distributed shared memory.
+    // The splits of this query group are the blocks of one cluster.  Every block has pushed
+    // its partials to the merging blocks; after the barrier (which makes those remote stores
+    // visible) block `split` merges rows split, split + S, ... by log-sum-exp from its own
+    // shared memory.  No block reads another's shared memory afterwards, so none waits.
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();
     const int S = p.splits;
     const int rows_valid = gq * p.H;
-    // r: row within this block's slice (index into every block's partials); rg: in the group
-    for (int r = split + S * warp; r < NW * 16; r += S * NW) {
-      const int rg = row_base + r;
-      if (rg >= rows_valid) break;
-      const float ls = lane < S ? cluster.map_shared_rank(plse, lane)[r] : -INFINITY;
+    for (int slot = warp; slot < rpo; slot += NW) {
+      const int r = split + S * slot;   // row within the block's slice
+      const int rg = row_base + r;      // row within the group
+      if (r >= NW * 16 || rg >= rows_valid) break;
+      const float ls = lane < S ? recv_lse[slot * S + lane] : -INFINITY;
       float M = ls;
 #pragma unroll
       for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
@@ -454,13 +491,12 @@ __global__ void __launch_bounds__(NW * 32)
       for (int o2 = 16; o2 > 0; o2 >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o2);
       if (p.sink && M > -INFINITY) den += exp2f(s2 - M);
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      // unrolled so every split's (remote) partial row is in flight at once
+      const float4* part = reinterpret_cast<const float4*>(recv + (size_t)slot * S * D);
 #pragma unroll
       for (int s = 0; s < MAX_CLUSTER_ROWS; s++) {
         const float wgt = __shfl_sync(0xffffffffu, wl, s);
         if (s < S && wgt != 0.f) {
-          const float4 v =
-              reinterpret_cast<const float4*>(cluster.map_shared_rank(part, s) + r * D)[lane];
+          const float4 v = part[s * (D / 4) + lane];
           acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
         }
       }
@@ -470,7 +506,6 @@ __global__ void __launch_bounds__(NW * 32)
           make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
       if (p.lse && lane == 0) p.lse[orow] = den > 0.f ? (M + log2f(den)) * LN2 : -INFINITY;
     }
-    cluster.sync();  // no block leaves while another may still read its partial
   }
 }
 
@@ -580,11 +615,18 @@ hcl_status_t launch_t(const AttnParams& p, cudaStream_t st, long long grid) {
     return check_cuda(launch_pdl(kern, dim3((unsigned)grid), dim3(NW * 32), smem, st, 1, p),
                       "attention launch");
   }
-  smem += (size_t)NW * 16 * (D + 1) * sizeof(float);
-  static bool attr_done = false;  // per instantiation, set once
+  // receive buffers: ceil(rows / splits) slots x splits partials (+ LSE)
+  auto recv_bytes = [](int S) {
+    return (size_t)((NW * 16 + S - 1) / S) * S * (D + 1) * sizeof(float);
+  };
+  size_t recv_max = 0;
+  for (int S = 2; S <= MAX_CLUSTER; S++) recv_max = std::max(recv_max, recv_bytes(S));
+  const size_t smem_max = smem + recv_max;
+  smem += recv_bytes(p.splits);
+  static bool attr_done = false;  // per instantiation, set once (for the largest cluster need)
   if (!attr_done) {
     hcl_status_t e = check_cuda(
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max),
         "attention smem attribute");
     if (e != HCL_OK) return e;
     e = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1),
@@ -656,6 +698,7 @@ hcl_status_t launch_attn(const AttnArgs& a, void* ws, size_t ws_bytes, cudaStrea
   p.rows_pad = pl.rows_pad;
   p.cmerge = pl.cmerge;
   p.hsplit = pl.hsplit;
+  p.prewait = a.prewait;
   p.status = a.status;
   p.ws_o = nullptr;
   p.ws_lse = nullptr;

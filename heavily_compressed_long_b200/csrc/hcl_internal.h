@@ -83,6 +83,10 @@ struct IndexerArgs {
   void* scores;
   int score_fmt;
   int32_t* status;
+  // optional (decode with MXFP4 keys and bf16 scores): per group of 16 entries, the largest
+  // visible score as an order-preserving 16-bit key (0: no visible entry), rows of
+  // gmax_row_stride(Nc) groups
+  uint16_t* gmax = nullptr;
 };
 hcl_status_t launch_indexer(const IndexerArgs& a, cudaStream_t st);
 // MXFP4 keys with the bf16 index query [B, Tq, HI, 64] quantised inside the indexer's prologue
@@ -97,9 +101,16 @@ struct TopkArgs {
   int m, k;
   int32_t* idx;
   int32_t* status;
+  int prewait = 0;  // 1: q_pos does not come from the previous kernel in the stream
 };
 size_t topk_workspace_bytes(int B, int Tq, int Nc, int k, int score_fmt);
 hcl_status_t launch_topk(const TopkArgs& a, void* ws, size_t ws_bytes, cudaStream_t st);
+// Decode rows (bf16 scores) whose per-16-entry maxima the indexer wrote (IndexerArgs::gmax);
+// rows of gmax_row_stride(Nc) groups (a multiple of 16 groups), for Nc with
+// topk_gmax_supported(Nc).
+inline int gmax_row_stride(int Nc) { return ((Nc + 15) / 16 + 15) / 16 * 16; }
+bool topk_gmax_supported(int Nc);
+hcl_status_t launch_topk_gmax(const TopkArgs& a, const uint16_t* gmax, cudaStream_t st);
 
 // One attention launch: CSA (selected entries + window) or HCA (visible entries + window).
 struct AttnArgs {
@@ -119,6 +130,7 @@ struct AttnArgs {
   void* out;
   float* lse;
   int32_t* status;
+  int prewait = 0;  // 1: q and q_pos do not come from the previous kernel in the stream
 };
 // n = k (CSA) or Nh (HCA)
 size_t attn_workspace_bytes(int mode, int B, int Tq, int H, int n, int W);

@@ -49,6 +49,8 @@ struct IdxParams {
   int score_fmt;
   int B, Tq, HI, Nc, m, cap;
   int vec_ok;                 // Nc % 4 == 0 and scores 16-byte aligned: vector score stores
+  uint16_t* gmax;             // packed-row decode, bf16 scores: per-16-entry maxima, or null
+  int NG;                     // gmax row stride in groups
   int n_qt, n_kt, n_kc, kt_per_chunk;
   int32_t* status;
   long long limit;
@@ -467,6 +469,22 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
         v[j] = key + j < nv ? s : -INFINITY;
       }
       if (t0 >= p.Tq) return;
+      if (p.gmax != nullptr) {
+        // largest visible bf16 score of each 16-entry group (lanes 4q .. 4q+3 hold group
+        // key/16) as an order-preserving key: the top-k's lower bound comes from these
+        uint32_t km = 0u;
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+          if (key + j < nv) {
+            const uint32_t bits = __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
+            km = max(km, bits ^ ((bits & 0x8000u) ? 0xFFFFu : 0x8000u));
+          }
+        }
+        km = max(km, __shfl_xor_sync(0xffffffffu, km, 1));
+        km = max(km, __shfl_xor_sync(0xffffffffu, km, 2));
+        if ((lane & 3) == 0 && key < p.Nc)
+          p.gmax[((size_t)b * p.Tq + t0) * p.NG + (key >> 4)] = uint16_t(km);
+      }
       const size_t o = ((size_t)b * p.Tq + t0) * p.Nc + key;
       if (p.vec_ok && key + 3 < p.Nc) {
         if (p.score_fmt == HCL_FP32) {
@@ -591,6 +609,8 @@ hcl_status_t run(const IndexerArgs& a, const void* qI_bf16, const CUtensorMap& t
   p.kI_sf = static_cast<const uint8_t*>(a.kI_sf);
   p.B = a.B; p.Tq = a.Tq; p.HI = a.HI; p.Nc = a.Nc; p.m = a.m; p.cap = a.kI_cap;
   p.vec_ok = (a.Nc % 4 == 0) && (reinterpret_cast<uintptr_t>(a.scores) % 16 == 0);
+  p.gmax = (KIND == 2 && a.score_fmt == HCL_BF16) ? a.gmax : nullptr;
+  p.NG = gmax_row_stride(a.Nc);
   p.n_qt = (a.Tq + QT - 1) / QT;
   p.n_kt = (a.Nc + Lay::TK - 1) / Lay::TK;
   // key chunks per (sequence, query tile): as many as fill the co-resident slots without

@@ -209,6 +209,39 @@ def test_topk_exact(hcl, fmt, B, Tq, Nc, k):
     assert np.array_equal(out.cpu().numpy(), want)
 
 
+@pytest.mark.parametrize("off,B,Nc,k,kind", [
+    (3, 3, 100003, 1024, "ties"),      # rows start at every alignment, heavy ties
+    (5, 2, 262147, 1024, "normal"),
+    (1, 1, 9999, 2000, "ties"),
+    (7, 2, 40000, 1, "ties"),
+    (2, 1, 50000, 1000, "equal"),      # one value everywhere: the tie run spans every block
+    (0, 2, 131072, 1024, "runs"),      # long equal runs across block boundaries
+])
+def test_topk_bf16_layouts(hcl, off, B, Nc, k, kind):
+    """bf16 rows whose first key sits at any position of a 16-byte vector (the score tensor is
+    an element-offset view), lengths that are no multiple of 8, and threshold ties spread over
+    the cluster's blocks."""
+    if kind == "equal":
+        s = np.full((B, 1, Nc), 3.0, np.float32)
+    elif kind == "runs":
+        s = np.repeat(np.round(RNG.standard_normal((B, 1, Nc // 4096)), 1), 4096, axis=2)
+        s = s.astype(np.float32)
+    elif kind == "ties":
+        s = np.round(RNG.standard_normal((B, 1, Nc)) * 2, 1).astype(np.float32)
+    else:
+        s = RNG.standard_normal((B, 1, Nc)).astype(np.float32)
+    st = gen.to_bf16(s)
+    pos = torch.full((B, 1), 4 * Nc + 3, dtype=torch.int32)
+    want = oracle.topk(st.double().numpy(), pos, 4, k)
+    store = torch.zeros(B * Nc + 16, dtype=torch.bfloat16, device="cuda")
+    view = store[off:off + B * Nc].view(B, 1, Nc)
+    view.copy_(cuda(st))
+    out = torch.empty(B, 1, k, dtype=torch.int32, device="cuda")
+    hcl.hcl_csa_topk(view, cuda(pos), 4, k, out)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.cpu().numpy(), want)
+
+
 def test_topk_fewer_visible_and_negative(hcl):
     s = torch.randn(3, 2, 5000)
     s[1] = -torch.rand(2, 5000) * 1e3
@@ -350,3 +383,53 @@ def test_invalid_arguments_rejected(hcl):
                                  torch.zeros(1, 8, 32, dtype=torch.bfloat16, device="cuda"),
                                  torch.zeros(1, 1, dtype=torch.int32, device="cuda"), 4,
                                  torch.empty(1, 1, 8, device="cuda"))
+
+
+# =========================================================================================
+# fused decode step: MXFP4 keys + bf16 scores select from the indexer's per-16-entry maxima
+
+@pytest.mark.parametrize("B,Nc,k,nvis,ties", [
+    (3, 70000, 1024, (70000, 5000, 700), False),   # the last row has fewer than k visible
+    (2, 40000, 512, (40000, 39999), True),          # many equal scores, visibility mid-group
+    (1, 4096, 1024, (1030,), True),                 # just above k visible
+    (2, 262144, 1024, (262144, 131075), False),     # full decode length
+])
+def test_decode_step_group_maxima(hcl, B, Nc, k, nvis, ties):
+    """The fused step's top-k (group maxima lower bound) against the oracle's top-k of the very
+    scores the separate calls produce, and the fused step against the separate calls bitwise."""
+    from heavily_compressed_long_b200.api import HCL_BF16, HCL_MXFP4, KV
+    from heavily_compressed_long_b200.pipeline import CsaDecode
+    H, HI, W, d = 16, 16, 128, 128
+    L = 4 * Nc
+    kb = rbf16(B, Nc, 64)
+    if ties:                                   # few distinct key rows -> heavily tied scores
+        kb = kb[:, RNG.integers(0, 37, Nc)]
+    kp = torch.empty(B, Nc, 32, dtype=torch.uint8, device="cuda")
+    ks = torch.empty(B, Nc, 2, dtype=torch.uint8, device="cuda")
+    hcl.hcl_quant_mxfp4(cuda(kb), kp, ks)
+    ent = rbf16(B, Nc, d)
+    cn = torch.empty(B, Nc, 64, dtype=torch.uint8, device="cuda")
+    cs = torch.empty(B, Nc, dtype=torch.float32, device="cuda")
+    cr = torch.empty(B, Nc, 64, dtype=torch.bfloat16, device="cuda")
+    hcl.hcl_quant_kv_fp8(cuda(ent), cn, cs, cr)
+    raw = rbf16(B, W, d)
+    rn = torch.empty(B, W, 64, dtype=torch.uint8, device="cuda")
+    rs = torch.empty(B, W, dtype=torch.float32, device="cuda")
+    rr = torch.empty(B, W, 64, dtype=torch.bfloat16, device="cuda")
+    hcl.hcl_quant_kv_fp8(cuda(raw), rn, rs, rr)
+    q, qI = rbf16(B, 1, H, d), rbf16(B, 1, HI, 64)
+    w = torch.from_numpy(RNG.random((B, 1, HI)).astype(np.float32))
+    pos = torch.tensor([[4 * v - 1] for v in nvis], dtype=torch.int32)
+    pipe = CsaDecode(cuda(q), cuda(qI), cuda(w), kp, KV(cn, cs, cr), Nc, KV(rn, rs, rr), L, W,
+                     cuda(pos), m=4, k=k, op_fmt=HCL_MXFP4, score_fmt=HCL_BF16, kI_sf=ks)
+    pipe.step_parts()
+    torch.cuda.synchronize()
+    want = oracle.topk(as_f64(pipe.scores), pos, 4, k)
+    assert np.array_equal(pipe.idx.cpu().numpy(), want)
+    out1, idx1 = pipe.out.clone(), pipe.idx.clone()
+    pipe.idx.fill_(-7)
+    pipe.step()
+    torch.cuda.synchronize()
+    assert torch.equal(pipe.idx, idx1)
+    assert torch.equal(pipe.out, out1)
+    assert pipe.status.item() == 0
