@@ -395,8 +395,8 @@ hcl_status_t hcl_csa_decode_step(const void* q, const void* qI_bf16, const float
     e = topk_common(scores, score_fmt, B, 1, Nc, q_pos, m, k, idx, nullptr, 0, status, stream, 1);
   }
   if (e != HCL_OK) return e;
-  // the attention's predecessor is the top-k above, which writes neither q nor q_pos: the
-  // attention may load its queries before waiting for it
+  // the attention's predecessor is the top-k above, which writes neither q, q_pos nor the raw
+  // window: the attention may load those before waiting for it
   return attn_common(0, q, B, 1, H, d, kvc, Nc, 1, idx, k, raw, L, W, q_pos, scale, sink, out,
                      lse, wsb + l.attn, ws_bytes - l.attn, status, stream, 1);
 }

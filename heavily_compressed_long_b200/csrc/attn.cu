@@ -56,8 +56,8 @@ struct AttnParams {
   int G, n_groups, splits, cps, rows_pad;
   int cmerge;  // 1: the splits of a group form one cluster and merge through DSMEM
   int hsplit;  // blocks sharing one group's (query, head) rows (cluster merge only)
-  int prewait; // 1: q, q_pos are not written by the previous kernel in the stream, so they may
-               // be read before waiting for it (set only inside the fused decode step)
+  int prewait; // 1: q, q_pos and the raw window store are not written by the previous kernel in
+               // the stream, so they may be read before waiting for it (fused decode step only)
   int32_t* status;
 };
 
@@ -193,7 +193,10 @@ __global__ void __launch_bounds__(NW * 32)
     }
   }
 
-  if (p.prewait) pdl_enter();
+  // A CSA block whose rows are all window rows needs nothing from the previous kernel (the
+  // top-k): with prewait it gathers its rows before waiting.
+  const bool early = p.prewait && MODE == 0 && c_begin * KVB >= n_a;
+  if (p.prewait && !early) pdl_enter();
 
   float o[16][4];
 #pragma unroll
@@ -299,6 +302,7 @@ __global__ void __launch_bounds__(NW * 32)
     issue(0);
     if (c_begin + 1 < c_end) issue(1);
   }
+  if (early) pdl_enter();
   for (int c = c_begin; c < c_end; c++) {
     const int buf = (c - c_begin) & 1;
     if (c + 1 < c_end) cp_async_wait<1>();   // chunk c landed; chunk c+1 may be in flight

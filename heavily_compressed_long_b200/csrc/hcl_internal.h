@@ -130,7 +130,7 @@ struct AttnArgs {
   void* out;
   float* lse;
   int32_t* status;
-  int prewait = 0;  // 1: q and q_pos do not come from the previous kernel in the stream
+  int prewait = 0;  // 1: q, q_pos and raw do not come from the previous kernel in the stream
 };
 // n = k (CSA) or Nh (HCA)
 size_t attn_workspace_bytes(int mode, int B, int Tq, int H, int n, int W);
