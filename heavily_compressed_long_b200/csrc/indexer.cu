@@ -96,6 +96,17 @@ struct IdxLayout {
       tmem_cols_for(ACC_COLS + (KIND != 0 ? 4 * SF_BLOCKS * TPS + 4 : 0));
 };
 
+// Two fp32 lanes packed in 64 bits (x in the low word) and their paired fused multiply-add.
+__device__ __forceinline__ unsigned long long pack2(float x, float y) {
+  return (unsigned long long)__float_as_uint(x) | ((unsigned long long)__float_as_uint(y) << 32);
+}
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
+                                                   unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
 template <int KIND, int QT, int TPS, int STAGES, int NACC, int EPI>
 __global__ void __launch_bounds__(64 + 32 * EPI, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmSF,
@@ -434,18 +445,33 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
     mbar_wait(drain, 0, p.limit, nullptr);
   } else {
     // ---------------- epilogue ----------------
-    constexpr int QPER = EPI >= 8 ? QT / 2 : QT;
-    constexpr bool ALL_AT_ONCE = QPER * TPS <= 4;   // every column of a stage in one batch
-    constexpr int QG = QPER < 4 ? QPER : 4;          // otherwise: queries per load batch
+    // EPI/4 groups of four warps (one warp per TMEM lane quarter) split the tile's queries
+    constexpr int NGRP = EPI / 4;
+    static_assert(EPI % 4 == 0 && QT % NGRP == 0, "epilogue warps must split the queries evenly");
+    constexpr int QPER = QT / NGRP;
+    // queries per TMEM load batch (16 fp32 columns each): with 16 epilogue warps the register
+    // budget is smaller, and four warps per scheduler hide the load latency instead
+    constexpr int LDB = EPI >= 16 ? 2 : 4;
+    constexpr bool ALL_AT_ONCE = QPER * TPS <= LDB;  // every column of a stage in one batch
+    constexpr int QG = QPER < LDB ? QPER : LDB;      // otherwise: queries per load batch
     const int quarter = warp & 3;
     const int qbeg = ((warp - 2) / 4) * QPER;
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
 
     auto emit = [&](int tile, int q, const uint32_t (&r)[16]) {
-      const float* wq = sW + q * HP;
-      float s = 0.f;
+      // ReLU-weighted head sum as two interleaved fp32 chains (paired FMA), the weights read
+      // as four 16-byte vectors
+      const float4* wq = reinterpret_cast<const float4*>(sW + q * HP);
+      unsigned long long acc = 0ull;
 #pragma unroll
-      for (int h = 0; h < HP; h++) s = fmaf(wq[h], fmaxf(__uint_as_float(r[h]), 0.f), s);
+      for (int h4 = 0; h4 < HP / 4; h4++) {
+        const float4 wv = wq[h4];
+        acc = fma2(pack2(wv.x, wv.y), pack2(fmaxf(__uint_as_float(r[4 * h4]), 0.f),
+                                            fmaxf(__uint_as_float(r[4 * h4 + 1]), 0.f)), acc);
+        acc = fma2(pack2(wv.z, wv.w), pack2(fmaxf(__uint_as_float(r[4 * h4 + 2]), 0.f),
+                                            fmaxf(__uint_as_float(r[4 * h4 + 3]), 0.f)), acc);
+      }
+      const float s = __uint_as_float(uint32_t(acc)) + __uint_as_float(uint32_t(acc >> 32));
       const int t = t0 + q;
       const int key = tile * KEYS + quarter * 32 + lane;
       if (t < p.Tq && key < p.Nc) {
@@ -530,6 +556,49 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
         mbar_arrive(&acce[a]);
 #pragma unroll
         for (int t = 0; t < TPS; t++) emit4(tile0 + t, r[t]);
+      } else if constexpr (KIND == 0 && TPS > 1 && QT > 1) {
+        // prefill with several key tiles per stage: query by query, the weights are read once
+        // and applied to this thread's key in every tile of the stage; the next query's
+        // accumulator columns are loaded while this one is reduced
+        uint32_t r[2][TPS][16];
+#pragma unroll
+        for (int t = 0; t < TPS; t++) tmem_ld16(tacc + t * N + qbeg * HP, r[0][t]);
+#pragma unroll
+        for (int g = 0; g < QPER; g++) {
+          const int q = qbeg + g;
+          const float4* wq = reinterpret_cast<const float4*>(sW + q * HP);
+          const float4 w0 = wq[0], w1 = wq[1], w2 = wq[2], w3 = wq[3];
+          tmem_ld_wait();
+          if (g + 1 < QPER) {
+#pragma unroll
+            for (int t = 0; t < TPS; t++) tmem_ld16(tacc + t * N + (q + 1) * HP, r[(g + 1) & 1][t]);
+          } else {
+            tc_fence_before();
+            mbar_arrive(&acce[a]);
+          }
+#pragma unroll
+          for (int t = 0; t < TPS; t++) {
+            const uint32_t* rr = r[g & 1][t];
+            unsigned long long acc = 0ull;
+            const float wv[16] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w,
+                                  w2.x, w2.y, w2.z, w2.w, w3.x, w3.y, w3.z, w3.w};
+#pragma unroll
+            for (int h = 0; h < HP; h += 2)
+              acc = fma2(pack2(wv[h], wv[h + 1]),
+                         pack2(fmaxf(__uint_as_float(rr[h]), 0.f),
+                               fmaxf(__uint_as_float(rr[h + 1]), 0.f)),
+                         acc);
+            const float sc = __uint_as_float(uint32_t(acc)) + __uint_as_float(uint32_t(acc >> 32));
+            const int tq = t0 + q;
+            const int key = (tile0 + t) * KEYS + quarter * 32 + lane;
+            if (tq < p.Tq && key < p.Nc) {
+              const float v = key < sNvis[q] ? sc : -INFINITY;
+              const size_t o = ((size_t)b * p.Tq + tq) * p.Nc + key;
+              if (p.score_fmt == HCL_FP32) static_cast<float*>(p.scores)[o] = v;
+              else static_cast<__nv_bfloat16*>(p.scores)[o] = __float2bfloat16_rn(v);
+            }
+          }
+        }
       } else if (ALL_AT_ONCE) {
         uint32_t r[TPS * QPER][16];
 #pragma unroll
@@ -619,6 +688,14 @@ hcl_status_t run(const IndexerArgs& a, const void* qI_bf16, const CUtensorMap& t
   const long long base = (long long)a.B * p.n_qt;
   const int n_stages_total = (p.n_kt + TPS - 1) / TPS;
   int n_kc = (int)std::max(1LL, std::min<long long>(n_stages_total, target / base));
+  if (base > target) {
+    // more (query tile) blocks than slots: split the keys so that the last wave is nearly
+    // full, as long as every block keeps >= 32 stages to amortise its prologue
+    for (int c = 1; c <= 8 && n_stages_total / c >= 32; c++) {
+      const long long blocks = base * c, waves = (blocks + target - 1) / target;
+      if (blocks * 100 >= waves * target * 95) { n_kc = c; break; }
+    }
+  }
   const int st_per_chunk = (n_stages_total + n_kc - 1) / n_kc;
   p.kt_per_chunk = st_per_chunk * TPS;
   p.n_kc = (p.n_kt + p.kt_per_chunk - 1) / p.kt_per_chunk;
@@ -649,6 +726,8 @@ hcl_status_t make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, 
 
 // Decode configurations: stage = TPS tiles; box rows = min(256, TPS*128).
 constexpr int DEC_BF16_TPS = 2;
+// bf16 prefill: 8 queries x 16 heads (N = 128) against two 128-key tiles per stage
+constexpr int PRE_BF16_TPS = 2;
 
 }  // namespace
 
@@ -660,12 +739,12 @@ hcl_status_t launch_indexer_q(const IndexerArgs& a, const void* qI_bf16, cudaStr
   const bool mx = a.op_fmt == HCL_MXFP4;
   const bool decode = a.Tq <= 2;
   if (!mx) {
-    const cuuint32_t rows = decode ? std::min(256, DEC_BF16_TPS * KEYS) : KEYS;
+    const cuuint32_t rows = std::min(256, (decode ? DEC_BF16_TPS : PRE_BF16_TPS) * KEYS);
     e = make_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.kI, 64, a.kI_cap, a.B, 128,
                  (cuuint64_t)a.kI_cap * 128, 64, rows, CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != HCL_OK) return e;
     if (decode) return run<0, 1, DEC_BF16_TPS, 3, 3, 4>(a, nullptr, tmK, tmSF, st, 0);
-    return run<0, 16, 1, 4, 2, 8>(a, nullptr, tmK, tmSF, st, 120 * 1024);
+    return run<0, 8, PRE_BF16_TPS, 4, 2, 8>(a, nullptr, tmK, tmSF, st, 0);
   }
   if (decode) {
     // packed rows: [B, cap/4, 128 B] (four keys per row), 16 KB boxes with SW128; the key
