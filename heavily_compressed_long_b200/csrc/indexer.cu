@@ -307,7 +307,9 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
     if (KIND == 0) {
       for (int u = et; u < QT * HP; u += ne) {
         const int q = u / HP, h = u % HP, t = t0 + q;
-        sW[u] = (t < p.Tq && h < p.HI) ? p.w[((size_t)b * p.Tq + t) * p.HI + h] : 0.f;
+        // (multi-tile prefill keeps w/2: its reduction forms w * relu(x) as (w/2) * (x + |x|))
+        const float wv = (t < p.Tq && h < p.HI) ? p.w[((size_t)b * p.Tq + t) * p.HI + h] : 0.f;
+        sW[u] = (TPS > 1 && QT > 1) ? 0.5f * wv : wv;
       }
       for (int q = et; q < QT; q += ne) {
         const int t = t0 + q;
@@ -582,12 +584,13 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
             unsigned long long acc = 0ull;
             const float wv[16] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w,
                                   w2.x, w2.y, w2.z, w2.w, w3.x, w3.y, w3.z, w3.w};
+            // w * relu(x) == (w/2) * (x + |x|) exactly (x + |x| is 2x or 0): an add with an
+            // absolute-value operand on the FMA pipe instead of a max on the ALU pipe
 #pragma unroll
-            for (int h = 0; h < HP; h += 2)
-              acc = fma2(pack2(wv[h], wv[h + 1]),
-                         pack2(fmaxf(__uint_as_float(rr[h]), 0.f),
-                               fmaxf(__uint_as_float(rr[h + 1]), 0.f)),
-                         acc);
+            for (int h = 0; h < HP; h += 2) {
+              const float x0 = __uint_as_float(rr[h]), x1 = __uint_as_float(rr[h + 1]);
+              acc = fma2(pack2(wv[h], wv[h + 1]), pack2(x0 + fabsf(x0), x1 + fabsf(x1)), acc);
+            }
             const float sc = __uint_as_float(uint32_t(acc)) + __uint_as_float(uint32_t(acc >> 32));
             const int tq = t0 + q;
             const int key = (tile0 + t) * KEYS + quarter * 32 + lane;
