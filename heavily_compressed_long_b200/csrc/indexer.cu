@@ -562,25 +562,34 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
         // prefill with several key tiles per stage: query by query, the weights are read once
         // and applied to this thread's key in every tile of the stage; the next query's
         // accumulator columns are loaded while this one is reduced
-        uint32_t r[2][TPS][16];
+        // (with 16 epilogue warps the registers do not allow the look-ahead; four warps per
+        // scheduler hide the load latency instead)
+        constexpr int PD = EPI >= 16 ? 1 : 2;
+        uint32_t r[PD][TPS][16];
+        if (PD == 2) {
 #pragma unroll
-        for (int t = 0; t < TPS; t++) tmem_ld16(tacc + t * N + qbeg * HP, r[0][t]);
+          for (int t = 0; t < TPS; t++) tmem_ld16(tacc + t * N + qbeg * HP, r[0][t]);
+        }
 #pragma unroll
         for (int g = 0; g < QPER; g++) {
           const int q = qbeg + g;
+          if (PD == 1) {
+#pragma unroll
+            for (int t = 0; t < TPS; t++) tmem_ld16(tacc + t * N + q * HP, r[0][t]);
+          }
           const float4* wq = reinterpret_cast<const float4*>(sW + q * HP);
           const float4 w0 = wq[0], w1 = wq[1], w2 = wq[2], w3 = wq[3];
           tmem_ld_wait();
-          if (g + 1 < QPER) {
+          if (PD == 2 && g + 1 < QPER) {
 #pragma unroll
-            for (int t = 0; t < TPS; t++) tmem_ld16(tacc + t * N + (q + 1) * HP, r[(g + 1) & 1][t]);
-          } else {
+            for (int t = 0; t < TPS; t++) tmem_ld16(tacc + t * N + (q + 1) * HP, r[(g + 1) % PD][t]);
+          } else if (g + 1 == QPER) {
             tc_fence_before();
             mbar_arrive(&acce[a]);
           }
 #pragma unroll
           for (int t = 0; t < TPS; t++) {
-            const uint32_t* rr = r[g & 1][t];
+            const uint32_t* rr = r[g % PD][t];
             unsigned long long acc = 0ull;
             const float wv[16] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w,
                                   w2.x, w2.y, w2.z, w2.w, w3.x, w3.y, w3.z, w3.w};
@@ -747,7 +756,7 @@ hcl_status_t launch_indexer_q(const IndexerArgs& a, const void* qI_bf16, cudaStr
                  (cuuint64_t)a.kI_cap * 128, 64, rows, CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != HCL_OK) return e;
     if (decode) return run<0, 1, DEC_BF16_TPS, 3, 3, 4>(a, nullptr, tmK, tmSF, st, 0);
-    return run<0, 8, PRE_BF16_TPS, 4, 2, 8>(a, nullptr, tmK, tmSF, st, 0);
+    return run<0, 8, PRE_BF16_TPS, 4, 2, 16>(a, nullptr, tmK, tmSF, st, 0);
   }
   if (decode) {
     // packed rows: [B, cap/4, 128 B] (four keys per row), 16 KB boxes with SW128; the key
