@@ -95,7 +95,6 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
-// 3-D tiled TMA load into shared memory, completing on `bar` (transaction bytes).
 // Untiled bulk copy global -> this CTA's shared memory, completing `bytes` on `bar`.  Both
 // addresses 16-byte aligned, bytes a multiple of 16 (no multicast).
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
@@ -107,6 +106,7 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
+// 3-D tiled TMA load into shared memory, completing on `bar` (transaction bytes).
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int x,
                                             int y, int z) {
   asm volatile(
