@@ -571,6 +571,389 @@ __global__ void attn_merge_kernel(AttnParams p) {
   if (p.lse && lane == 0) p.lse[gw] = den > 0.f ? (M + log2f(den)) * LN2 : -INFINITY;
 }
 
+// ---------------------------------------------------------------------------------------
+// CSA decode on tcgen05 tensor cores (one query per sequence, up to 128 heads).
+// Block = (sequence, KV split of up to TC_MAXC chunks of 64 rows); thread t <-> head t <->
+// TMEM lane t.  Shared memory holds Q (128 heads x 128 dims), the gathered KV rows of the
+// split and P, all as 128-byte SW128 rows (dims 0-63 and 64-127 in two halves).  The same
+// KV tile is the K-major B operand of S = Q K^T (N = 64 rows per chunk) and the MN-major B
+// operand of O = P V (K = rows, N = 128 dims), so V needs no transpose.  S (64 fp32 columns
+// per chunk) and O (128 columns) live in TMEM.  The softmax is two-pass over the split's
+// chunks: row maximum, then exp2 / row sum / P in bf16.  Splits merge as in attn_kernel.
+constexpr int TC_MAXC = 4;          // chunks per block with a single split
+constexpr int TC_MAXC_MERGE = 2;    // chunks per block when splits merge in a cluster
+constexpr int TC_ROWS = 128;        // head rows per block = UMMA M = TMEM lanes
+constexpr int TC_THREADS = 256;     // two threads per row (column halves)
+
+struct TcOff {
+  uint32_t q, kv, pm, stg, scl, rs, bar, vis, xch, recv, lse, total;
+};
+__host__ __device__ inline TcOff tc_offsets(int cps, int splits) {
+  TcOff o;
+  o.q = 0;                                   // 2 halves x 128 rows x 128 B
+  o.kv = 32768;                              // cps x (2 halves x 64 rows x 128 B)
+  o.pm = o.kv + cps * 16384;                 // cps x (128 rows x 128 B)
+  o.stg = o.pm + cps * 16384;                // fp8: cps x 64 rows x 64 B codes
+  o.scl = o.stg + cps * 4096;                // fp8: cps x 64 scales
+  o.rs = o.scl + cps * 256;                  // cps x 64 RowSrc
+  o.bar = o.rs + cps * 64 * (uint32_t)sizeof(RowSrc);   // 2 mbarriers + TMEM base
+  o.vis = o.bar + 32;                        // row-visibility bits, 64 per chunk
+  o.xch = (o.vis + 8 * cps + 15) & ~15u;     // partial maxima / sums of the two column halves
+  o.recv = o.xch + 2 * TC_THREADS * 4;       // cluster merge: rpo x splits x D floats
+  const int rpo = splits > 1 ? (TC_ROWS + splits - 1) / splits : 0;
+  o.lse = o.recv + (uint32_t)(rpo * splits * D * 4);
+  o.total = o.lse + (uint32_t)(rpo * splits * 4);
+  return o;
+}
+
+template <int KVFMT>
+__global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
+  const bool early_ok = p.prewait != 0;
+  extern __shared__ __align__(1024) uint8_t tc_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tc_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int row = tid & (TC_ROWS - 1);   // head row = TMEM lane (warps w and w+4 share a quadrant)
+  const int hc = tid / TC_ROWS;          // which half of the columns this thread handles
+  const int split = blockIdx.x % p.splits;
+  const int b = blockIdx.x / p.splits;
+  const TcOff off = tc_offsets(p.cps, p.splits);
+  uint8_t* sQ = sm + off.q;
+  RowSrc* rsrc = reinterpret_cast<RowSrc*>(sm + off.rs);
+  uint64_t* bar_s = reinterpret_cast<uint64_t*>(sm + off.bar);
+  uint64_t* bar_o = bar_s + 1;
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + off.bar + 16);
+  uint32_t* visw = reinterpret_cast<uint32_t*>(sm + off.vis);
+  float* xch = reinterpret_cast<float*>(sm + off.xch);   // [2][TC_THREADS]: partial max, sum
+  float* recv = reinterpret_cast<float*>(sm + off.recv);
+  float* recv_lse = reinterpret_cast<float*>(sm + off.lse);
+
+  // row list of this split: k selected entries, then the W window rows
+  const int n_a = p.k, total = p.k + p.W;
+  const int n_chunks = (total + KVB - 1) / KVB;
+  const int c_begin = split * p.cps;
+  const int c_end = split == p.splits - 1 ? n_chunks : min(n_chunks, c_begin + p.cps);
+  const int nch = max(0, min(TC_MAXC, c_end - c_begin));
+  const uint32_t ocol = uint32_t(p.cps * 64);              // O columns after the S columns
+  const uint32_t ncols = ocol + D <= 256 ? 256u : 512u;
+
+  if (tid == 0) {
+    mbar_init(bar_s, 1);
+    mbar_init(bar_o, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(sTmem, ncols);
+    tmem_relinquish();
+  }
+  const bool early = early_ok && c_begin * KVB >= n_a;     // window rows only
+  if (!early_ok) pdl_enter();
+  const int pos = p.q_pos[b];
+  const int raw_lo = pos - p.W + 1;
+
+  // Q: thread (row, hc) loads dims 64*hc .. 64*hc+63 of head `row` into SW128 half hc
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.H + row) * D) + hc * 8;
+#pragma unroll
+    for (int c = 0; c < 8; c++) {
+      const uint4 v = row < p.H ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(sQ + hc * 16384 + row * 128 + ((c ^ (row & 7)) << 4)) = v;
+    }
+  }
+  if (early_ok && !early) pdl_enter();
+
+  // rows of the split: resolve, then gather (rope half / bf16 rows straight into the SW128
+  // tile with cp.async, E4M3 codes and scales into staging)
+  const int nrows = nch * KVB;
+  for (int jj = tid; jj < nrows; jj += TC_THREADS) {
+    const int e = c_begin * KVB + jj;
+    RowSrc rs{-1, 0};
+    if (e < n_a) {
+      long long ent = p.idx[(size_t)b * p.k + e];
+      if (ent < -1 || ent >= p.n_comp) {
+        report(p.status, HCL_ERR_DEVICE_FAULT);
+        ent = -1;
+      }
+      if (ent >= 0) rs.slot = (long long)b * p.comp.cap + (ent % p.comp.cap);
+    } else if (e < total) {
+      const long long u = (long long)raw_lo + (e - n_a);
+      if (u >= 0) { rs.slot = (long long)b * p.raw.cap + (u % p.raw.cap); rs.from_raw = 1; }
+    }
+    rsrc[jj] = rs;
+  }
+  __syncthreads();
+  // one bit per row of the split (row j of chunk c: word 2c + j/32, bit j%32)
+  for (int w0 = 0; w0 < nrows; w0 += TC_THREADS) {
+    const int jj = w0 + tid;
+    const uint32_t bits = __ballot_sync(0xffffffffu, jj < nrows && rsrc[jj].slot >= 0);
+    if (lane == 0 && jj < nrows) visw[jj >> 5] = bits;
+  }
+  {
+    constexpr int PIECES = KVFMT == HCL_BF16 ? 16 : 13;
+    for (int u = tid; u < nrows * PIECES; u += TC_THREADS) {
+      const int jj = u / PIECES, c = u % PIECES;
+      const int ch = jj / KVB, r = jj % KVB;
+      const RowSrc rs = rsrc[jj];
+      const hcl_kv_t& st = rs.from_raw ? p.raw : p.comp;
+      uint8_t* kv = sm + off.kv + ch * 16384;
+      if (KVFMT == HCL_BF16) {
+        uint8_t* dst = kv + (c >> 3) * 8192 + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+        if (rs.slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.data) + rs.slot * 256 + c * 16);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+      } else if (c < 8) {          // RoPE dims 64..127: the second half, as stored
+        uint8_t* dst = kv + 8192 + r * 128 + ((c ^ (r & 7)) << 4);
+        if (rs.slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.rope) + rs.slot * 128 + c * 16);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+      } else if (c < 12) {         // E4M3 codes of dims 0..63
+        uint8_t* dst = sm + off.stg + (ch * KVB + r) * 64 + (c - 8) * 16;
+        if (rs.slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.data) + rs.slot * 64 + (c - 8) * 16);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+      } else {
+        float* dst = reinterpret_cast<float*>(sm + off.scl) + ch * KVB + r;
+        if (rs.slot >= 0)
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)),
+                       "l"(st.scale + rs.slot)
+                       : "memory");
+        else *dst = 0.f;
+      }
+    }
+    cp_async_commit();
+  }
+  if (early) pdl_enter();
+  cp_async_wait<0>();
+  __syncthreads();
+  if (KVFMT == HCL_FP8SPLIT) {
+    // widen: 8 codes x scale -> one 16-byte bf16 chunk of the first half
+    for (int u = tid; u < nrows * 8; u += TC_THREADS) {
+      const int jj = u >> 3, c = u & 7, ch = jj / KVB, r = jj % KVB;
+      const uint2 codes = *reinterpret_cast<const uint2*>(sm + off.stg + (ch * KVB + r) * 64 + c * 8);
+      const float sc = reinterpret_cast<const float*>(sm + off.scl)[ch * KVB + r];
+      uint4 v;
+      v.x = e4m3x2_to_bf16x2(uint16_t(codes.x & 0xffff), sc);
+      v.y = e4m3x2_to_bf16x2(uint16_t(codes.x >> 16), sc);
+      v.z = e4m3x2_to_bf16x2(uint16_t(codes.y & 0xffff), sc);
+      v.w = e4m3x2_to_bf16x2(uint16_t(codes.y >> 16), sc);
+      *reinterpret_cast<uint4*>(sm + off.kv + ch * 16384 + r * 128 + ((c ^ (r & 7)) << 4)) = v;
+    }
+  }
+  fence_proxy_async_smem();      // Q, the gathered rows and the widened halves -> UMMA
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *sTmem;
+  const long long limit = 2000000000LL;
+
+  // S_c = Q K_c^T (M = 128 heads, N = 64 rows, K = 128 dims in 8 steps of 16)
+  if (tid == 0 && nch > 0) {
+    const uint32_t aq = smem_u32(sQ);
+    for (int c = 0; c < nch; c++) {
+      const uint32_t ak = smem_u32(sm + off.kv + c * 16384);
+#pragma unroll
+      for (int ks = 0; ks < 8; ks++) {
+        const uint32_t h = ks >> 2, kk = ks & 3;
+        umma_bf16(tbase + c * 64, make_sdesc(aq + h * 16384 + kk * 32, 16, 1024, SMEM_SWIZZLE_128B),
+                  make_sdesc(ak + h * 8192 + kk * 32, 16, 1024, SMEM_SWIZZLE_128B),
+                  idesc_bf16(128, 64), ks > 0 ? 1u : 0u);
+      }
+    }
+    umma_commit(bar_s);
+  }
+  bool ok = nch == 0 || mbar_wait(bar_s, 0, limit, nullptr);
+  if (!ok) report(p.status, HCL_ERR_TIMEOUT);
+  tc_fence_after();
+
+  // softmax for head `row` over the split's rows (log2 domain); this thread holds columns
+  // 32*hc .. 32*hc+31 of every chunk and exchanges its partial maximum and sum with the
+  // other half's thread through shared memory
+  const uint32_t trow = tbase + (uint32_t((warp & 3) * 32) << 16);
+  float lmax = -INFINITY;
+  auto cols = [&](int c, uint32_t (&r32)[32]) {
+    tmem_ld16(trow + c * 64 + hc * 32, *reinterpret_cast<uint32_t(*)[16]>(&r32[0]));
+    tmem_ld16(trow + c * 64 + hc * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r32[16]));
+  };
+  uint32_t sv[2][32];
+  const bool inreg = nch <= 2;
+  if (inreg) {
+#pragma unroll
+    for (int c = 0; c < 2; c++)
+      if (c < nch) cols(c, sv[c]);
+    tmem_ld_wait();
+#pragma unroll
+    for (int c = 0; c < 2; c++)
+      if (c < nch) {
+        const uint32_t vb = visw[2 * c + hc];
+#pragma unroll
+        for (int j = 0; j < 32; j++)
+          if ((vb >> j) & 1u) lmax = fmaxf(lmax, __uint_as_float(sv[c][j]) * p.scale_log2);
+      }
+  } else {
+    for (int c = 0; c < nch; c++) {
+      uint32_t r32[32];
+      cols(c, r32);
+      tmem_ld_wait();
+      const uint32_t vb = visw[2 * c + hc];
+#pragma unroll
+      for (int j = 0; j < 32; j++)
+        if ((vb >> j) & 1u) lmax = fmaxf(lmax, __uint_as_float(r32[j]) * p.scale_log2);
+    }
+  }
+  xch[tid] = lmax;
+  __syncthreads();
+  const float mrow = fmaxf(xch[row], xch[row + TC_ROWS]);
+  const float muse = mrow == -INFINITY ? 0.f : mrow;
+  float lsum = 0.f;
+  auto emit_p = [&](int c, const uint32_t (&r32)[32]) {
+    const uint32_t vb = visw[2 * c + hc];
+    uint8_t* prow = sm + off.pm + c * 16384 + row * 128;
+#pragma unroll
+    for (int q4 = 0; q4 < 4; q4++) {
+      uint32_t pk[4];
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        const int j = q4 * 8 + i;
+        const float p0 = ((vb >> j) & 1u) ? exp2f(__uint_as_float(r32[j]) * p.scale_log2 - muse) : 0.f;
+        const float p1 = ((vb >> (j + 1)) & 1u) ? exp2f(__uint_as_float(r32[j + 1]) * p.scale_log2 - muse) : 0.f;
+        lsum += p0 + p1;
+        pk[i >> 1] = pack_bf16(p0, p1);
+      }
+      *reinterpret_cast<uint4*>(prow + (((hc * 4 + q4) ^ (row & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+  };
+  if (inreg) {
+#pragma unroll
+    for (int c = 0; c < 2; c++)
+      if (c < nch) emit_p(c, sv[c]);
+  } else {
+    for (int c = 0; c < nch; c++) {
+      uint32_t r32[32];
+      cols(c, r32);
+      tmem_ld_wait();
+      emit_p(c, r32);
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();               // (also: every thread has read the partial maxima)
+  xch[TC_THREADS + tid] = lsum;
+  tc_fence_after();
+
+  // O = sum_c P_c V_c (M = 128 heads, N = 128 dims, K = 64 rows per chunk in 4 steps of 16);
+  // V is MN-major: 64-dim halves 8 KB apart (LBO), 8-row groups 1 KB apart (SBO)
+  if (tid == 0 && nch > 0) {
+    for (int c = 0; c < nch; c++) {
+      const uint32_t ap = smem_u32(sm + off.pm + c * 16384);
+      const uint32_t av = smem_u32(sm + off.kv + c * 16384);
+#pragma unroll
+      for (int ks = 0; ks < 4; ks++)
+        umma_bf16(tbase + ocol, make_sdesc(ap + ks * 32, 16, 1024, SMEM_SWIZZLE_128B),
+                  make_sdesc(av + ks * 2048, 8192, 1024, SMEM_SWIZZLE_128B),
+                  idesc_bf16(128, D) | (1u << 16), (c > 0 || ks > 0) ? 1u : 0u);
+    }
+    umma_commit(bar_o);
+  }
+  ok = nch == 0 || mbar_wait(bar_o, 0, limit, nullptr);
+  if (!ok) report(p.status, HCL_ERR_TIMEOUT);
+  __syncthreads();               // the partial sums
+  tc_fence_after();
+
+  // output dims 64*hc .. 64*hc+63 of head `row`: normalised partial (o, lse) or the output
+  const bool hv = row < p.H;
+  float m2 = mrow, l2 = xch[TC_THREADS + row] + xch[TC_THREADS + row + TC_ROWS];
+  const float inv_l = l2 > 0.f ? 1.f / l2 : 0.f;
+  float* pdst = nullptr;
+  if (p.splits > 1) {
+    cg::cluster_group cluster = cg::this_cluster();
+    const int owner = row % p.splits, slot = row / p.splits;
+    pdst = cluster.map_shared_rank(recv, owner) + ((size_t)slot * p.splits + split) * D + hc * 64;
+    if (hv && hc == 0)
+      *(cluster.map_shared_rank(recv_lse, owner) + slot * p.splits + split) =
+          l2 > 0.f ? m2 + log2f(l2) : -INFINITY;
+  }
+  float f = inv_l;
+  if (p.splits == 1 && p.sink) {
+    const float s2 = p.sink[min(row, p.H - 1)] * LOG2E;
+    const float mm = fmaxf(m2, s2);
+    const float fa = l2 > 0.f ? exp2f(m2 - mm) : 0.f;
+    const float l3 = l2 * fa + exp2f(s2 - mm);
+    f = l3 > 0.f ? fa / l3 : 0.f;
+    l2 = l3;
+    m2 = mm;
+  }
+  {
+    uint32_t r64[64];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; q4++)
+      tmem_ld16(trow + ocol + hc * 64 + q4 * 16, *reinterpret_cast<uint32_t(*)[16]>(&r64[q4 * 16]));
+    tmem_ld_wait();
+    if (hv) {
+      if (p.splits > 1) {
+#pragma unroll
+        for (int i = 0; i < 64; i += 4)
+          *reinterpret_cast<float4*>(pdst + i) =
+              make_float4(__uint_as_float(r64[i]) * inv_l, __uint_as_float(r64[i + 1]) * inv_l,
+                          __uint_as_float(r64[i + 2]) * inv_l, __uint_as_float(r64[i + 3]) * inv_l);
+      } else {
+        __nv_bfloat16* dst = p.out + ((size_t)b * p.H + row) * D + hc * 64;
+#pragma unroll
+        for (int i = 0; i < 64; i += 8) {
+          reinterpret_cast<uint4*>(dst + i)[0] =
+              make_uint4(pack_bf16(__uint_as_float(r64[i]) * f, __uint_as_float(r64[i + 1]) * f),
+                         pack_bf16(__uint_as_float(r64[i + 2]) * f, __uint_as_float(r64[i + 3]) * f),
+                         pack_bf16(__uint_as_float(r64[i + 4]) * f, __uint_as_float(r64[i + 5]) * f),
+                         pack_bf16(__uint_as_float(r64[i + 6]) * f, __uint_as_float(r64[i + 7]) * f));
+        }
+      }
+    }
+  }
+  if (p.splits == 1 && hv && hc == 0 && p.lse)
+    p.lse[(size_t)b * p.H + row] = l2 > 0.f ? (m2 + log2f(l2)) * LN2 : -INFINITY;
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, ncols);
+  }
+  if (p.splits > 1) {
+    // merge the rows this block owns (row r -> block r % splits, slot r / splits)
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    const int S = p.splits;
+    const int rpo = (TC_ROWS + S - 1) / S;
+    for (int slot = warp; slot < rpo; slot += TC_THREADS / 32) {
+      const int h = split + S * slot;
+      if (h >= p.H) break;
+      const float ls = lane < S ? recv_lse[slot * S + lane] : -INFINITY;
+      float M = ls;
+#pragma unroll
+      for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
+      float s2 = -INFINITY;
+      if (p.sink) {
+        s2 = p.sink[h] * LOG2E;
+        M = fmaxf(M, s2);
+      }
+      const float wl = (ls == -INFINITY || M == -INFINITY) ? 0.f : exp2f(ls - M);
+      float den = wl;
+#pragma unroll
+      for (int o2 = 16; o2 > 0; o2 >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o2);
+      if (p.sink && M > -INFINITY) den += exp2f(s2 - M);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4* part = reinterpret_cast<const float4*>(recv + (size_t)slot * S * D);
+#pragma unroll
+      for (int s = 0; s < MAX_CLUSTER_ROWS; s++) {
+        const float wgt = __shfl_sync(0xffffffffu, wl, s);
+        if (s < S && wgt != 0.f) {
+          const float4 v = part[s * (D / 4) + lane];
+          acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
+        }
+      }
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+      const size_t orow = (size_t)b * p.H + h;
+      reinterpret_cast<uint2*>(p.out + orow * D)[lane] =
+          make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
+      if (p.lse && lane == 0) p.lse[orow] = den > 0.f ? (M + log2f(den)) * LN2 : -INFINITY;
+    }
+  }
+}
+
 struct Plan {
   int G, NW, n_groups, splits, cps, rows_pad, n_chunks_max, cmerge, hsplit;
 };
@@ -665,6 +1048,48 @@ hcl_status_t launch_nw(const AttnParams& p, int NW, cudaStream_t st, long long g
   }
 }
 
+// CSA decode on tcgen05 when the plan allows it: one query per sequence, all heads in one
+// block (up to 128), splits merged in a cluster (or a single split), <= TC_MAXC chunks each.
+bool tc_usable(const AttnArgs& a, const Plan& pl) {
+  return a.mode == 0 && a.Tq == 1 && a.H <= TC_ROWS &&
+         ((pl.splits == 1 && pl.cps <= TC_MAXC) || (pl.cmerge && pl.cps <= TC_MAXC_MERGE));
+}
+
+template <int KVFMT>
+hcl_status_t launch_tc(const AttnParams& p, cudaStream_t st) {
+  auto kern = attn_tc_kernel<KVFMT>;
+  size_t smem_max = (size_t)tc_offsets(TC_MAXC, 1).total + 1024;
+  for (int S = 2; S <= MAX_CLUSTER; S++)
+    smem_max = std::max(smem_max, (size_t)tc_offsets(TC_MAXC_MERGE, S).total + 1024);
+  static bool attr_done = false;
+  if (!attr_done) {
+    hcl_status_t e = check_cuda(
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max),
+        "attention smem attribute");
+    if (e != HCL_OK) return e;
+    e = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1),
+                   "attention cluster attribute");
+    if (e != HCL_OK) return e;
+    attr_done = true;
+  }
+  const size_t smem = (size_t)tc_offsets(p.cps, p.splits).total + 1024;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = p.splits;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.gridDim = dim3((unsigned)(p.B * p.splits));
+  cfg.blockDim = dim3(TC_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.splits > 1 ? 2 : 1;
+  return check_cuda(cudaLaunchKernelEx(&cfg, kern, p), "attention launch");
+}
+
 // Longest row list a block may process: CSA k selected entries + W window rows; HCA every
 // entry (n = Nh) plus the union of the G windows of a query group.  The workspace query and
 // the launch both plan from this one number.
@@ -714,6 +1139,9 @@ hcl_status_t launch_attn(const AttnArgs& a, void* ws, size_t ws_bytes, cudaStrea
                   need, ws_bytes);
     p.ws_o = static_cast<float*>(ws);
     p.ws_lse = p.ws_o + items * pl.rows_pad * D;
+  }
+  if (tc_usable(a, pl)) {
+    return a.comp.fmt == HCL_FP8SPLIT ? launch_tc<HCL_FP8SPLIT>(p, st) : launch_tc<HCL_BF16>(p, st);
   }
   const long long grid = (long long)a.B * pl.n_groups * pl.hsplit * pl.splits;
   hcl_status_t e;
