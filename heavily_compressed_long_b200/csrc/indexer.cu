@@ -333,6 +333,8 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
     // ---------------- TMA producer ----------------
     asm volatile("bar.sync 3, %0;" ::"r"(32 + 32 * EPI) : "memory");  // prologue loads issued
     if (lane == 0) {
+      // decode streams every key exactly once: keep it from displacing the scores in L2
+      const uint64_t pol = l2_evict_first_policy();
       int issued = 0;
       for (int i = 0; i < nstages; i++) {
         const int s = i % STAGES;
@@ -349,14 +351,19 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
             KIND == 2 ? 2u * (uint32_t)min(TPS * Lay::TK, p.cap - key0) : TPS * Lay::SF_TILE;
         mbar_arrive_expect_tx(&full[s], TPS * Lay::A_TILE + sf_bytes);
 #pragma unroll
-        for (int r = 0; r < TPS * KEYS; r += Lay::BOX_ROWS)
-          tma_load_3d(sA + s * Lay::A_STAGE + r * Lay::ROWB, &tmK, &full[s], 0,
-                      key0 / Lay::KPR + r, b);
+        for (int r = 0; r < TPS * KEYS; r += Lay::BOX_ROWS) {
+          if (KIND == 2)
+            tma_load_3d_hint(sA + s * Lay::A_STAGE + r * Lay::ROWB, &tmK, &full[s], 0,
+                             key0 / Lay::KPR + r, b, pol);
+          else
+            tma_load_3d(sA + s * Lay::A_STAGE + r * Lay::ROWB, &tmK, &full[s], 0,
+                        key0 / Lay::KPR + r, b);
+        }
         if (KIND == 1)
           tma_load_3d(sSFraw + s * TPS * 256, &tmSF, &full[s], 0, key0 / 8, b);
         if (KIND == 2)
-          bulk_load(sSFraw + s * TPS * Lay::SF_TILE, p.kI_sf + ((size_t)b * p.cap + key0) * 2,
-                    sf_bytes, &full[s]);
+          bulk_load_hint(sSFraw + s * TPS * Lay::SF_TILE, p.kI_sf + ((size_t)b * p.cap + key0) * 2,
+                         sf_bytes, &full[s], pol);
         issued++;
       }
       // Drain: every issued copy has landed before the block may exit.
