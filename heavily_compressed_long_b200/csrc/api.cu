@@ -187,7 +187,8 @@ static hcl_status_t index_scores_impl(int op_fmt, const void* qI, const void* qI
                                       const void* kI_sf, int B, int Tq, int HI, int dI, int Nc,
                                       int kI_cap, const int32_t* q_pos, int m, void* scores,
                                       int score_fmt, int32_t* status, void* stream,
-                                      uint16_t* gmax = nullptr) {
+                                      uint16_t* gmax = nullptr, uint16_t* g2nd = nullptr,
+                                      uint8_t* garg = nullptr) {
   HCL_REQUIRE(op_fmt == HCL_BF16 || op_fmt == HCL_MXFP4, "op_fmt must be HCL_BF16 or HCL_MXFP4");
   HCL_REQUIRE(score_fmt == HCL_FP32 || score_fmt == HCL_BF16, "score_fmt must be HCL_FP32 or HCL_BF16");
   HCL_REQUIRE(B >= 0 && Tq >= 0 && Nc >= 0, "negative size");
@@ -204,7 +205,7 @@ static hcl_status_t index_scores_impl(int op_fmt, const void* qI, const void* qI
     HCL_REQUIRE((qI_bf16 || qI_sf) && kI_sf && aligned16(kI_sf),
                 "MXFP4 needs 16-byte aligned scale arrays");
   IndexerArgs a{op_fmt, qI, qI_sf, w, kI, kI_sf, B, Tq, HI, dI, Nc, kI_cap, q_pos, m, scores,
-                score_fmt, status, gmax};
+                score_fmt, status, gmax, g2nd, garg};
   return launch_indexer_q(a, qI_bf16, as_stream(stream));
 }
 
@@ -347,7 +348,8 @@ static DecodeWs decode_ws_layout(int B, int H, int HI, int Nc, int k, int W, int
   l.scores = off;
   off += align256((size_t)B * Nc * (score_fmt == HCL_BF16 ? 2 : 4));
   l.gmax = off;
-  if (decode_uses_gmax(op_fmt, score_fmt, Nc)) off += align256((size_t)B * hcl::gmax_row_stride(Nc) * 2);
+  // group maxima, second maxima (u16) and positions (u8)
+  if (decode_uses_gmax(op_fmt, score_fmt, Nc)) off += align256((size_t)B * hcl::gmax_row_stride(Nc) * 5);
   l.idx = off;
   off += align256((size_t)B * k * 4);
   l.attn = off;
@@ -378,9 +380,12 @@ hcl_status_t hcl_csa_decode_step(const void* q, const void* qI_bf16, const float
   void* scores = wsb + l.scores;
   uint16_t* gmax =
       decode_uses_gmax(op_fmt, score_fmt, Nc) ? reinterpret_cast<uint16_t*>(wsb + l.gmax) : nullptr;
+  const size_t ngs = (size_t)B * hcl::gmax_row_stride(Nc);
+  uint16_t* g2nd = gmax ? gmax + ngs : nullptr;
+  uint8_t* garg = gmax ? reinterpret_cast<uint8_t*>(g2nd + ngs) : nullptr;
   if (op_fmt == HCL_MXFP4)
     e = index_scores_impl(op_fmt, nullptr, nullptr, qI_bf16, w, kI, kI_sf, B, 1, HI, dI, Nc,
-                          kI_cap, q_pos, m, scores, score_fmt, status, stream, gmax);
+                          kI_cap, q_pos, m, scores, score_fmt, status, stream, gmax, g2nd, garg);
   else
     e = index_scores_impl(op_fmt, qI_bf16, nullptr, nullptr, w, kI, kI_sf, B, 1, HI, dI, Nc,
                           kI_cap, q_pos, m, scores, score_fmt, status, stream);
@@ -390,7 +395,7 @@ hcl_status_t hcl_csa_decode_step(const void* q, const void* qI_bf16, const float
   if (gmax != nullptr) {
     HCL_REQUIRE(k >= 1 && k <= 4096, "k must be in [1, 4096]");
     TopkArgs ta{scores, score_fmt, B, 1, Nc, q_pos, m, k, idx, status, 1};
-    e = launch_topk_gmax(ta, gmax, as_stream(stream));
+    e = launch_topk_gmax(ta, gmax, g2nd, garg, as_stream(stream));
   } else {
     e = topk_common(scores, score_fmt, B, 1, Nc, q_pos, m, k, idx, nullptr, 0, status, stream, 1);
   }

@@ -87,6 +87,8 @@ struct IndexerArgs {
   // visible score as an order-preserving 16-bit key (0: no visible entry), rows of
   // gmax_row_stride(Nc) groups
   uint16_t* gmax = nullptr;
+  uint16_t* g2nd = nullptr;   // with gmax: the second largest per group
+  uint8_t* garg = nullptr;    // with gmax: the largest's position in its group (0..15)
 };
 hcl_status_t launch_indexer(const IndexerArgs& a, cudaStream_t st);
 // MXFP4 keys with the bf16 index query [B, Tq, HI, 64] quantised inside the indexer's prologue
@@ -110,7 +112,8 @@ hcl_status_t launch_topk(const TopkArgs& a, void* ws, size_t ws_bytes, cudaStrea
 // topk_gmax_supported(Nc).
 inline int gmax_row_stride(int Nc) { return ((Nc + 15) / 16 + 15) / 16 * 16; }
 bool topk_gmax_supported(int Nc);
-hcl_status_t launch_topk_gmax(const TopkArgs& a, const uint16_t* gmax, cudaStream_t st);
+hcl_status_t launch_topk_gmax(const TopkArgs& a, const uint16_t* gmax, const uint16_t* g2nd,
+                              const uint8_t* garg, cudaStream_t st);
 
 // One attention launch: CSA (selected entries + window) or HCA (visible entries + window).
 struct AttnArgs {

@@ -50,6 +50,8 @@ struct IdxParams {
   int B, Tq, HI, Nc, m, cap;
   int vec_ok;                 // Nc % 4 == 0 and scores 16-byte aligned: vector score stores
   uint16_t* gmax;             // packed-row decode, bf16 scores: per-16-entry maxima, or null
+  uint16_t* g2nd;             //   second largest per group
+  uint8_t* garg;              //   position of the largest in its group
   int NG;                     // gmax row stride in groups
   int n_qt, n_kt, n_kc, kt_per_chunk;
   int32_t* status;
@@ -505,20 +507,36 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
       }
       if (t0 >= p.Tq) return;
       if (p.gmax != nullptr) {
-        // largest visible bf16 score of each 16-entry group (lanes 4q .. 4q+3 hold group
-        // key/16) as an order-preserving key: the top-k's lower bound comes from these
-        uint32_t km = 0u;
+        // per 16-entry group (lanes 4q .. 4q+3 hold group key/16), as order-preserving keys of
+        // the bf16 scores: the largest visible score, its position in the group (the lowest
+        // on ties) and the second largest (equal to the largest when that repeats; 0 when
+        // there is none).  The top-k's lower bound and its candidate list come from these.
+        uint32_t m1 = 0u, m2 = 0u, a1 = 0u;
 #pragma unroll
         for (int j = 0; j < 4; j++) {
           if (key + j < nv) {
             const uint32_t bits = __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
-            km = max(km, bits ^ ((bits & 0x8000u) ? 0xFFFFu : 0x8000u));
+            const uint32_t kk = bits ^ ((bits & 0x8000u) ? 0xFFFFu : 0x8000u);
+            if (kk > m1) { m2 = m1; m1 = kk; a1 = uint32_t((lane & 3) * 4 + j); }
+            else if (kk > m2) { m2 = kk; }
           }
         }
-        km = max(km, __shfl_xor_sync(0xffffffffu, km, 1));
-        km = max(km, __shfl_xor_sync(0xffffffffu, km, 2));
-        if ((lane & 3) == 0 && key < p.Nc)
-          p.gmax[((size_t)b * p.Tq + t0) * p.NG + (key >> 4)] = uint16_t(km);
+#pragma unroll
+        for (int o = 1; o <= 2; o <<= 1) {
+          const uint32_t n1 = __shfl_xor_sync(0xffffffffu, m1, o);
+          const uint32_t n2 = __shfl_xor_sync(0xffffffffu, m2, o);
+          const uint32_t b1 = __shfl_xor_sync(0xffffffffu, a1, o);
+          const uint32_t second = max(min(m1, n1), max(m2, n2));
+          if (n1 > m1 || (n1 == m1 && b1 < a1)) a1 = b1;
+          m1 = max(m1, n1);
+          m2 = second;
+        }
+        if ((lane & 3) == 0 && key < p.Nc) {
+          const size_t gi = ((size_t)b * p.Tq + t0) * p.NG + (key >> 4);
+          p.gmax[gi] = uint16_t(m1);
+          p.g2nd[gi] = uint16_t(m2);
+          p.garg[gi] = uint8_t(a1);
+        }
       }
       const size_t o = ((size_t)b * p.Tq + t0) * p.Nc + key;
       if (p.vec_ok && key + 3 < p.Nc) {
@@ -698,6 +716,8 @@ hcl_status_t run(const IndexerArgs& a, const void* qI_bf16, const CUtensorMap& t
   p.B = a.B; p.Tq = a.Tq; p.HI = a.HI; p.Nc = a.Nc; p.m = a.m; p.cap = a.kI_cap;
   p.vec_ok = (a.Nc % 4 == 0) && (reinterpret_cast<uintptr_t>(a.scores) % 16 == 0);
   p.gmax = (KIND == 2 && a.score_fmt == HCL_BF16) ? a.gmax : nullptr;
+  p.g2nd = a.g2nd;
+  p.garg = a.garg;
   p.NG = gmax_row_stride(a.Nc);
   p.n_qt = (a.Tq + QT - 1) / QT;
   p.n_kt = (a.Nc + Lay::TK - 1) / Lay::TK;

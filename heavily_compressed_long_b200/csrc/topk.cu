@@ -1052,26 +1052,35 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
 
 // ---------------------------------------------------------------------------------------
 // Decode selection from group maxima (inside the fused decode step, bf16 scores).  The indexer
-// also writes, for every group of 16 entries, the largest visible score as an order-preserving
-// key.  The k-th largest of those maxima, L, is a lower bound of the row's k-th largest score
-// (the maxima are scores of k distinct entries), so only groups whose maximum reaches L can
-// hold selected entries -- on typical data about k groups, a few per cent of the row.  One
-// block per row: histogram of the maxima -> L; histogram of the visible scores >= L in those
-// groups -> the exact threshold T; then an index-ordered scan of the groups whose maximum
-// reaches T places every selected entry.  No cluster, no exchange between blocks.
+// also writes, for every group of 16 entries, a summary of its visible scores as
+// order-preserving keys: the largest, the second largest and the position of the largest.  The
+// k-th largest of the maxima, L, is a lower bound of the row's k-th largest score (the maxima
+// are scores of k distinct entries), so only groups whose maximum reaches L can hold selected
+// entries -- on typical data about k groups, a few per cent of the row -- and a group whose
+// second largest key is below L holds exactly one candidate, known from the summary.  One block
+// per row: histogram of the maxima -> L; histogram of the candidate keys (scores read only for
+// the few groups with two or more) -> the exact threshold T; then an index-ordered scan places
+// every selected entry.  No cluster, no exchange between blocks.
 
 constexpr int GM_G = 16;         // entries per group
 constexpr int GM_GPT = 16;       // groups per thread: rows of up to 16 x 1024 groups
 constexpr int GM_MAX_GROUPS = GM_GPT * TK_THREADS;
 
-constexpr int GM_CAND = 12288;   // candidate keys compacted in shared memory
 constexpr int GM_WWORDS = 4096;  // window histogram: 8192 digits
+constexpr int GM_POOL = 512;     // groups with several candidates staged in shared memory
 
 struct alignas(16) GmShared {
-  uint16_t list[GM_MAX_GROUPS];  // candidate group ids, in index order
-  uint16_t ckey[GM_CAND];        // candidate keys and their entries, in index order
-  uint32_t cidx[GM_CAND];
-  uint32_t wh[GM_WWORDS];        // u16 pairs over the digit window [wb, wb + 8191]
+  union {
+    uint16_t list[GM_MAX_GROUPS];    // candidate group ids, in index order (fallback)
+    uint32_t praw[GM_POOL][8];       // scores of the pooled groups as copied (bf16 pairs)
+  };
+  uint32_t wh[GM_WWORDS];        // u16 pairs over the digit window [wb, wb + 8191]: maxima
+  uint32_t wc[GM_WWORDS];        // the same over the candidate keys
+  uint32_t sc[GM_GPT][TK_THREADS];   // single candidate of group 16t+i: key << 4 | position
+  uint32_t pent[GM_POOL][GM_G];  // candidates of the pooled groups: key << 4 | position
+  uint32_t pcnt[GM_POOL];        // and their number
+  uint32_t ncand;                // candidate keys in the row
+  uint32_t npool;                // pool slots asked for
   uint32_t wcnt[TK_WARPS][16];   // per-warp digit counts of one radix pass
   uint32_t scan_tmp[TK_WARPS + 1];
   uint32_t red[2][TK_WARPS];
@@ -1247,6 +1256,7 @@ __device__ __forceinline__ uint32_t key_of(const uint32_t (&kk)[8], int i) {
 // thread never straddle a row.
 __global__ void __launch_bounds__(TK_THREADS, 1)
     topk_gm_kernel(const __nv_bfloat16* __restrict__ scores, const uint16_t* __restrict__ gmax,
+                   const uint16_t* __restrict__ g2nd, const uint8_t* __restrict__ garg,
                    int Nc, int NGP, const int32_t* __restrict__ q_pos, int m, int k,
                    int32_t* __restrict__ idx, int32_t* status, int prewait) {
   extern __shared__ __align__(16) uint8_t tk_smem[];
@@ -1280,6 +1290,26 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
       if (g0 + i >= ngv) gmr[i >> 1] &= (i & 1) ? 0x0000FFFFu : 0xFFFF0000u;
   }
   auto gm_of = [&](int i) { return (gmr[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu; };
+  // their second maxima and the positions of the maxima
+  uint32_t g2r[GM_GPT / 2], gar[GM_GPT / 4];
+  {
+    const int g0 = GM_GPT * tid;
+    uint4 a = make_uint4(0, 0, 0, 0), b2 = a, c = a;
+    if (g0 < ngv) {
+      const uint4* v2 = reinterpret_cast<const uint4*>(g2nd + row * (long long)NGP + g0);
+      a = __ldg(v2);
+      b2 = __ldg(v2 + 1);
+      c = __ldg(reinterpret_cast<const uint4*>(garg + row * (long long)NGP + g0));
+    }
+    g2r[0] = a.x; g2r[1] = a.y; g2r[2] = a.z; g2r[3] = a.w;
+    g2r[4] = b2.x; g2r[5] = b2.y; g2r[6] = b2.z; g2r[7] = b2.w;
+    gar[0] = c.x; gar[1] = c.y; gar[2] = c.z; gar[3] = c.w;
+  }
+  auto sec_of = [&](int i) { return (g2r[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu; };
+  auto arg_of = [&](int i) { return (gar[i >> 2] >> ((i & 3) * 8)) & 0xFu; };
+  static_assert(GM_WWORDS == 4 * TK_THREADS, "one uint4 of the candidate histogram per thread");
+  reinterpret_cast<uint4*>(S.wc)[tid] = make_uint4(0, 0, 0, 0);
+  if (tid == 0) { S.ncand = 0u; S.npool = 0u; }
   // block: number of maxima and the largest (the row's largest visible key)
   uint32_t nz = 0, tmax = 0;
 #pragma unroll
@@ -1359,8 +1389,126 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
     }
   }
 
-  // ---- candidate groups (maximum >= L) listed in index order (thread t owns groups
-  // 16t .. 16t+15), so that the loads can be spread evenly over the threads
+  // ---- candidates: the visible keys >= L.  Thread t owns groups 16t .. 16t+15, in index
+  // order.  A group with one candidate gives it (key, position) from the summary; the scores
+  // of a group with more are copied into a pool slot (all copies in flight together) and its
+  // candidates listed there.  Every candidate key goes into the window histogram, and the
+  // block counts them.
+  const uint32_t L1 = max(L, 1u);   // key 0 marks an invisible entry
+  uint32_t qm = 0, dm = 0;          // bit i: group 16t+i holds one candidate / two or more
+  const bool inwin = L >= wb;       // every candidate key lies in the window
+#pragma unroll
+  for (int i = 0; i < GM_GPT; i++) {
+    const uint32_t mx = gm_of(i);
+    if (mx >= L1) {
+      if (sec_of(i) >= L) {
+        dm |= 1u << i;
+      } else {
+        qm |= 1u << i;
+        S.sc[i][tid] = (mx << 4) | arg_of(i);
+        if (inwin) atomicAdd(&S.wc[(mx - wb) >> 1], 1u << (((mx - wb) & 1) << 4));
+      }
+    }
+  }
+  uint32_t c = __popc(qm);
+  const uint32_t ndm = __popc(dm);
+  const uint32_t pbase = ndm ? atomicAdd(&S.npool, ndm) : 0u;
+  if (ndm && pbase + ndm <= GM_POOL) {
+    uint32_t sl = pbase;
+    for (uint32_t mm = dm; mm; mm &= mm - 1u, sl++) {
+      const int e0 = GM_G * (GM_GPT * tid + __ffs(mm) - 1);
+      if (al && e0 + GM_G <= nvis) {
+        cp_async16(&S.praw[sl][0], sr + e0);
+        cp_async16(&S.praw[sl][4], sr + e0 + 8);
+      } else {
+#pragma unroll
+        for (int w = 0; w < 8; w++)
+          S.praw[sl][w] = uint32_t(sr[min(e0 + 2 * w, nvis - 1)]) |
+                          (uint32_t(sr[min(e0 + 2 * w + 1, nvis - 1)]) << 16);
+      }
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    sl = pbase;
+    for (uint32_t mm = dm; mm; mm &= mm - 1u, sl++) {
+      const int nv = nvis - GM_G * (GM_GPT * tid + __ffs(mm) - 1);   // visible: min(nv, 16)
+      uint32_t n = 0;
+#pragma unroll
+      for (int j = 0; j < GM_G; j++) {
+        const uint32_t key = ordered_key_bf16(uint16_t(S.praw[sl][j >> 1] >> ((j & 1) * 16)));
+        if (j < nv && key >= L1) {
+          S.pent[sl][n++] = (key << 4) | uint32_t(j);
+          if (inwin) atomicAdd(&S.wc[(key - wb) >> 1], 1u << (((key - wb) & 1) << 4));
+        }
+      }
+      S.pcnt[sl] = n;
+      c += n;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if (lane == 0 && c) atomicAdd(&S.ncand, c);
+  __syncthreads();
+
+  uint32_t T = 0u, above = 0u;
+  // u16 digit counts cannot overflow while the row has fewer than 2^16 candidates
+  if (inwin && S.ncand < 65536u && S.npool <= (uint32_t)GM_POOL) {
+    local_suffix(S.wc, int((Mx - wb) >> 1), int((L - wb) >> 1), (uint32_t)k, S.scan_tmp, S.res);
+    if (S.res[2]) {
+      T = S.res[0] + wb;
+      above = S.res[1];
+      const uint32_t krem = (uint32_t)k - above;
+      // ---- emission in index order: one packed (ties, above) scan over the threads
+      uint32_t gt = 0, eq = 0;
+      for (uint32_t mm = qm; mm; mm &= mm - 1u) {
+        const uint32_t key = S.sc[__ffs(mm) - 1][tid] >> 4;
+        gt += key > T;
+        eq += key == T;
+      }
+      for (uint32_t sl = pbase; sl < pbase + ndm; sl++) {
+        const uint32_t n = S.pcnt[sl];
+        for (uint32_t e = 0; e < n; e++) {
+          const uint32_t key = S.pent[sl][e] >> 4;
+          gt += key > T;
+          eq += key == T;
+        }
+      }
+      unsigned long long tot64;
+      const unsigned long long ex =
+          block_scan64((static_cast<unsigned long long>(eq) << 32) | gt, S.tmp64, tot64);
+      if (gt | eq) {
+        uint32_t e_before = uint32_t(ex >> 32);
+        uint32_t slot = uint32_t(ex) + min(e_before, krem);
+        auto place = [&](uint32_t v, int e0) {
+          const uint32_t key = v >> 4;
+          bool sel = key > T;
+          if (!sel && key == T) { sel = e_before < krem; e_before++; }
+          if (sel) {
+            if (slot < (uint32_t)k) out[slot] = e0 + int(v & 15u);
+            else report(status, HCL_ERR_DEVICE_FAULT);
+            slot++;
+          }
+        };
+        uint32_t sl = pbase;
+        for (uint32_t mm = qm | dm; mm; mm &= mm - 1u) {
+          const int i = __ffs(mm) - 1, e0 = GM_G * (GM_GPT * tid + i);
+          if ((qm >> i) & 1u) {
+            place(S.sc[i][tid], e0);
+          } else {
+            const uint32_t n = S.pcnt[sl];
+            for (uint32_t e = 0; e < n; e++) place(S.pent[sl][e], e0);
+            sl++;
+          }
+        }
+      }
+      return;
+    }
+  }
+  T = 0u;
+  above = 0u;
+
+  // ---- keys spread below the window or 2^16 candidates and more (heavy ties): select over the
+  // candidate groups, listed in index order, reloading their keys in every pass
   uint32_t ngc;
   {
     uint32_t nq = 0;
@@ -1372,155 +1520,6 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
       if (gm_of(i) != 0u && gm_of(i) >= L) S.list[o++] = uint16_t(GM_GPT * tid + i);
   }
   __syncthreads();
-  // ---- candidate keys (visible, >= L) compacted in index order: (key, entry) pairs.  With at
-  // most 2 * 1024 candidate groups, thread t takes list items 2t and 2t+1, with all four
-  // 16-byte loads issued before any is used; otherwise the groups are taken 1024 at a time.
-  uint32_t ncand = 0;
-  bool fits = true;
-  if (ngc <= 2u * TK_THREADS) {
-    const int ja = 2 * tid, jb = 2 * tid + 1;
-    const int ga = ja < int(ngc) ? S.list[ja] : -1;
-    const int gb = jb < int(ngc) ? S.list[jb] : -1;
-    const bool fa = ga >= 0 && al && GM_G * ga + GM_G <= nvis;   // full, aligned groups
-    const bool fb = gb >= 0 && al && GM_G * gb + GM_G <= nvis;
-    uint4 ra0 = make_uint4(0, 0, 0, 0), ra1 = ra0, rb0 = ra0, rb1 = ra0;
-    if (fa) { const uint4* v = reinterpret_cast<const uint4*>(sr + GM_G * ga); ra0 = __ldg(v); ra1 = __ldg(v + 1); }
-    if (fb) { const uint4* v = reinterpret_cast<const uint4*>(sr + GM_G * gb); rb0 = __ldg(v); rb1 = __ldg(v + 1); }
-    uint32_t ka[8], kb[8];
-    if (fa) {
-      ka[0] = ordered_key_bf16x2(ra0.x); ka[1] = ordered_key_bf16x2(ra0.y);
-      ka[2] = ordered_key_bf16x2(ra0.z); ka[3] = ordered_key_bf16x2(ra0.w);
-      ka[4] = ordered_key_bf16x2(ra1.x); ka[5] = ordered_key_bf16x2(ra1.y);
-      ka[6] = ordered_key_bf16x2(ra1.z); ka[7] = ordered_key_bf16x2(ra1.w);
-    } else if (ga >= 0) {
-      load_group(sr, al, ga, nvis, ka);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; i++) ka[i] = 0u;
-    }
-    if (fb) {
-      kb[0] = ordered_key_bf16x2(rb0.x); kb[1] = ordered_key_bf16x2(rb0.y);
-      kb[2] = ordered_key_bf16x2(rb0.z); kb[3] = ordered_key_bf16x2(rb0.w);
-      kb[4] = ordered_key_bf16x2(rb1.x); kb[5] = ordered_key_bf16x2(rb1.y);
-      kb[6] = ordered_key_bf16x2(rb1.z); kb[7] = ordered_key_bf16x2(rb1.w);
-    } else if (gb >= 0) {
-      load_group(sr, al, gb, nvis, kb);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; i++) kb[i] = 0u;
-    }
-    uint32_t ca = 0, cb = 0;
-#pragma unroll
-    for (int i = 0; i < 16; i++) {
-      const uint32_t x = key_of(ka, i), y = key_of(kb, i);
-      ca += x != 0u && x >= L;
-      cb += y != 0u && y >= L;
-    }
-    uint32_t tot;
-    uint32_t o = block_scan_total(ca + cb, S.scan_tmp, tot);
-    ncand = tot;
-    fits = tot <= (uint32_t)GM_CAND;
-    if (fits) {
-      if (ca) {
-#pragma unroll
-        for (int i = 0; i < 16; i++) {
-          const uint32_t key = key_of(ka, i);
-          if (key != 0u && key >= L) { S.ckey[o] = uint16_t(key); S.cidx[o] = GM_G * ga + i; o++; }
-        }
-      }
-      if (cb) {
-#pragma unroll
-        for (int i = 0; i < 16; i++) {
-          const uint32_t key = key_of(kb, i);
-          if (key != 0u && key >= L) { S.ckey[o] = uint16_t(key); S.cidx[o] = GM_G * gb + i; o++; }
-        }
-      }
-    }
-  } else {
-    for (int j0 = 0; j0 < int(ngc); j0 += TK_THREADS) {
-      const int j = j0 + tid;
-      uint32_t kk[8];
-      uint32_t c = 0;
-      int g = 0;
-      if (j < int(ngc)) {
-        g = S.list[j];
-        load_group(sr, al, g, nvis, kk);
-#pragma unroll
-        for (int i = 0; i < 16; i++) { const uint32_t key = key_of(kk, i); c += key != 0u && key >= L; }
-      }
-      uint32_t tot;
-      uint32_t o = ncand + block_scan_total(c, S.scan_tmp, tot);
-      if (ncand + tot > GM_CAND) fits = false;     // uniform over the block
-      if (fits && c) {
-#pragma unroll
-        for (int i = 0; i < 16; i++) {
-          const uint32_t key = key_of(kk, i);
-          if (key != 0u && key >= L) { S.ckey[o] = uint16_t(key); S.cidx[o] = GM_G * g + i; o++; }
-        }
-      }
-      ncand += tot;
-      if (!fits) break;
-    }
-  }
-  __syncthreads();
-
-  uint32_t T = 0u, above = 0u;
-  if (fits) {
-    // ---- T over the compacted candidates: thread t holds candidates [t*cpt, (t+1)*cpt)
-    const int cpt = (int(ncand) + TK_THREADS - 1) / TK_THREADS;
-    const int c0 = min(int(ncand), tid * cpt), c1 = min(int(ncand), c0 + cpt);
-    bool done = false;
-    if (L >= wb) {
-      // every candidate lies in the window [wb, Mx]: one histogram and one suffix search
-      for (int w = tid; w < GM_WWORDS; w += TK_THREADS) S.wh[w] = 0u;
-      __syncthreads();
-      for (int j = c0; j < c1; j++) {
-        const uint32_t d = S.ckey[j] - wb;
-        atomicAdd(&S.wh[d >> 1], 1u << ((d & 1) << 4));
-      }
-      __syncthreads();
-      local_suffix(S.wh, int((Mx - wb) >> 1), int((L - wb) >> 1), (uint32_t)k, S.scan_tmp, S.res);
-      if (S.res[2]) { T = S.res[0] + wb; above = S.res[1]; done = true; }
-    }
-    if (!done) {
-      uint32_t target = (uint32_t)k, pmask = 0u;
-      T = 0u;
-      above = 0u;
-#pragma unroll 1
-      for (int shift = 12; shift >= 0; shift -= 4) {
-        Digits4 c;
-        for (int j = c0; j < c1; j++) {
-          const uint32_t key = S.ckey[j];
-          if ((key & pmask) == T) c.add((key >> shift) & 15u);
-        }
-        T |= radix4_reduce(c, target, above, S.wcnt, S.res) << shift;
-        pmask |= 15u << shift;
-      }
-    }
-    const uint32_t krem = (uint32_t)k - above;
-    // ---- emission in index order: one packed (ties, above) scan over the candidate slices
-    uint32_t gt = 0, eq = 0;
-    for (int j = c0; j < c1; j++) { const uint32_t key = S.ckey[j]; gt += key > T; eq += key == T; }
-    unsigned long long tot64;
-    const unsigned long long ex =
-        block_scan64((static_cast<unsigned long long>(eq) << 32) | gt, S.tmp64, tot64);
-    uint32_t e_before = uint32_t(ex >> 32);
-    uint32_t slot = uint32_t(ex) + min(e_before, krem);
-    for (int j = c0; j < c1; j++) {
-      const uint32_t key = S.ckey[j];
-      bool sel = key > T;
-      if (!sel && key == T) { sel = e_before < krem; e_before++; }
-      if (sel) {
-        if (slot < (uint32_t)k) out[slot] = int32_t(S.cidx[j]);
-        else report(status, HCL_ERR_DEVICE_FAULT);
-        slot++;
-      }
-    }
-    return;
-  }
-
-  // ---- too many candidates for shared memory (heavy ties): select over the listed candidate
-  // groups, reloading their keys in every pass
   {
     uint32_t target = (uint32_t)k, pmask = 0u;
 #pragma unroll 1
@@ -1579,7 +1578,8 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
   }
 }
 
-hcl_status_t run_topk_gm(const TopkArgs& a, const uint16_t* gmax, cudaStream_t st) {
+hcl_status_t run_topk_gm(const TopkArgs& a, const uint16_t* gmax, const uint16_t* g2nd,
+                        const uint8_t* garg, cudaStream_t st) {
   auto kern = topk_gm_kernel;
   const int smem = (int)sizeof(GmShared);
   static bool attr_done = false;
@@ -1593,7 +1593,8 @@ hcl_status_t run_topk_gm(const TopkArgs& a, const uint16_t* gmax, cudaStream_t s
   const long long rows = (long long)a.B * a.Tq;
   const int NGP = gmax_row_stride(a.Nc);
   return check_cuda(launch_pdl(kern, dim3((unsigned)rows), dim3(TK_THREADS), (size_t)smem, st, 1,
-                               static_cast<const __nv_bfloat16*>(a.scores), gmax, a.Nc, NGP,
+                               static_cast<const __nv_bfloat16*>(a.scores), gmax, g2nd, garg,
+                               a.Nc, NGP,
                                a.q_pos, a.m, a.k, a.idx, a.status, a.prewait),
                     "topk launch");
 }
@@ -1805,10 +1806,11 @@ hcl_status_t run_topk_reg(const TopkArgs& a, cudaStream_t st, bool* used) {
 
 bool topk_gmax_supported(int Nc) { return (Nc + GM_G - 1) / GM_G <= GM_MAX_GROUPS; }
 
-hcl_status_t launch_topk_gmax(const TopkArgs& a, const uint16_t* gmax, cudaStream_t st) {
+hcl_status_t launch_topk_gmax(const TopkArgs& a, const uint16_t* gmax, const uint16_t* g2nd,
+                              const uint8_t* garg, cudaStream_t st) {
   if ((long long)a.B * a.Tq == 0 || a.k == 0) return HCL_OK;
   if (!topk_gmax_supported(a.Nc)) return fail(HCL_ERR_UNSUPPORTED, "group-maxima top-k: Nc too large");
-  return run_topk_gm(a, gmax, st);
+  return run_topk_gm(a, gmax, g2nd, garg, st);
 }
 
 hcl_status_t launch_topk(const TopkArgs& a, void*, size_t, cudaStream_t st) {
