@@ -1074,9 +1074,11 @@ struct alignas(16) GmShared {
     uint16_t list[GM_MAX_GROUPS];    // candidate group ids, in index order (fallback)
     uint32_t praw[GM_POOL][8];       // scores of the pooled groups as copied (bf16 pairs)
   };
+  uint4 gms[2][TK_THREADS];      // thread t's 16 group maxima (0: no visible entry),
+  uint4 g2s[2][TK_THREADS];      // their second maxima
+  uint4 gas[TK_THREADS];         // and the positions of the maxima (low 4 bits of a byte)
   uint32_t wh[GM_WWORDS];        // u16 pairs over the digit window [wb, wb + 8191]: maxima
   uint32_t wc[GM_WWORDS];        // the same over the candidate keys
-  uint32_t sc[GM_GPT][TK_THREADS];   // single candidate of group 16t+i: key << 4 | position
   uint32_t pent[GM_POOL][GM_G];  // candidates of the pooled groups: key << 4 | position
   uint32_t pcnt[GM_POOL];        // and their number
   uint32_t ncand;                // candidate keys in the row
@@ -1118,17 +1120,18 @@ __device__ unsigned long long block_scan64(unsigned long long v, unsigned long l
   return res;
 }
 
-// Block-local suffix search over one histogram (u16 pairs) between words w_bot and w_top, in
-// rounds of 4096 words (4 per thread, one 16-byte load).  res[0] = digit T of the target-th
-// largest key, res[1] = keys above T, res[2] = 1 if found.
-__device__ void local_suffix(const uint32_t* hist, int w_top, int w_bot, uint32_t target,
-                             uint32_t* tmp, uint32_t* res) {
-  const int tid = threadIdx.x;
-  if (tid == 0) res[2] = 0;
-  __syncthreads();
+// Suffix search over one histogram of u16 digit pairs (word w: digit 2w low, 2w+1 high)
+// between words w_bot and w_top, done by one warp from the top down in chunks of 128 words
+// (4 per lane) and stopping at the chunk that holds the target: the keys sit near the top of
+// the window, so a chunk or two usually suffices.  res[0] = digit T of the target-th largest
+// counted key, res[1] = keys in digits above T, res[2] = 1 if found.  The caller publishes
+// res with a barrier.
+__device__ void warp_suffix(const uint32_t* hist, int w_top, int w_bot, uint32_t target,
+                            uint32_t* res) {
+  const int lane = threadIdx.x & 31;
   uint32_t run = 0;
-  for (int gtop = w_top >> 2; gtop >= (w_bot >> 2); gtop -= TK_THREADS) {
-    const int gi = gtop - tid;
+  for (int ghi = w_top >> 2; ghi >= (w_bot >> 2); ghi -= 32) {
+    const int gi = ghi - lane;
     uint32_t c[8];
 #pragma unroll
     for (int i = 0; i < 8; i++) c[i] = 0u;
@@ -1147,9 +1150,15 @@ __device__ void local_suffix(const uint32_t* hist, int w_top, int w_bot, uint32_
     uint32_t tot = 0;
 #pragma unroll
     for (int i = 0; i < 8; i++) tot += c[i];
-    uint32_t total;
-    const uint32_t before = run + block_scan_total(tot, tmp, total);
-    if (before < target && target <= before + tot) {
+    uint32_t inc = tot;                     // lanes in descending digit order
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    const uint32_t before = run + inc - tot;
+    const bool hit = before < target && target <= before + tot;
+    if (hit) {
       uint32_t acc = before;
       int ti = 7;
 #pragma unroll
@@ -1161,11 +1170,10 @@ __device__ void local_suffix(const uint32_t* hist, int w_top, int w_bot, uint32_
       res[1] = acc;
       res[2] = 1;
     }
-    __syncthreads();
-    if (res[2]) break;
-    run += total;
+    if (__ballot_sync(0xffffffffu, hit)) return;
+    run += __shfl_sync(0xffffffffu, inc, 31);
   }
-  __syncthreads();
+  if (lane == 0) res[2] = 0;
 }
 
 // Radix-4 selection over 16-bit keys spread across the block, without atomics: each thread
@@ -1276,39 +1284,41 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
   const uint16_t* sr = reinterpret_cast<const uint16_t*>(scores) + row * (long long)Nc;
   const bool al = (reinterpret_cast<uintptr_t>(sr) & 15) == 0;
 
-  // ---- this thread's 16 group maxima (groups 16t .. 16t+15), kept in registers
+  // ---- this thread's 16 group summaries (groups 16t .. 16t+15) in shared memory: maxima
+  // (groups past the visible ones read as 0), second maxima, positions of the maxima
+  const int g0 = GM_GPT * tid;
   uint32_t gmr[GM_GPT / 2];
   {
-    const int g0 = GM_GPT * tid;
     const uint4* v = reinterpret_cast<const uint4*>(gmax + row * (long long)NGP + g0);
     uint4 a = make_uint4(0, 0, 0, 0), b = a;
-    if (g0 < ngv) { a = __ldg(v); b = __ldg(v + 1); }
+    if (g0 < ngv) {
+      a = __ldg(v);
+      b = __ldg(v + 1);
+      const long long o = row * (long long)NGP + g0;
+      cp_async16(&S.g2s[0][tid], g2nd + o);
+      cp_async16(&S.g2s[1][tid], g2nd + o + 8);
+      cp_async16(&S.gas[tid], garg + o);
+    }
+    cp_async_commit();
     gmr[0] = a.x; gmr[1] = a.y; gmr[2] = a.z; gmr[3] = a.w;
     gmr[4] = b.x; gmr[5] = b.y; gmr[6] = b.z; gmr[7] = b.w;
 #pragma unroll
-    for (int i = 0; i < GM_GPT; i++)   // groups past the visible ones do not exist
+    for (int i = 0; i < GM_GPT; i++)
       if (g0 + i >= ngv) gmr[i >> 1] &= (i & 1) ? 0x0000FFFFu : 0xFFFF0000u;
+    S.gms[0][tid] = make_uint4(gmr[0], gmr[1], gmr[2], gmr[3]);
+    S.gms[1][tid] = make_uint4(gmr[4], gmr[5], gmr[6], gmr[7]);
   }
   auto gm_of = [&](int i) { return (gmr[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu; };
-  // their second maxima and the positions of the maxima
-  uint32_t g2r[GM_GPT / 2], gar[GM_GPT / 4];
-  {
-    const int g0 = GM_GPT * tid;
-    uint4 a = make_uint4(0, 0, 0, 0), b2 = a, c = a;
-    if (g0 < ngv) {
-      const uint4* v2 = reinterpret_cast<const uint4*>(g2nd + row * (long long)NGP + g0);
-      a = __ldg(v2);
-      b2 = __ldg(v2 + 1);
-      c = __ldg(reinterpret_cast<const uint4*>(garg + row * (long long)NGP + g0));
-    }
-    g2r[0] = a.x; g2r[1] = a.y; g2r[2] = a.z; g2r[3] = a.w;
-    g2r[4] = b2.x; g2r[5] = b2.y; g2r[6] = b2.z; g2r[7] = b2.w;
-    gar[0] = c.x; gar[1] = c.y; gar[2] = c.z; gar[3] = c.w;
-  }
-  auto sec_of = [&](int i) { return (g2r[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu; };
-  auto arg_of = [&](int i) { return (gar[i >> 2] >> ((i & 3) * 8)) & 0xFu; };
+  // maximum and position of the maximum of group 16t+i, i dynamic
+  auto gm_sh = [&](int i) {
+    return uint32_t(reinterpret_cast<const uint16_t*>(&S.gms[i >> 3][tid])[i & 7]);
+  };
+  auto arg_sh = [&](int i) {
+    return uint32_t(reinterpret_cast<const uint8_t*>(&S.gas[tid])[i]) & 15u;
+  };
   static_assert(GM_WWORDS == 4 * TK_THREADS, "one uint4 of the candidate histogram per thread");
   reinterpret_cast<uint4*>(S.wc)[tid] = make_uint4(0, 0, 0, 0);
+  reinterpret_cast<uint4*>(S.wh)[tid] = make_uint4(0, 0, 0, 0);
   if (tid == 0) { S.ncand = 0u; S.npool = 0u; }
   // block: number of maxima and the largest (the row's largest visible key)
   uint32_t nz = 0, tmax = 0;
@@ -1337,123 +1347,131 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
 
   // ---- L: a lower bound of the row's k-th largest key.  The k-th largest group maximum is
   // one (the maxima are keys of k distinct groups); it is estimated from one maximum per
-  // thread (a 1/16 sample), taken a little low, and verified by counting the maxima >= the
-  // estimate.  If too few reach it, the exact k-th largest maximum is selected instead.
+  // thread (a 1/16 sample), taken a little low, and checked when the candidates are counted:
+  // if fewer than k keys reach it, the exact k-th largest maximum is selected instead.
   uint32_t L = 0u;
+  bool need_exact = false;
   if (S.res[5] >= (uint32_t)k) {
     const uint32_t ns = (uint32_t)min(TK_THREADS, (ngv + GM_GPT - 1) / GM_GPT);   // samples
     const uint32_t want = (uint32_t)(((unsigned long long)k * ns * 3) / (2ull * (uint32_t)ngv)) + 8u;
-    uint32_t est = 0u;
     if (want < ns) {
       const uint32_t sv = gm_of(0);             // group 16t: thread t's sample (0: none)
-      for (int w = tid; w < GM_WWORDS; w += TK_THREADS) S.wh[w] = 0u;
-      __syncthreads();
       if (sv != 0u && sv >= wb) atomicAdd(&S.wh[(sv - wb) >> 1], 1u << (((sv - wb) & 1) << 4));
       __syncthreads();
-      local_suffix(S.wh, int((Mx - wb) >> 1), 0, want, S.scan_tmp, S.res);
-      if (S.res[2]) {
-        est = S.res[0] + wb;
-        uint32_t cnt = 0;
-#pragma unroll
-        for (int i = 0; i < GM_GPT; i++) cnt += gm_of(i) >= est && gm_of(i) != 0u;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-        if (lane == 0) S.red[0][warp] = cnt;
-        __syncthreads();
-        if (warp == 0) {
-          uint32_t t = S.red[0][lane];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-          if (lane == 0) S.res[4] = t;
-        }
-        __syncthreads();
-        if (S.res[4] < (uint32_t)k) est = 0u;     // estimate too high
-      }
+      if (warp == 0) warp_suffix(S.wh, int((Mx - wb) >> 1), 0, want, S.res);
+      __syncthreads();
+      if (S.res[2]) L = S.res[0] + wb;
     }
-    if (est != 0u) {
-      L = est;
-    } else {
-      // exact: the k-th largest of all maxima (radix-4, no atomics)
+    need_exact = L == 0u;
+  }
+
+  uint32_t qm = 0, dm = 0;          // bit i: group 16t+i holds one candidate / two or more
+  uint32_t ndm = 0, pbase = 0;
+  bool inwin = false;               // every candidate key lies in the window
+  for (int pass = 0; pass < 2; pass++) {
+    if (need_exact) {
+      // the k-th largest of all maxima (radix-4, no atomics)
       uint32_t target = (uint32_t)k, ab = 0u, pmask = 0u;
+      L = 0u;
 #pragma unroll 1
       for (int shift = 12; shift >= 0; shift -= 4) {
         Digits4 c;
 #pragma unroll
         for (int i = 0; i < GM_GPT; i++) {
-          const uint32_t v = gm_of(i);
+          const uint32_t v = gm_sh(i);
           if (v != 0u && (v & pmask) == L) c.add((v >> shift) & 15u);
         }
         L |= radix4_reduce(c, target, ab, S.wcnt, S.res) << shift;
         pmask |= 15u << shift;
       }
     }
-  }
-
-  // ---- candidates: the visible keys >= L.  Thread t owns groups 16t .. 16t+15, in index
-  // order.  A group with one candidate gives it (key, position) from the summary; the scores
-  // of a group with more are copied into a pool slot (all copies in flight together) and its
-  // candidates listed there.  Every candidate key goes into the window histogram, and the
-  // block counts them.
-  const uint32_t L1 = max(L, 1u);   // key 0 marks an invisible entry
-  uint32_t qm = 0, dm = 0;          // bit i: group 16t+i holds one candidate / two or more
-  const bool inwin = L >= wb;       // every candidate key lies in the window
-#pragma unroll
-  for (int i = 0; i < GM_GPT; i++) {
-    const uint32_t mx = gm_of(i);
-    if (mx >= L1) {
-      if (sec_of(i) >= L) {
-        dm |= 1u << i;
-      } else {
-        qm |= 1u << i;
-        S.sc[i][tid] = (mx << 4) | arg_of(i);
-        if (inwin) atomicAdd(&S.wc[(mx - wb) >> 1], 1u << (((mx - wb) & 1) << 4));
-      }
-    }
-  }
-  uint32_t c = __popc(qm);
-  const uint32_t ndm = __popc(dm);
-  const uint32_t pbase = ndm ? atomicAdd(&S.npool, ndm) : 0u;
-  if (ndm && pbase + ndm <= GM_POOL) {
-    uint32_t sl = pbase;
-    for (uint32_t mm = dm; mm; mm &= mm - 1u, sl++) {
-      const int e0 = GM_G * (GM_GPT * tid + __ffs(mm) - 1);
-      if (al && e0 + GM_G <= nvis) {
-        cp_async16(&S.praw[sl][0], sr + e0);
-        cp_async16(&S.praw[sl][4], sr + e0 + 8);
-      } else {
-#pragma unroll
-        for (int w = 0; w < 8; w++)
-          S.praw[sl][w] = uint32_t(sr[min(e0 + 2 * w, nvis - 1)]) |
-                          (uint32_t(sr[min(e0 + 2 * w + 1, nvis - 1)]) << 16);
-      }
-    }
-    cp_async_commit();
+    // ---- candidates: the visible keys >= L.  Thread t owns groups 16t .. 16t+15, in index
+    // order.  A group with one candidate gives it (key, position) from the summary; the scores
+    // of a group with more are copied into a pool slot (all copies in flight together) and its
+    // candidates listed there.  Every candidate key goes into the window histogram, and the
+    // block counts them.
+    const uint32_t L1 = max(L, 1u);   // key 0 marks an invisible entry
+    inwin = L >= wb;
     cp_async_wait<0>();
-    sl = pbase;
-    for (uint32_t mm = dm; mm; mm &= mm - 1u, sl++) {
-      const int nv = nvis - GM_G * (GM_GPT * tid + __ffs(mm) - 1);   // visible: min(nv, 16)
-      uint32_t n = 0;
+    {
+      const uint4 m0 = S.gms[0][tid], m1 = S.gms[1][tid], s0 = S.g2s[0][tid], s1 = S.g2s[1][tid];
+      const uint32_t mw[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+      const uint32_t sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+      uint32_t qa = 0u, sa = 0u;
 #pragma unroll
-      for (int j = 0; j < GM_G; j++) {
-        const uint32_t key = ordered_key_bf16(uint16_t(S.praw[sl][j >> 1] >> ((j & 1) * 16)));
-        if (j < nv && key >= L1) {
+      for (int w = 0; w < 8; w++) {
+        qa |= (uint32_t((mw[w] & 0xFFFFu) >= L1) | (uint32_t((mw[w] >> 16) >= L1) << 1)) << (2 * w);
+        sa |= (uint32_t((sw[w] & 0xFFFFu) >= L) | (uint32_t((sw[w] >> 16) >= L) << 1)) << (2 * w);
+      }
+      dm = qa & sa;
+      qm = qa & ~sa;
+    }
+    uint32_t c = __popc(qm);
+    if (inwin) {
+      for (uint32_t mm = qm; mm; mm &= mm - 1u) {
+        const uint32_t d = gm_sh(__ffs(mm) - 1) - wb;
+        atomicAdd(&S.wc[d >> 1], 1u << ((d & 1) << 4));
+      }
+    }
+    ndm = __popc(dm);
+    pbase = ndm ? atomicAdd(&S.npool, ndm) : 0u;
+    if (ndm && pbase + ndm <= GM_POOL) {
+      uint32_t sl = pbase;
+      for (uint32_t mm = dm; mm; mm &= mm - 1u, sl++) {
+        const int e0 = GM_G * (g0 + __ffs(mm) - 1);
+        if (al && e0 + GM_G <= nvis) {
+          cp_async16(&S.praw[sl][0], sr + e0);
+          cp_async16(&S.praw[sl][4], sr + e0 + 8);
+        } else {
+#pragma unroll
+          for (int w = 0; w < 8; w++)
+            S.praw[sl][w] = uint32_t(sr[min(e0 + 2 * w, nvis - 1)]) |
+                            (uint32_t(sr[min(e0 + 2 * w + 1, nvis - 1)]) << 16);
+        }
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+      sl = pbase;
+      for (uint32_t mm = dm; mm; mm &= mm - 1u, sl++) {
+        // keys of the group in place, the mask of those >= L among the visible ones, then
+        // one pass over the set bits
+        const int nv = nvis - GM_G * (g0 + __ffs(mm) - 1);
+        uint32_t msk = 0u;
+#pragma unroll
+        for (int w = 0; w < 8; w++) {
+          const uint32_t kk = ordered_key_bf16x2(S.praw[sl][w]);
+          S.praw[sl][w] = kk;
+          msk |= (uint32_t((kk & 0xFFFFu) >= L1) | (uint32_t((kk >> 16) >= L1) << 1)) << (2 * w);
+        }
+        if (nv < GM_G) msk &= (1u << nv) - 1u;
+        uint32_t n = 0;
+        for (; msk; msk &= msk - 1u) {
+          const int j = __ffs(msk) - 1;
+          const uint32_t key = (S.praw[sl][j >> 1] >> ((j & 1) * 16)) & 0xFFFFu;
           S.pent[sl][n++] = (key << 4) | uint32_t(j);
           if (inwin) atomicAdd(&S.wc[(key - wb) >> 1], 1u << (((key - wb) & 1) << 4));
         }
+        S.pcnt[sl] = n;
+        c += n;
       }
-      S.pcnt[sl] = n;
-      c += n;
     }
-  }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-  if (lane == 0 && c) atomicAdd(&S.ncand, c);
-  __syncthreads();
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    if (lane == 0 && c) atomicAdd(&S.ncand, c);
+    __syncthreads();
+    if (S.ncand >= (uint32_t)k) break;
+    // the estimate was too high (an exact L always has k candidates): start over from it
+    __syncthreads();
+    reinterpret_cast<uint4*>(S.wc)[tid] = make_uint4(0, 0, 0, 0);
+    if (tid == 0) { S.ncand = 0u; S.npool = 0u; }
+    need_exact = true;
+  }
 
   uint32_t T = 0u, above = 0u;
   // u16 digit counts cannot overflow while the row has fewer than 2^16 candidates
   if (inwin && S.ncand < 65536u && S.npool <= (uint32_t)GM_POOL) {
-    local_suffix(S.wc, int((Mx - wb) >> 1), int((L - wb) >> 1), (uint32_t)k, S.scan_tmp, S.res);
+    if (warp == 0) warp_suffix(S.wc, int((Mx - wb) >> 1), int((L - wb) >> 1), (uint32_t)k, S.res);
+    __syncthreads();
     if (S.res[2]) {
       T = S.res[0] + wb;
       above = S.res[1];
@@ -1461,7 +1479,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
       // ---- emission in index order: one packed (ties, above) scan over the threads
       uint32_t gt = 0, eq = 0;
       for (uint32_t mm = qm; mm; mm &= mm - 1u) {
-        const uint32_t key = S.sc[__ffs(mm) - 1][tid] >> 4;
+        const uint32_t key = gm_sh(__ffs(mm) - 1);
         gt += key > T;
         eq += key == T;
       }
@@ -1493,7 +1511,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
         for (uint32_t mm = qm | dm; mm; mm &= mm - 1u) {
           const int i = __ffs(mm) - 1, e0 = GM_G * (GM_GPT * tid + i);
           if ((qm >> i) & 1u) {
-            place(S.sc[i][tid], e0);
+            place((gm_sh(i) << 4) | arg_sh(i), e0);
           } else {
             const uint32_t n = S.pcnt[sl];
             for (uint32_t e = 0; e < n; e++) place(S.pent[sl][e], e0);
@@ -1513,11 +1531,11 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
   {
     uint32_t nq = 0;
 #pragma unroll
-    for (int i = 0; i < GM_GPT; i++) nq += (gm_of(i) != 0u && gm_of(i) >= L);
+    for (int i = 0; i < GM_GPT; i++) nq += (gm_sh(i) != 0u && gm_sh(i) >= L);
     uint32_t o = block_scan_total(nq, S.scan_tmp, ngc);
 #pragma unroll
     for (int i = 0; i < GM_GPT; i++)
-      if (gm_of(i) != 0u && gm_of(i) >= L) S.list[o++] = uint16_t(GM_GPT * tid + i);
+      if (gm_sh(i) != 0u && gm_sh(i) >= L) S.list[o++] = uint16_t(GM_GPT * tid + i);
   }
   __syncthreads();
   {
