@@ -71,8 +71,8 @@ def max_over_ranks(x, world, device):
 # DRAM traffic of one indexer launch as measured once with ncu (dram__bytes_read.sum +
 # dram__bytes_write.sum over 16 sequences; profiles/indexer_mxfp4_decode_B16.md), per sequence.
 # It is reported only while the indexer source is the one that was profiled.
-INDEXER_TRAFFIC = {"source_sha256_16": "b2c672a212a5db8a",
-                   "bytes_per_seq": (142.650624e6 + 6.076160e6) / 16}
+INDEXER_TRAFFIC = {"source_sha256_16": "c86a27bf044c3ace",
+                   "bytes_per_seq": (142.651904e6 + 5.133568e6) / 16}
 
 
 def indexer_traffic(B):
