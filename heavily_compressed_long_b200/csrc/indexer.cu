@@ -590,6 +590,13 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
         // (with 16 epilogue warps the registers do not allow the look-ahead; four warps per
         // scheduler hide the load latency instead)
         constexpr int PD = EPI >= 16 ? 1 : 2;
+        // a warp whose 32 keys are visible to all of its queries (and in range) stores without
+        // per-score checks
+        int lim = p.Nc;
+#pragma unroll
+        for (int g = 0; g < QPER; g++) lim = min(lim, sNvis[qbeg + g]);
+        const int kw = tile0 * KEYS + quarter * 32;
+        const bool bf = p.score_fmt != HCL_FP32;
         uint32_t r[PD][TPS][16];
         if (PD == 2) {
 #pragma unroll
@@ -628,7 +635,11 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
             const float sc = __uint_as_float(uint32_t(acc)) + __uint_as_float(uint32_t(acc >> 32));
             const int tq = t0 + q;
             const int key = (tile0 + t) * KEYS + quarter * 32 + lane;
-            if (tq < p.Tq && key < p.Nc) {
+            if (kw + t * KEYS + 32 <= lim) {
+              const size_t o = ((size_t)b * p.Tq + tq) * p.Nc + key;
+              if (bf) static_cast<__nv_bfloat16*>(p.scores)[o] = __float2bfloat16_rn(sc);
+              else static_cast<float*>(p.scores)[o] = sc;
+            } else if (tq < p.Tq && key < p.Nc) {
               const float v = key < sNvis[q] ? sc : -INFINITY;
               const size_t o = ((size_t)b * p.Tq + tq) * p.Nc + key;
               if (p.score_fmt == HCL_FP32) static_cast<float*>(p.scores)[o] = v;
