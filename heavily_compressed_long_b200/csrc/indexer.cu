@@ -561,6 +561,20 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
       }
     };
 
+    // prefill with several key tiles per stage: this thread's queries are the same in every
+    // stage, so their (halved) weights stay in registers
+    constexpr bool PRE_MT = KIND == 0 && TPS > 1 && QT > 1;
+    float wreg[PRE_MT ? QPER : 1][16];
+    if constexpr (PRE_MT) {
+#pragma unroll
+      for (int g = 0; g < QPER; g++)
+#pragma unroll
+        for (int h = 0; h < 16; h += 4) {
+          const float4 w4 = *reinterpret_cast<const float4*>(sW + (qbeg + g) * HP + h);
+          wreg[g][h] = w4.x; wreg[g][h + 1] = w4.y; wreg[g][h + 2] = w4.z; wreg[g][h + 3] = w4.w;
+        }
+    }
+
     for (int i = 0; i < nstages; i++) {
       const int a = i % NACC;
       bool ok = mbar_wait(&accf[a], (i / NACC) & 1, p.limit, sAbort);
@@ -584,8 +598,8 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
 #pragma unroll
         for (int t = 0; t < TPS; t++) emit4(tile0 + t, r[t]);
       } else if constexpr (KIND == 0 && TPS > 1 && QT > 1) {
-        // prefill with several key tiles per stage: query by query, the weights are read once
-        // and applied to this thread's key in every tile of the stage; the next query's
+        // prefill with several key tiles per stage: query by query, the weights (registers) are
+        // applied to this thread's key in every tile of the stage; the next query's
         // accumulator columns are loaded while this one is reduced
         // (with 16 epilogue warps the registers do not allow the look-ahead; four warps per
         // scheduler hide the load latency instead)
@@ -609,8 +623,6 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
 #pragma unroll
             for (int t = 0; t < TPS; t++) tmem_ld16(tacc + t * N + q * HP, r[0][t]);
           }
-          const float4* wq = reinterpret_cast<const float4*>(sW + q * HP);
-          const float4 w0 = wq[0], w1 = wq[1], w2 = wq[2], w3 = wq[3];
           tmem_ld_wait();
           if (PD == 2 && g + 1 < QPER) {
 #pragma unroll
@@ -623,8 +635,7 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
           for (int t = 0; t < TPS; t++) {
             const uint32_t* rr = r[g % PD][t];
             unsigned long long acc = 0ull;
-            const float wv[16] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w,
-                                  w2.x, w2.y, w2.z, w2.w, w3.x, w3.y, w3.z, w3.w};
+            const float* wv = wreg[g];
             // w * relu(x) == (w/2) * (x + |x|) exactly (x + |x| is 2x or 0): an add with an
             // absolute-value operand on the FMA pipe instead of a max on the ALU pipe
 #pragma unroll
