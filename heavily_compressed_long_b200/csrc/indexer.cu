@@ -28,6 +28,8 @@
 #include <algorithm>
 #include <cstring>
 
+#include <type_traits>
+
 #include "hcl_common.cuh"
 #include "hcl_internal.h"
 #include "mxfp4.cuh"
@@ -106,6 +108,11 @@ __device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigne
                                                    unsigned long long c) {
   unsigned long long d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
 
@@ -562,10 +569,14 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
     };
 
     // prefill with several key tiles per stage: this thread's queries are the same in every
-    // stage, so their (halved) weights stay in registers
+    // stage, so their (halved) weights stay in registers, and so does the number of keys that
+    // all of them see (lim)
     constexpr bool PRE_MT = KIND == 0 && TPS > 1 && QT > 1;
     float wreg[PRE_MT ? QPER : 1][16];
+    int lim = p.Nc;
     if constexpr (PRE_MT) {
+#pragma unroll
+      for (int g = 0; g < QPER; g++) lim = min(lim, sNvis[qbeg + g]);
 #pragma unroll
       for (int g = 0; g < QPER; g++)
 #pragma unroll
@@ -599,65 +610,58 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
         for (int t = 0; t < TPS; t++) emit4(tile0 + t, r[t]);
       } else if constexpr (KIND == 0 && TPS > 1 && QT > 1) {
         // prefill with several key tiles per stage: query by query, the weights (registers) are
-        // applied to this thread's key in every tile of the stage; the next query's
-        // accumulator columns are loaded while this one is reduced
-        // (with 16 epilogue warps the registers do not allow the look-ahead; four warps per
-        // scheduler hide the load latency instead)
-        constexpr int PD = EPI >= 16 ? 1 : 2;
-        // a warp whose 32 keys are visible to all of its queries (and in range) stores without
-        // per-score checks
-        int lim = p.Nc;
-#pragma unroll
-        for (int g = 0; g < QPER; g++) lim = min(lim, sNvis[qbeg + g]);
+        // applied to this thread's key in every tile of the stage (with 16 epilogue warps the
+        // registers do not allow loading the next query's columns ahead; four warps per
+        // scheduler hide the load latency instead).  A stage whose keys all of this warp's
+        // queries see, with bf16 scores, takes a body without per-score checks.
+        constexpr bool ILP2 = true;    // two accumulator chains per (query, tile)
         const int kw = tile0 * KEYS + quarter * 32;
         const bool bf = p.score_fmt != HCL_FP32;
-        uint32_t r[PD][TPS][16];
-        if (PD == 2) {
+        auto stage = [&](auto fast_c) {
+          constexpr bool FAST = decltype(fast_c)::value;
 #pragma unroll
-          for (int t = 0; t < TPS; t++) tmem_ld16(tacc + t * N + qbeg * HP, r[0][t]);
-        }
+          for (int g = 0; g < QPER; g++) {
+            const int q = qbeg + g;
+            uint32_t r[TPS][16];
 #pragma unroll
-        for (int g = 0; g < QPER; g++) {
-          const int q = qbeg + g;
-          if (PD == 1) {
-#pragma unroll
-            for (int t = 0; t < TPS; t++) tmem_ld16(tacc + t * N + q * HP, r[0][t]);
-          }
-          tmem_ld_wait();
-          if (PD == 2 && g + 1 < QPER) {
-#pragma unroll
-            for (int t = 0; t < TPS; t++) tmem_ld16(tacc + t * N + (q + 1) * HP, r[(g + 1) % PD][t]);
-          } else if (g + 1 == QPER) {
-            tc_fence_before();
-            mbar_arrive(&acce[a]);
-          }
-#pragma unroll
-          for (int t = 0; t < TPS; t++) {
-            const uint32_t* rr = r[g % PD][t];
-            unsigned long long acc = 0ull;
-            const float* wv = wreg[g];
-            // w * relu(x) == (w/2) * (x + |x|) exactly (x + |x| is 2x or 0): an add with an
-            // absolute-value operand on the FMA pipe instead of a max on the ALU pipe
-#pragma unroll
-            for (int h = 0; h < HP; h += 2) {
-              const float x0 = __uint_as_float(rr[h]), x1 = __uint_as_float(rr[h + 1]);
-              acc = fma2(pack2(wv[h], wv[h + 1]), pack2(x0 + fabsf(x0), x1 + fabsf(x1)), acc);
+            for (int t = 0; t < TPS; t++) tmem_ld16(tacc + t * N + q * HP, r[t]);
+            tmem_ld_wait();
+            if (g + 1 == QPER) {
+              tc_fence_before();
+              mbar_arrive(&acce[a]);
             }
-            const float sc = __uint_as_float(uint32_t(acc)) + __uint_as_float(uint32_t(acc >> 32));
-            const int tq = t0 + q;
-            const int key = (tile0 + t) * KEYS + quarter * 32 + lane;
-            if (kw + t * KEYS + 32 <= lim) {
-              const size_t o = ((size_t)b * p.Tq + tq) * p.Nc + key;
-              if (bf) static_cast<__nv_bfloat16*>(p.scores)[o] = __float2bfloat16_rn(sc);
-              else static_cast<float*>(p.scores)[o] = sc;
-            } else if (tq < p.Tq && key < p.Nc) {
-              const float v = key < sNvis[q] ? sc : -INFINITY;
-              const size_t o = ((size_t)b * p.Tq + tq) * p.Nc + key;
-              if (p.score_fmt == HCL_FP32) static_cast<float*>(p.scores)[o] = v;
-              else static_cast<__nv_bfloat16*>(p.scores)[o] = __float2bfloat16_rn(v);
+            const size_t orow = ((size_t)b * p.Tq + t0 + q) * p.Nc;
+#pragma unroll
+            for (int t = 0; t < TPS; t++) {
+              const float* wv = wreg[g];
+              // w * relu(x) == (w/2) * (x + |x|) exactly (x + |x| is 2x or 0): an add with an
+              // absolute-value operand on the FMA pipe instead of a max on the ALU pipe
+              unsigned long long acc0 = 0ull, acc1 = 0ull;
+#pragma unroll
+              for (int h = 0; h < HP; h += 4) {
+                const float x0 = __uint_as_float(r[t][h]), x1 = __uint_as_float(r[t][h + 1]);
+                const float x2 = __uint_as_float(r[t][h + 2]), x3 = __uint_as_float(r[t][h + 3]);
+                acc0 = fma2(pack2(wv[h], wv[h + 1]), pack2(x0 + fabsf(x0), x1 + fabsf(x1)), acc0);
+                if (ILP2)
+                  acc1 = fma2(pack2(wv[h + 2], wv[h + 3]), pack2(x2 + fabsf(x2), x3 + fabsf(x3)), acc1);
+                else
+                  acc0 = fma2(pack2(wv[h + 2], wv[h + 3]), pack2(x2 + fabsf(x2), x3 + fabsf(x3)), acc0);
+              }
+              const unsigned long long acc = ILP2 ? add2(acc0, acc1) : acc0;
+              const float sc = __uint_as_float(uint32_t(acc)) + __uint_as_float(uint32_t(acc >> 32));
+              const int key = (tile0 + t) * KEYS + quarter * 32 + lane;
+              if constexpr (FAST) {
+                static_cast<__nv_bfloat16*>(p.scores)[orow + key] = __float2bfloat16_rn(sc);
+              } else if (t0 + q < p.Tq && key < p.Nc) {
+                const float v = key < sNvis[q] ? sc : -INFINITY;
+                if (!bf) static_cast<float*>(p.scores)[orow + key] = v;
+                else static_cast<__nv_bfloat16*>(p.scores)[orow + key] = __float2bfloat16_rn(v);
+              }
             }
           }
-        }
+        };
+        if (bf && kw + (TPS - 1) * KEYS + 32 <= lim) stage(std::integral_constant<bool, true>{});
+        else stage(std::integral_constant<bool, false>{});
       } else if (ALL_AT_ONCE) {
         uint32_t r[TPS * QPER][16];
 #pragma unroll
