@@ -1051,7 +1051,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------------------
-// Decode selection from group maxima (inside the fused decode step, bf16 scores).  The indexer
+// Decode selection from group summaries (inside the fused decode step, bf16 scores).  The indexer
 // also writes, for every group of 16 entries, a summary of its visible scores as
 // order-preserving keys: the largest, the second largest and the position of the largest.  The
 // k-th largest of the maxima, L, is a lower bound of the row's k-th largest score (the maxima

@@ -386,17 +386,23 @@ def test_invalid_arguments_rejected(hcl):
 
 
 # =========================================================================================
-# fused decode step: MXFP4 keys + bf16 scores select from the indexer's per-16-entry maxima
+# fused decode step: MXFP4 keys + bf16 scores select from the indexer's per-16-entry summaries
 
-@pytest.mark.parametrize("B,Nc,k,nvis,ties", [
-    (3, 70000, 1024, (70000, 5000, 700), False),   # the last row has fewer than k visible
-    (2, 40000, 512, (40000, 39999), True),          # many equal scores, visibility mid-group
-    (1, 4096, 1024, (1030,), True),                 # just above k visible
-    (2, 262144, 1024, (262144, 131075), False),     # full decode length
+@pytest.mark.parametrize("B,Nc,k,nvis,ties,plant", [
+    (3, 70000, 1024, (70000, 5000, 700), False, None),   # the last row has fewer than k visible
+    (2, 40000, 512, (40000, 39999), True, None),          # many equal scores, visibility mid-group
+    (1, 4096, 1024, (1030,), True, None),                 # just above k visible
+    (2, 262144, 1024, (262144, 131075), False, None),     # full decode length
+    # keys doubled in the groups the top-k samples (every 16th group) of the first P*16
+    # groups: the sampled lower bound overshoots, so the exact k-th largest maximum is taken;
+    # P = 200 keeps the multi-candidate groups within the shared-memory pool, P = 1024 does not
+    (1, 262144, 1024, (262144,), False, (200, 2.0)),
+    (1, 262144, 1024, (262144,), False, (1024, 2.0)),
 ])
-def test_decode_step_group_maxima(hcl, B, Nc, k, nvis, ties):
-    """The fused step's top-k (group maxima lower bound) against the oracle's top-k of the very
-    scores the separate calls produce, and the fused step against the separate calls bitwise."""
+def test_decode_step_group_maxima(hcl, B, Nc, k, nvis, ties, plant):
+    """The fused step's top-k (group summaries lower bound) against the oracle's top-k of the
+    very scores the separate calls produce, and the fused step against the separate calls
+    bitwise."""
     from heavily_compressed_long_b200.api import HCL_BF16, HCL_MXFP4, KV
     from heavily_compressed_long_b200.pipeline import CsaDecode
     H, HI, W, d = 16, 16, 128, 128
@@ -404,6 +410,13 @@ def test_decode_step_group_maxima(hcl, B, Nc, k, nvis, ties):
     kb = rbf16(B, Nc, 64)
     if ties:                                   # few distinct key rows -> heavily tied scores
         kb = kb[:, RNG.integers(0, 37, Nc)]
+    if plant is not None:
+        P, gain = plant
+        e = np.arange(Nc)
+        sampled = torch.from_numpy((((e // 16) % 16) == 0) & (e < 256 * P))
+        kf = kb.float()
+        kf[:, sampled] *= gain                 # a power of two: exact in bf16 and MXFP4
+        kb = kf.to(torch.bfloat16)
     kp = torch.empty(B, Nc, 32, dtype=torch.uint8, device="cuda")
     ks = torch.empty(B, Nc, 2, dtype=torch.uint8, device="cuda")
     hcl.hcl_quant_mxfp4(cuda(kb), kp, ks)
