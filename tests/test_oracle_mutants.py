@@ -8,6 +8,7 @@ only, on the CPU; the real oracle is untouched.
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 import pytest
 
@@ -47,23 +48,60 @@ MUTANTS = {
     "hca_uses_overlap_visibility": ("long nvis = or_num_visible(q_pos[row], mh, Nh);",
                                     "long nvis = or_num_visible(q_pos[row] + mh, mh, Nh);"),
     "value_weights_unnormalised": ("double p = exp(z[j] - zmax) / den;", "double p = exp(z[j] - zmax);"),
+    "compress_pools_gate_not_value": ("num += e * or_bf16_to_f64(x[(b * L + t) * d + ch]);",
+                                      "num += e * or_bf16_to_f64(g[(b * L + t) * d + ch]);"),
+    "compress_unnormalised": ("o[ch] = (den > 0.0) ? num / den : 0.0;", "o[ch] = num;"),
+    "compress_bias_dropped": (" + (double)bias[j];", ";"),
+    "index_abs_instead_of_relu": ("(dot > 0.0 ? dot : 0.0)", "(dot > 0.0 ? dot : -dot)"),
+    "visibility_counts_incomplete_entry": ("long v = (p + 1) / m;", "long v = (p + m) / m;"),
+    "topk_output_in_score_order": ("qsort(out, take, sizeof(int), by_index);", "(void)by_index;"),
+    "topk_takes_lowest_scores": ("if (a->s > b->s) return -1;\n    if (a->s < b->s) return 1;",
+                                 "if (a->s > b->s) return 1;\n    if (a->s < b->s) return -1;"),
+    "topk_pads_with_zero": ("for (long j = take; j < k; j++) out[j] = -1;",
+                            "for (long j = take; j < k; j++) out[j] = 0;"),
+    "csa_drops_last_selected": ("for (int j = 0; j < k; j++) {\n                    int e = idx[row * k + j];",
+                                "for (int j = 0; j < k - 1; j++) {\n                    int e = idx[row * k + j];"),
+    "hca_drops_last_visible": ("for (long i = 0; i < nvis; i++, n++) {", "for (long i = 1; i < nvis; i++, n++) {"),
+    "fp8_rope_half_from_nope_dims": ("rope[r * h + c] = x[h + c];", "rope[r * h + c] = x[c];"),
+    "fp8_amax_over_all_dims": ("for (int c = 0; c < h; c++) {\n            float v = fabsf(",
+                               "for (int c = 0; c < 2 * h; c++) {\n            float v = fabsf("),
+    "mxfp4_amax_signed": ("double a = fabs(or_bf16_to_f64(v[c]));", "double a = or_bf16_to_f64(v[c]);"),
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_mutant(name, tmp_path):
+def _run_mutant(name, workdir):
+    """Build the oracle with mutant `name` planted and run the pin suite against it; returns
+    (pytest exit code, end of its output)."""
     old, new = MUTANTS[name]
     src = open(SRC).read()
-    assert src.count(old) >= 1, f"mutation site for {name} not found"
-    mutated = src.replace(old, new)
-    csrc = tmp_path / "mutant.c"
-    csrc.write_text(mutated)
-    so = tmp_path / "libmutant.so"
-    sys.path.insert(0, ROOT)
+    if src.count(old) < 1:
+        return None, f"mutation site for {name} not found"
+    csrc = os.path.join(workdir, name + ".c")
+    with open(csrc, "w") as fh:
+        fh.write(src.replace(old, new))
+    so = os.path.join(workdir, "lib" + name + ".so")
     from oracle.build import build_oracle
-    build_oracle(force=True, src=str(csrc), out=str(so))
-    env = dict(os.environ, HCL_ORACLE_LIB=str(so), PYTHONPATH=ROOT)
+    build_oracle(force=True, src=csrc, out=so)
+    env = dict(os.environ, HCL_ORACLE_LIB=so, PYTHONPATH=ROOT, OMP_NUM_THREADS="2")
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
-                       env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
-    assert r.returncode != 0, f"no pin caught mutant {name}:\n{r.stdout[-2000:]}"
+                       env=env, cwd=ROOT, capture_output=True, text=True, timeout=900)
+    return r.returncode, r.stdout[-2000:]
+
+
+@pytest.fixture(scope="module")
+def mutant_results(tmp_path_factory):
+    """Every mutant's pin run, several at a time (each run is a separate process)."""
+    sys.path.insert(0, ROOT)
+    workdir = str(tmp_path_factory.mktemp("mutants"))
+    workers = max(1, min(8, (os.cpu_count() or 2) // 2))
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        futs = {name: ex.submit(_run_mutant, name, workdir) for name in sorted(MUTANTS)}
+        return {name: f.result() for name, f in futs.items()}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, mutant_results):
+    code, out = mutant_results[name]
+    assert code is not None, out
+    assert code != 0, f"no pin caught mutant {name}:\n{out}"
