@@ -218,7 +218,11 @@ HCL_API hcl_status_t hcl_hca_dense_attn(const void* q, int B, int Tq, int H, int
  * quantised (MXFP4 operands only), scored against all entries, the top-k kept, and
  * attention run over them plus the window -- a4 -> a5 -> a6 enqueued back to back on
  * `stream`.  Arguments as in the individual calls; qI_bf16 is the unquantised bf16 index
- * query [B, 1, HI, dI]; Tq == 1.  ws: hcl_csa_decode_step_workspace_bytes() bytes.
+ * query [B, 1, HI, dI]; Tq == 1.  ws: hcl_csa_decode_step_workspace_bytes() bytes; it holds
+ * the scores and, with MXFP4 operands and bf16 scores, a 5-byte summary per 16-entry group
+ * (largest and second largest score as order-preserving keys, position of the largest) that
+ * the indexer writes and the top-k reads instead of most of the scores.  The workspace is
+ * scratch owned by the caller; its contents after the call are unspecified.
  */
 HCL_API size_t hcl_csa_decode_step_workspace_bytes(int B, int H, int HI, int Nc, int k, int W,
                                            int op_fmt, int score_fmt);
