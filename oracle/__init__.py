@@ -65,6 +65,7 @@ def _declare(L):
     L.or_hca_attn.restype = None
     L.or_quant_kv_fp8.argtypes = [P, LG, I, P, P, P]; L.or_quant_kv_fp8.restype = None
     L.or_quant_mxfp4.argtypes = [P, LG, I, P, P]; L.or_quant_mxfp4.restype = None
+    L.or_rmsnorm.argtypes = [P, LG, I, P, D, P]; L.or_rmsnorm.restype = None
 
 
 # ------------------------------------------------------------------------------------------
@@ -220,6 +221,19 @@ def hca_attn(q, kvh: KV, Nh, mh, raw: KV, W, q_pos, scale=None, sink=None):
     lib().or_hca_attn(_p(q), B, Tq, H, d, *kvh.args(), Nh, mh, *raw.args(), W, _p(q_pos),
                       scale, _p(sink), _p(o), _p(lse))
     return o, lse
+
+
+def rmsnorm(x, gamma=None, eps=1e-6):
+    """RMSNorm over the last axis in fp64: x / sqrt(mean(x^2) + eps) * gamma.  x: fp64, or
+    bf16 (uint16 bits / torch bfloat16), any leading shape; gamma fp32 [d] or None."""
+    a = _np(x)
+    xd = dequant_bf16(a) if a.dtype == np.uint16 else np.ascontiguousarray(a, dtype=np.float64)
+    d = xd.shape[-1]
+    rows = xd.size // d if d else 0
+    out = np.empty_like(xd)
+    g = _np(gamma, np.float32)
+    lib().or_rmsnorm(_p(xd), rows, d, _p(g), float(eps), _p(out))
+    return out
 
 
 def quant_kv_fp8(kv):

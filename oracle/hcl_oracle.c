@@ -457,6 +457,26 @@ void or_hca_attn(const uint16_t *q, int B, int Tq, int H, int d,
 }
 
 /* ------------------------------------------------------------------------------------ */
+/* RMSNorm of queries and compressed entries                                              */
+
+/* The attention normalises its queries and its KV entries with RMSNorm, which is why no
+ * separate QK-Norm is needed                                            [Tripbot §5].
+ * Per row of d values: out_c = x_c / sqrt(mean_c(x_c^2) + eps) * gamma_c (gamma NULL: 1).
+ * x, out: fp64 [rows, d] (out may alias x). */
+void or_rmsnorm(const double *x, long rows, int d, const float *gamma, double eps, double *out)
+{
+#pragma omp parallel for schedule(static)
+    for (long r = 0; r < rows; r++) {
+        const double *xr = x + r * d;
+        double ss = 0.0;
+        for (int c = 0; c < d; c++) ss += xr[c] * xr[c];
+        double inv = 1.0 / sqrt(ss / d + eps);
+        double *o = out + r * d;
+        for (int c = 0; c < d; c++) o[c] = xr[c] * inv * (gamma ? (double)gamma[c] : 1.0);
+    }
+}
+
+/* ------------------------------------------------------------------------------------ */
 /* a3: cache quantisers                                                                   */
 
 /* Split KV row: RoPE dims (the last d/2) stay bf16; the other d/2 dims are stored as E4M3

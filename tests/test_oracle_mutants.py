@@ -66,6 +66,10 @@ MUTANTS = {
     "fp8_amax_over_all_dims": ("for (int c = 0; c < h; c++) {\n            float v = fabsf(",
                                "for (int c = 0; c < 2 * h; c++) {\n            float v = fabsf("),
     "mxfp4_amax_signed": ("double a = fabs(or_bf16_to_f64(v[c]));", "double a = or_bf16_to_f64(v[c]);"),
+    "rmsnorm_eps_outside_sqrt": ("double inv = 1.0 / sqrt(ss / d + eps);",
+                                 "double inv = 1.0 / (sqrt(ss / d) + eps);"),
+    "rmsnorm_sum_not_mean": ("double inv = 1.0 / sqrt(ss / d + eps);", "double inv = 1.0 / sqrt(ss + eps);"),
+    "rmsnorm_gamma_ignored": ("(gamma ? (double)gamma[c] : 1.0)", "1.0"),
 }
 
 

@@ -585,3 +585,47 @@ def test_hca_visibility_and_empty(orc):
     z = f64(ent[0, :2]) @ f64(q[0, 2, 0]) / math.sqrt(d)
     p = np.exp(z - z.max()) / np.exp(z - z.max()).sum()
     assert np.allclose(o[0, 2, 0], p @ f64(ent[0, :2]), atol=1e-13)  # entries 0, 1 at p=300
+
+
+# -----------------------------------------------------------------------------------------
+# RMSNorm of queries and entries [Tripbot §5]: hand values, identities, and torch's own
+# RMSNorm as an independent implementation.
+
+def test_rmsnorm_hand_values(orc):
+    # x = (3, 4): mean of squares 12.5
+    out = orc.rmsnorm(np.array([[3.0, 4.0]]), eps=0.0)
+    assert np.allclose(out, np.array([[3.0, 4.0]]) / math.sqrt(12.5), rtol=0, atol=1e-15)
+    # a constant row of 1e-3 with eps = 1e-6: mean square equals eps -> 1e-3 / sqrt(2e-6)
+    out = orc.rmsnorm(np.full((1, 128), 1e-3), eps=1e-6)
+    assert np.allclose(out, 1.0 / math.sqrt(2.0), rtol=1e-14, atol=0)
+    # a zero row stays zero (eps keeps the denominator finite)
+    assert np.array_equal(orc.rmsnorm(np.zeros((2, 64))), np.zeros((2, 64)))
+
+
+def test_rmsnorm_identities(orc):
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((5, 128))
+    y = orc.rmsnorm(x, eps=0.0)
+    # unit root-mean-square per row, direction kept, invariant to a positive scale
+    assert np.allclose(np.sqrt((y * y).mean(-1)), 1.0, rtol=1e-14)
+    assert np.allclose(y / np.linalg.norm(y, axis=-1, keepdims=True),
+                       x / np.linalg.norm(x, axis=-1, keepdims=True), rtol=1e-13)
+    assert np.allclose(orc.rmsnorm(7.5 * x, eps=0.0), y, rtol=1e-13)
+    # gamma multiplies per channel
+    gamma = rng.random(128).astype(np.float32) + 0.5
+    assert np.allclose(orc.rmsnorm(x, gamma, eps=0.0), y * gamma.astype(np.float64), rtol=1e-14)
+    # rows are independent
+    assert np.allclose(orc.rmsnorm(x[2:3], eps=0.0), y[2:3], rtol=0, atol=0)
+
+
+def test_rmsnorm_against_torch(orc):
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((3, 4, 128)) * 3.0
+    gamma = (rng.random(128) + 0.25).astype(np.float32)
+    want = torch.nn.functional.rms_norm(torch.from_numpy(x), (128,),
+                                        torch.from_numpy(gamma.astype(np.float64)), eps=1e-6)
+    got = orc.rmsnorm(x, gamma, eps=1e-6)
+    assert np.allclose(got, want.numpy(), rtol=1e-13, atol=1e-15)
+    # bf16 input (as the queries and entries are stored) is read exactly
+    xb = gen.to_bf16(x.astype(np.float32))
+    assert np.allclose(orc.rmsnorm(xb, gamma), orc.rmsnorm(xb.double().numpy(), gamma), rtol=0, atol=0)
