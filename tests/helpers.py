@@ -33,8 +33,8 @@ def bf16_ulp(x):
 
 
 def bf16_out_ratio(gpu, ref, rel=1e-3):
-    """Worst ratio of |gpu - ref| to the bf16-output allowance: the benchmark spec's fp32
-    tolerance (rel, norm-wise per row) plus one bf16 ulp of ref for the output rounding.
+    """Worst ratio of |gpu - ref| to the bf16-output allowance: the fp32 score tolerance
+    (rel, norm-wise per row) plus one bf16 ulp of ref for the output rounding.
     <= 1 passes.  -inf entries must match exactly."""
     g = np.asarray(gpu, np.float64)
     r = np.asarray(ref, np.float64)
