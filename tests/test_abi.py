@@ -97,3 +97,14 @@ def test_workspace_queries(libhcl):
     assert L.hcl_csa_sparse_attn_workspace_bytes(1, 4096, 64, 1024, 128) == 0
     assert L.hcl_csa_decode_step_workspace_bytes(8, 128, 16, 262144, 1024, 128,
                                                  libhcl.HCL_MXFP4, libhcl.HCL_BF16) > 8 * 262144 * 2
+    # MXFP4 keys + bf16 scores: the workspace also holds 5 bytes per 16-entry group of every row
+    # (largest, second largest, position of the largest) for the top-k; fp32 scores do not
+    for Nc in (262144, 70000, 4096):
+        ngp = ((Nc + 15) // 16 + 15) // 16 * 16
+        with_sum = L.hcl_csa_decode_step_workspace_bytes(8, 128, 16, Nc, 1024, 128,
+                                                         libhcl.HCL_MXFP4, libhcl.HCL_BF16)
+        scores_only = 8 * Nc * 2 + 8 * 1024 * 4
+        assert with_sum >= scores_only + 8 * ngp * 5
+    fp32 = L.hcl_csa_decode_step_workspace_bytes(8, 128, 16, 262144, 1024, 128,
+                                                 libhcl.HCL_MXFP4, libhcl.HCL_FP32)
+    assert fp32 >= 8 * 262144 * 4 and fp32 < 8 * 262144 * 4 + 8 * 16384 * 5
