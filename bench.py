@@ -68,9 +68,10 @@ def max_over_ranks(x, world, device):
     return float(t.item())
 
 
-# DRAM traffic of one indexer launch as measured once with ncu (dram__bytes_read.sum +
-# dram__bytes_write.sum over 16 sequences; profiles/indexer_mxfp4_decode_B16.md), per sequence.
-# It is reported only while the indexer source is the one that was profiled.
+# DRAM traffic of one decode indexer launch as measured once with ncu (dram__bytes_read.sum +
+# dram__bytes_write.sum of one launch over 16 sequences, `--kernel indexer --batch 16`), per
+# sequence.  It is reported only while the indexer source is byte-identical to the source that
+# was profiled (its hash below); after any change it is null until the next capture.
 INDEXER_TRAFFIC = {"source_sha256_16": "c86a27bf044c3ace",
                    "bytes_per_seq": (142.651904e6 + 5.133568e6) / 16}
 
@@ -509,6 +510,84 @@ def run_prefill_indexer(args, local_rank):
                       "scores_bytes": Tq * Nc * 2}), flush=True)
 
 
+def run_hca_shape_micro(args, local_rank):
+    """The compressors and the HCA prefill attention alone on the HCA workload's shapes (4
+    sequences x 65536 raw tokens; 2048 queries x 16 heads per sequence for the attention), one
+    kernel back to back from a CUDA graph.  Prints achieved GB/s (compressors: kv + gate read,
+    entries written) or TFLOP/s (attention: 4 flops per (query, head, row, dim) over the rows
+    each query sees)."""
+    import torch
+    from heavily_compressed_long_b200 import api
+    from heavily_compressed_long_b200.api import KV
+    from synth.configs import HCA_64K as cfg
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    g = torch.Generator(device=device)
+    g.manual_seed(cfg.seed)
+    B, L, d, mh, W, Tq, H = cfg.B, cfg.L, cfg.d, cfg.mh, cfg.W, cfg.Tq, cfg.H
+    kv = torch.randn(B, L, d, generator=g, device=device).to(torch.bfloat16)
+    gate = torch.randn(B, L, d, generator=g, device=device).to(torch.bfloat16)
+    stream = torch.cuda.Stream(device)
+    if args.kernel == "compress_csa":
+        m, n_ent = cfg.m, -(-L // cfg.m)
+        bias = 0.1 * torch.randn(2 * m, generator=g, device=device)
+        out = torch.empty(B, n_ent, d, dtype=torch.bfloat16, device=device)
+        launch = lambda: api.hcl_csa_compress(kv, gate, bias, m, out, stream=stream)
+        nbytes, flops = 2 * kv.numel() * 2 + out.numel() * 2, None
+    elif args.kernel == "compress_hca":
+        n_ent = -(-L // mh)
+        bias = 0.1 * torch.randn(mh, generator=g, device=device)
+        out = torch.empty(B, n_ent, d, dtype=torch.bfloat16, device=device)
+        launch = lambda: api.hcl_hca_compress(kv, gate, bias, mh, out, stream=stream)
+        nbytes, flops = 2 * kv.numel() * 2 + out.numel() * 2, None
+    else:
+        Nh = -(-L // mh)
+        ent = torch.randn(B, Nh, d, generator=g, device=device).to(torch.bfloat16)
+        q = torch.randn(B, Tq, H, d, generator=g, device=device).to(torch.bfloat16)
+        pos = torch.arange(L - Tq, L, dtype=torch.int32, device=device).repeat(B, 1).contiguous()
+        layer = None
+        from heavily_compressed_long_b200.pipeline import HcaLayer
+        layer = HcaLayer(q, KV(ent), Nh, mh, KV(kv), L, W, pos)
+        launch = lambda: layer.step(stream=stream)
+        rows = sum(min(Nh, (p + 1) // mh) + min(W, p + 1) for p in range(L - Tq, L))
+        nbytes, flops = None, 4.0 * B * H * d * rows
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            launch()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for _ in range(args.steps):
+            launch()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    del graph
+    line = {"kernel": args.kernel, "workload": f"{cfg.name} shapes", "ms_per_launch": ms,
+            "launches": args.steps}
+    if nbytes:
+        hbm, src = peaks()
+        line.update({"bytes_per_launch": nbytes, "achieved_gbs": nbytes / ms / 1e6,
+                     "peak_gbs": hbm, "frac": nbytes / ms / 1e6 / hbm, "peak_source": src})
+    else:
+        line.update({"flops_per_launch": flops, "achieved_tflops": flops / ms / 1e9,
+                     "frac_of_bf16_peak": flops / ms / 1e9 / bf16_peak()})
+    print(json.dumps(line), flush=True)
+
+
+def bf16_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"])
+    return 1590.0
+
+
 def run_kernel_micro(args, local_rank):
     """One kernel alone on one input set of `--batch` sequences (indexer: larger than L2),
     for profiling: times back-to-back launches with CUDA events and prints a JSON line."""
@@ -517,6 +596,8 @@ def run_kernel_micro(args, local_rank):
     from heavily_compressed_long_b200.api import HCL_MXFP4
     if args.kernel == "indexer_prefill":
         return run_prefill_indexer(args, local_rank)
+    if args.kernel in ("compress_csa", "compress_hca", "hca_prefill"):
+        return run_hca_shape_micro(args, local_rank)
     cfg = workload()
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
@@ -534,6 +615,8 @@ def run_kernel_micro(args, local_rank):
                                      Nc=p.Nc, qI_sf=p.qI_sf, kI_sf=p.kI_sf, stream=stream)
         elif args.kernel == "topk":
             api.hcl_csa_topk(p.scores, p.q_pos, p.m, p.k, p.idx, stream=stream)
+        elif args.kernel == "step":
+            p.step(stream=stream)
         else:
             api.hcl_csa_sparse_attn(p.q, p.kvc, p.Nc, p.idx, p.raw, p.L, p.W, p.q_pos, p.out,
                                     lse=p.lse, ws=p.attn_ws, stream=stream)
@@ -569,7 +652,9 @@ def run_kernel_micro(args, local_rank):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kernel", default=None, choices=["indexer", "topk", "attn", "indexer_prefill"],
+    ap.add_argument("--kernel", default=None,
+                    choices=["indexer", "topk", "attn", "step", "indexer_prefill", "compress_csa",
+                             "compress_hca", "hca_prefill"],
                     help="time one kernel alone (profiling aid) instead of the whole step")
     ap.add_argument("--batch", type=int, default=16, help="sequences for --kernel")
     ap.add_argument("--gpus", type=int, default=1)

@@ -7,6 +7,8 @@
 #include <stdio.h>
 
 #include <mutex>
+#include <set>
+#include <tuple>
 
 #include "hcl_common.cuh"
 #include "hcl_internal.h"
@@ -61,6 +63,50 @@ static long long clock_khz() {
 }
 
 long long wait_limit_cycles() { return clock_khz() * 1000LL; }  // about one second
+
+unsigned long long current_ctx_id() {
+  typedef CUresult (*GetCurrentFn)(CUcontext*);
+  typedef CUresult (*GetIdFn)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetIdFn>(p);
+  });
+  CUcontext c = nullptr;
+  if (get_current == nullptr || get_id == nullptr || get_current(&c) != CUDA_SUCCESS || !c) return 0;
+  unsigned long long id = 0;
+  return get_id(c, &id) == CUDA_SUCCESS ? id : 0;
+}
+
+hcl_status_t set_kernel_attrs(const void* kern, int smem, bool nonportable_cluster) {
+  static std::mutex mu;
+  static std::set<std::tuple<const void*, unsigned long long, int, bool>> done;
+  const unsigned long long ctx = current_ctx_id();
+  std::lock_guard<std::mutex> lock(mu);
+  if (ctx != 0 && done.count(std::make_tuple(kern, ctx, smem, nonportable_cluster))) return HCL_OK;
+  hcl_status_t e = check_cuda(
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+      "kernel shared-memory attribute");
+  if (e != HCL_OK) return e;
+  if (nonportable_cluster) {
+    e = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1),
+                   "kernel cluster attribute");
+    if (e != HCL_OK) return e;
+  }
+  // the attribute call makes a context current if none was; record under its id
+  const unsigned long long now = current_ctx_id();
+  if (now != 0) done.insert(std::make_tuple(kern, now, smem, nonportable_cluster));
+  return HCL_OK;
+}
 
 EncodeTiledFn encode_tiled() {
   static EncodeTiledFn fn = nullptr;

@@ -1010,17 +1010,9 @@ hcl_status_t launch_t(const AttnParams& p, cudaStream_t st, long long grid) {
   for (int S = 2; S <= MAX_CLUSTER; S++) recv_max = std::max(recv_max, recv_bytes(S));
   const size_t smem_max = smem + recv_max;
   smem += recv_bytes(p.splits);
-  static bool attr_done = false;  // per instantiation, set once (for the largest cluster need)
-  if (!attr_done) {
-    hcl_status_t e = check_cuda(
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max),
-        "attention smem attribute");
-    if (e != HCL_OK) return e;
-    e = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1),
-                   "attention cluster attribute");
-    if (e != HCL_OK) return e;
-    attr_done = true;
-  }
+  // set for the largest cluster need, once per kernel and context
+  hcl_status_t ea = set_kernel_attrs(reinterpret_cast<const void*>(kern), (int)smem_max, true);
+  if (ea != HCL_OK) return ea;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1061,17 +1053,8 @@ hcl_status_t launch_tc(const AttnParams& p, cudaStream_t st) {
   size_t smem_max = (size_t)tc_offsets(TC_MAXC, 1).total + 1024;
   for (int S = 2; S <= MAX_CLUSTER; S++)
     smem_max = std::max(smem_max, (size_t)tc_offsets(TC_MAXC_MERGE, S).total + 1024);
-  static bool attr_done = false;
-  if (!attr_done) {
-    hcl_status_t e = check_cuda(
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max),
-        "attention smem attribute");
-    if (e != HCL_OK) return e;
-    e = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1),
-                   "attention cluster attribute");
-    if (e != HCL_OK) return e;
-    attr_done = true;
-  }
+  hcl_status_t ea = set_kernel_attrs(reinterpret_cast<const void*>(kern), (int)smem_max, true);
+  if (ea != HCL_OK) return ea;
   const size_t smem = (size_t)tc_offsets(p.cps, p.splits).total + 1024;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
@@ -1165,22 +1148,28 @@ hcl_status_t launch_attn(const AttnArgs& a, void* ws, size_t ws_bytes, cudaStrea
 // partial (o, lse) slot the merge reads is written earlier in the same call.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
 
-// Device address of the scratch array on the current device.  The array's name is only a
-// host-side stand-in in host code, so the address is looked up once per device (with that
-// device current) by cudaGetSymbolAddress and cached.
+// Device address of the scratch array in the calling thread's current CUDA context.  The
+// array's name is only a host-side stand-in in host code, so the address is looked up by
+// cudaGetSymbolAddress with the device current and cached per device together with the id of
+// the context it belongs to: a call in another context (one created after cudaDeviceReset, or
+// a non-primary context) finds no cached entry for its context id and looks the address up
+// again.  Context ids are never reused within a process.
 hcl_status_t noalloc_scratch(void** ptr) {
   static std::mutex mu;
+  static unsigned long long ctx_of[64] = {};
   static void* cache[64] = {};
   int dev = 0;
   hcl_status_t e = check_cuda(cudaGetDevice(&dev), "cudaGetDevice");
   if (e != HCL_OK) return e;
   if (dev < 0 || dev >= 64) return fail(HCL_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
+  const unsigned long long ctx = current_ctx_id();
   std::lock_guard<std::mutex> lock(mu);
-  if (cache[dev] == nullptr) {
+  if (ctx == 0 || ctx_of[dev] != ctx || cache[dev] == nullptr) {
     void* p = nullptr;
     e = check_cuda(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
     if (e != HCL_OK) return e;
     cache[dev] = p;
+    ctx_of[dev] = current_ctx_id();   // the lookup made the device's context current
   }
   *ptr = cache[dev];
   return HCL_OK;

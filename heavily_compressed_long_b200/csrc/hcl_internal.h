@@ -49,6 +49,15 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 
 // Number of SMs of the current device (cached per device).
 int num_sms();
+// Id of the calling thread's current CUDA context, 0 when none is current yet.  Ids are never
+// reused within a process (a context created after cudaDeviceReset gets a new one), so they
+// key per-context caches safely, unlike device numbers or context handles.
+unsigned long long current_ctx_id();
+// Sets `kern`'s maximum dynamic shared memory to `smem` bytes (and, with nonportable_cluster,
+// allows cluster sizes above 8), once per (kernel, CUDA context, smem): function attributes
+// belong to a context, so every device -- and a context re-created after a reset -- gets its
+// own.  Thread-safe.
+hcl_status_t set_kernel_attrs(const void* kern, int smem, bool nonportable_cluster);
 // Bounded-wait budget for device spin loops, in SM clock cycles (about one second).
 long long wait_limit_cycles();
 

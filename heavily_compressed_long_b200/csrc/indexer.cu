@@ -703,14 +703,10 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
 }
 
 int smem_per_sm() {
-  static int v = 0;
-  if (v == 0) {
-    int dev = 0, b = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&b, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
-    v = b > 0 ? b : 228 * 1024;
-  }
-  return v;
+  int dev = 0, b = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&b, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  return b > 0 ? b : 228 * 1024;
 }
 
 template <int KIND, int QT, int TPS, int STAGES, int NACC, int EPI>
@@ -719,14 +715,8 @@ hcl_status_t run(const IndexerArgs& a, const void* qI_bf16, const CUtensorMap& t
   using Lay = IdxLayout<KIND, QT, TPS, STAGES, NACC, EPI>;
   auto kern = indexer_kernel<KIND, QT, TPS, STAGES, NACC, EPI>;
   const int smem = std::max(Lay::BYTES + 1024, min_smem);
-  static int configured_smem = -1;  // per instantiation
-  if (configured_smem != smem) {
-    hcl_status_t e = check_cuda(
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
-        "indexer smem attribute");
-    if (e != HCL_OK) return e;
-    configured_smem = smem;
-  }
+  hcl_status_t ea = set_kernel_attrs(reinterpret_cast<const void*>(kern), smem, false);
+  if (ea != HCL_OK) return ea;
   // blocks per SM: shared memory (+1 KB reserved per block), TMEM (512 columns), threads
   int per_sm = smem_per_sm() / (smem + 1024);
   per_sm = std::max(1, std::min({per_sm, int(512 / Lay::TMEM_COLS), 2048 / Lay::NT}));

@@ -19,6 +19,8 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <map>
+#include <mutex>
 
 #include "hcl_common.cuh"
 #include "hcl_internal.h"
@@ -1600,14 +1602,8 @@ hcl_status_t run_topk_gm(const TopkArgs& a, const uint16_t* gmax, const uint16_t
                         const uint8_t* garg, cudaStream_t st) {
   auto kern = topk_gm_kernel;
   const int smem = (int)sizeof(GmShared);
-  static bool attr_done = false;
-  if (!attr_done) {
-    hcl_status_t e = check_cuda(
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
-        "topk smem attribute");
-    if (e != HCL_OK) return e;
-    attr_done = true;
-  }
+  hcl_status_t ea = set_kernel_attrs(reinterpret_cast<const void*>(kern), smem, false);
+  if (ea != HCL_OK) return ea;
   const long long rows = (long long)a.B * a.Tq;
   const int NGP = gmax_row_stride(a.Nc);
   return check_cuda(launch_pdl(kern, dim3((unsigned)rows), dim3(TK_THREADS), (size_t)smem, st, 1,
@@ -1631,6 +1627,19 @@ int choose_cluster(long long rows, int nvis_max, size_t cap_keys) {
   return C;
 }
 
+// Co-resident cluster counts of one kernel per cluster size (index C), queried on first use
+// and cached per (kernel, CUDA context): 0 unknown, -1 not schedulable.
+struct ClusterCounts {
+  int n[17] = {0};
+  int& operator[](int C) { return n[C]; }
+};
+ClusterCounts& cluster_counts(const void* kern) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, unsigned long long>, ClusterCounts> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  return cache[std::make_pair(kern, current_ctx_id())];   // map nodes never move
+}
+
 template <bool BF16>
 hcl_status_t run_topk(const TopkArgs& a, cudaStream_t st) {
   const long long rows = (long long)a.B * a.Tq;
@@ -1638,17 +1647,12 @@ hcl_status_t run_topk(const TopkArgs& a, cudaStream_t st) {
   const size_t cap_keys = (200 * 1024 - sizeof(TkShared)) / key_bytes;
   int C = choose_cluster(rows, a.Nc, cap_keys);
   auto kern = topk_kernel<BF16>;
-  hcl_status_t e = check_cuda(
-      cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1),
-      "topk cluster attribute");
-  if (e != HCL_OK) return e;
+  hcl_status_t e;
   for (;;) {
     const size_t chunk = (size_t)(a.Nc + C - 1) / C;
     const int chunk_cap = (int)std::min(chunk, cap_keys);
     const size_t smem = sizeof(TkShared) + ((size_t)chunk_cap * key_bytes + 15) / 16 * 16;
-    e = check_cuda(
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
-        "topk smem attribute");
+    e = set_kernel_attrs(reinterpret_cast<const void*>(kern), (int)smem, true);
     if (e != HCL_OK) return e;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
@@ -1690,20 +1694,11 @@ hcl_status_t run_topk16(const TopkArgs& a, cudaStream_t st, bool* used) {
   const int key_bytes = BF16 ? 2 : 4;
   const size_t cap_keys = (226 * 1024 - sizeof(Tk16Shared) - 16) / key_bytes;
   auto kern = topk16_kernel<BF16>;
-  // attributes and the co-resident cluster count of each size are set / queried once
-  static bool attr_done = false;
-  static int max_clusters[17] = {0};   // 0 unknown, -1 not schedulable
-  hcl_status_t e;
-  if (!attr_done) {
-    e = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1),
-                   "topk cluster attribute");
-    if (e != HCL_OK) return e;
-    e = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        226 * 1024),
-                   "topk smem attribute");
-    if (e != HCL_OK) return e;
-    attr_done = true;
-  }
+  // attributes are set once per context; the co-resident cluster count of each size is
+  // queried once per context (0 unknown, -1 not schedulable)
+  hcl_status_t e = set_kernel_attrs(reinterpret_cast<const void*>(kern), 226 * 1024, true);
+  if (e != HCL_OK) return e;
+  ClusterCounts& max_clusters = cluster_counts(reinterpret_cast<const void*>(kern));
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1764,18 +1759,9 @@ hcl_status_t run_topk_reg(const TopkArgs& a, cudaStream_t st, bool* used) {
   if (rows > num_sms()) return HCL_OK;          // many rows: the shared-memory kernels
   auto kern = topk_reg_kernel;
   const int smem = (int)sizeof(TrShared);
-  static bool attr_done = false;
-  static int max_clusters[17] = {0};
-  hcl_status_t e;
-  if (!attr_done) {
-    e = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1),
-                   "topk cluster attribute");
-    if (e != HCL_OK) return e;
-    e = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
-                   "topk smem attribute");
-    if (e != HCL_OK) return e;
-    attr_done = true;
-  }
+  hcl_status_t e = set_kernel_attrs(reinterpret_cast<const void*>(kern), smem, true);
+  if (e != HCL_OK) return e;
+  ClusterCounts& max_clusters = cluster_counts(reinterpret_cast<const void*>(kern));
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;

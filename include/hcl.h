@@ -189,10 +189,12 @@ HCL_API hcl_status_t hcl_csa_sparse_attn(const void* q, int B, int Tq, int H, in
  * that loads the library, held until the process exits.  A problem whose partials need more
  * (hcl_csa_sparse_attn_workspace_bytes() > 16 MiB) is rejected with HCL_ERR_INVALID_ARG and
  * a message naming the limit.  The first call on a device looks the array's device address
- * up (cudaGetSymbolAddress); make that first call before any stream capture.  All calls
- * share the array and leave their partials in it; calls that overlap on the GPU (different
- * streams, or threads) race on it, so serialise them.  Nothing in the array needs clearing:
- * each call writes every slot it later reads.
+ * up (cudaGetSymbolAddress) and caches it for that device's current CUDA context; make that
+ * first call before any stream capture.  A call made in a different context (for example
+ * after cudaDeviceReset, which destroys the old one) looks the address up again, so it is
+ * again a first call.  All calls share the array and leave their partials in it; calls that
+ * overlap on the GPU (different streams, or threads) race on it, so serialise them.  Nothing
+ * in the array needs clearing: each call writes every slot it later reads.
  */
 #define HCL_NOALLOC_SCRATCH_BYTES (16u << 20)
 HCL_API hcl_status_t hcl_csa_sparse_attn_noalloc(const void* q, int B, int Tq, int H, int d,

@@ -3,9 +3,13 @@
 The GPU runs every sequence and query of a workload through the same calls the benchmark
 times; the oracle recomputes sampled sequences / query rows from the same seeded inputs.
 Stored entries and scores compare within 1 bf16 ulp (bf16) or 1e-3 norm-wise (fp32);
-selections compare with the ambiguity band; attention within 2e-2 (bf16 KV) / 5e-2 (FP8 KV)
-on rows whose selection equals the oracle's (the selection itself is checked separately);
-quantised caches compare bit-exact."""
+quantised caches compare bit-exact.  A selection is not unique where scores tie within the
+ambiguity band (|s - s_k| <= max(1e-3 |s_k|, 1 bf16 ulp)), so it is checked in two parts: the
+part outside the band must equal the oracle's top-k, and the GPU's selection must be a valid
+one (unique, visible, ascending, of the right size).  The oracle then attends over that very
+validated selection and every sampled row's attention must agree with it within 2e-2 (bf16
+KV) / 5e-2 (FP8 KV) -- on every sampled row, whether or not the selection equals the
+oracle's own."""
 import numpy as np
 import pytest
 import torch
@@ -51,8 +55,6 @@ def test_cfg1_csa_tiny_end_to_end(hcl):
     ent = oracle.compress(kv, g, bias, cfg.m, True)
     ent16 = bf16_of(ent)
     s_ref = oracle.index_scores(oracle.FMT_BF16, qI, w, kI, pos, cfg.m)
-    idx_ref = oracle.topk(s_ref, pos, cfg.m, cfg.k)
-    o_ref, l_ref = oracle.csa_attn(q, oracle.KV(0, ent16, Nc), idx_ref, oracle.KV(0, kv, cfg.L), cfg.W, pos)
     # GPU chain
     comp = torch.empty(1, Nc, cfg.d, dtype=torch.bfloat16, device="cuda")
     hcl.hcl_csa_compress(cuda(kv), cuda(g), cuda(bias), cfg.m, comp)
@@ -63,10 +65,10 @@ def test_cfg1_csa_tiny_end_to_end(hcl):
     assert bf16_out_ratio(as_f64(comp), ent) <= 1.0
     assert rel_rowwise(as_f64(pipe.scores), s_ref) <= 1e-3
     gidx = pipe.idx.cpu().numpy()
-    diff = check_topk_band(gidx[0, 0], s_ref[0, 0], Nc, cfg.k, False)
-    if diff == 0:
-        assert np.abs(as_f64(pipe.out) - o_ref).max() <= 2e-2
-        assert np.abs(as_f64(pipe.lse) - l_ref).max() <= 2e-2
+    check_topk_band(gidx[0, 0], s_ref[0, 0], Nc, cfg.k, False)
+    o_ref, l_ref = oracle.csa_attn(q, oracle.KV(0, ent16, Nc), gidx, oracle.KV(0, kv, cfg.L), cfg.W, pos)
+    assert np.abs(as_f64(pipe.out) - o_ref).max() <= 2e-2
+    assert np.abs(as_f64(pipe.lse) - l_ref).max() <= 2e-2
     # the fused C-ABI decode step launches the same kernels: identical bits
     out1, idx1 = pipe.out.clone(), pipe.idx.clone()
     pipe.step()
@@ -132,12 +134,11 @@ def test_cfg3_csa_128k_planted(hcl):
         sl = slice(b, b + 1)
         s_ref = oracle.index_scores(oracle.FMT_BF16, qI[sl], w[sl], kI[sl], pos[sl], cfg.m)
         assert rel_rowwise(as_f64(pipe.scores[sl]), s_ref) <= 1e-3
-        idx_ref = oracle.topk(s_ref, pos[sl], cfg.m, cfg.k)
-        diff = check_topk_band(gidx[b, 0], s_ref[0, 0], Nc, cfg.k, False)
-        o_ref, l_ref = oracle.csa_attn(q[sl], oracle.KV(0, kvc[sl], Nc), idx_ref,
+        check_topk_band(gidx[b, 0], s_ref[0, 0], Nc, cfg.k, False)
+        o_ref, l_ref = oracle.csa_attn(q[sl], oracle.KV(0, kvc[sl], Nc), gidx[sl],
                                        oracle.KV(0, ring[sl], W), W, pos[sl])
-        if diff == 0:
-            assert np.abs(as_f64(pipe.out[sl]) - o_ref).max() <= 2e-2
+        assert np.abs(as_f64(pipe.out[sl]) - o_ref).max() <= 2e-2
+        assert np.abs(as_f64(pipe.lse[sl]) - l_ref).max() <= 2e-2
     assert pipe.status.item() == 0
 
 
@@ -183,14 +184,12 @@ def test_cfg4_csa_1m_mxfp4_fp8(hcl):
         s_ref = oracle.index_scores(oracle.FMT_MXFP4, qp, w[sl], kp, pos[sl], cfg.m, qI_sf=qs,
                                     kI_sf=ks, bf16_scores=True)
         assert bf16_out_ratio(as_f64(pipe.scores[sl]), s_ref) <= 1.0
-        idx_ref = oracle.topk(s_ref, pos[sl], cfg.m, cfg.k)
-        diff = check_topk_band(gidx[b, 0], s_ref[0, 0], Nc, cfg.k, True)
+        check_topk_band(gidx[b, 0], s_ref[0, 0], Nc, cfg.k, True)
         okc = oracle.KV(oracle.FMT_FP8SPLIT, cn, Nc, scale=cs, rope=cr)
         okr = oracle.KV(oracle.FMT_FP8SPLIT, rn, W, scale=rs, rope=rr)
-        o_ref, l_ref = oracle.csa_attn(q[sl], okc, idx_ref, okr, W, pos[sl])
-        if diff == 0:
-            assert np.abs(as_f64(pipe.out[sl]) - o_ref).max() <= 5e-2
-            assert np.abs(as_f64(pipe.lse[sl]) - l_ref).max() <= 5e-2
+        o_ref, l_ref = oracle.csa_attn(q[sl], okc, gidx[sl], okr, W, pos[sl])
+        assert np.abs(as_f64(pipe.out[sl]) - o_ref).max() <= 5e-2
+        assert np.abs(as_f64(pipe.lse[sl]) - l_ref).max() <= 5e-2
     assert pipe.status.item() == 0
     # the fused C-ABI decode step (q_I quantised inside the indexer) gives the same bits
     out1, idx1, sc1 = pipe.out.clone(), pipe.idx.clone(), pipe.scores.clone()
@@ -230,17 +229,14 @@ def test_cfg5_pair_prefill(hcl):
     s_ref = oracle.index_scores(oracle.FMT_BF16, qI[:, rows].contiguous(), w[:, rows].contiguous(),
                                 kI, ps, m, bf16_scores=True)
     assert bf16_out_ratio(as_f64(pp.scores[:, rows]), s_ref) <= 1.0
-    idx_ref = oracle.topk(s_ref, ps, m, cfg.k)
-    gidx = pp.idx[:, rows].cpu().numpy()
-    same = []
-    for r in range(len(rows)):
+    gidx = np.ascontiguousarray(pp.idx[:, rows].cpu().numpy())
+    for r in range(len(rows)):                 # every sampled row's selection is checked
         nvis = oracle.num_visible(int(ps[0, r]), m, Nc)
-        if check_topk_band(gidx[0, r], s_ref[0, r], nvis, cfg.k, True) == 0:
-            same.append(r)
-    assert len(same) >= 0.8 * len(rows)
-    o_ref, _ = oracle.csa_attn(q_csa[:, rows].contiguous(), oracle.KV(0, bf16_of(ent_c), Nc), idx_ref,
-                               oracle.KV(0, kv, L), W, ps)
-    assert np.abs(as_f64(pp.out_csa[:, rows][:, same]) - o_ref[:, same]).max() <= 2e-2
+        check_topk_band(gidx[0, r], s_ref[0, r], nvis, cfg.k, True)
+    o_ref, l_ref = oracle.csa_attn(q_csa[:, rows].contiguous(), oracle.KV(0, bf16_of(ent_c), Nc), gidx,
+                                   oracle.KV(0, kv, L), W, ps)
+    assert np.abs(as_f64(pp.out_csa[:, rows]) - o_ref).max() <= 2e-2
+    assert np.abs(as_f64(pp.lse_csa[:, rows]) - l_ref).max() <= 2e-2
     oh_ref, lh_ref = oracle.hca_attn(q_hca[:, rows].contiguous(), oracle.KV(0, bf16_of(ent_h), Nh), Nh, mh,
                                      oracle.KV(0, kv, L), W, ps)
     assert np.abs(as_f64(pp.hca.out[:, rows]) - oh_ref).max() <= 2e-2

@@ -3,17 +3,22 @@ memory (serving runtimes that own the device's memory pool and forbid cudaMalloc
 request path; plugin hosts that pass a kernel only its inputs and outputs).  Its split-KV
 partials live in a fixed 16 MiB array inside the library instead of a caller workspace.
 
-Checked through the C ABI against hcl_csa_sparse_attn (the workspace entry point) on two
-calls in a row with different inputs, within the attention tolerance the other tests use
-(5e-2 max abs for FP8 KV rows, 2e-2 for bf16); and a problem needing more scratch than the
-fixed array is refused with a message naming the limit.  This file is collected last so a
-run that stops at the first failure has already run every other test."""
+Checked through the C ABI on two calls in a row with different inputs: each call's output
+and log-sum-exp must equal, bit for bit, those of hcl_csa_sparse_attn (the workspace entry
+point: same plan, same kernels, and results are deterministic -- so stale partials left in the
+shared array by the previous call would show), and both must agree with the CPU oracle within
+the attention tolerance the other tests use (5e-2 max abs for FP8 KV rows, 2e-2 for bf16).
+A problem needing more scratch than the fixed array is refused with a message naming the
+limit.  This file is collected last so a run that stops at the first failure has already run
+every other test."""
 import ctypes
 import math
 
 import numpy as np
 import pytest
 import torch
+
+import oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -26,30 +31,33 @@ def _kv_struct(_lib, data, scale=None, rope=None):
 
 
 def _problem(seed, B, H, Nc, k, W, fp8):
-    g = torch.Generator(device="cuda")
+    """Seeded inputs generated on the host (torch's CPU generator), copied to the device; the
+    oracle gets the same host values (FP8 rows quantised by the oracle, bit-equal to the
+    library's quantiser as the parity tests show)."""
+    g = torch.Generator()
     g.manual_seed(seed)
     d, L = 128, 4 * Nc
-    q = torch.randn(B, 1, H, d, generator=g, device="cuda").to(torch.bfloat16)
-    idx = torch.stack([torch.randperm(Nc, generator=g, device="cuda")[:k].sort().values
+    q = torch.randn(B, 1, H, d, generator=g).to(torch.bfloat16)
+    idx = torch.stack([torch.randperm(Nc, generator=g)[:k].sort().values
                        for _ in range(B)]).view(B, 1, k).to(torch.int32).contiguous()
-    pos = torch.full((B, 1), L - 1, dtype=torch.int32, device="cuda")
-    ent = torch.randn(B, Nc, d, generator=g, device="cuda").to(torch.bfloat16)
-    raw = torch.randn(B, W, d, generator=g, device="cuda").to(torch.bfloat16)
+    pos = torch.full((B, 1), L - 1, dtype=torch.int32)
+    ent = torch.randn(B, Nc, d, generator=g).to(torch.bfloat16)
+    raw = torch.randn(B, W, d, generator=g).to(torch.bfloat16)
+    host = dict(q=q, idx=idx, pos=pos)
     if not fp8:
-        return q, idx, pos, (ent,), (raw,), L
-    from heavily_compressed_long_b200 import api
-    out = []
-    for t in (ent, raw):
-        n = torch.empty(t.shape[0], t.shape[1], 64, dtype=torch.uint8, device="cuda")
-        s = torch.empty(t.shape[0], t.shape[1], dtype=torch.float32, device="cuda")
-        r = torch.empty(t.shape[0], t.shape[1], 64, dtype=torch.bfloat16, device="cuda")
-        api.hcl_quant_kv_fp8(t, n, s, r)
-        out.append((n, s, r))
-    return q, idx, pos, out[0], out[1], L
+        host.update(okc=oracle.KV(oracle.FMT_BF16, ent, Nc), okr=oracle.KV(oracle.FMT_BF16, raw, W))
+        return (q.cuda(), idx.cuda(), pos.cuda(), (ent.cuda(),), (raw.cuda(),), L, host)
+    dev = []
+    for name, t, cap in (("okc", ent, Nc), ("okr", raw, W)):
+        n, sc, r = oracle.quant_kv_fp8(t)
+        host[name] = oracle.KV(oracle.FMT_FP8SPLIT, n, cap, scale=sc, rope=r)
+        dev.append((torch.from_numpy(n).cuda(), torch.from_numpy(sc).cuda(),
+                    torch.from_numpy(r.view(np.int16)).view(torch.bfloat16).cuda()))
+    return (q.cuda(), idx.cuda(), pos.cuda(), dev[0], dev[1], L, host)
 
 
 def _call_both(hcl, _lib, L_, B, H, Nc, k, W, fp8, seed):
-    q, idx, pos, kvc_t, raw_t, L = _problem(seed, B, H, Nc, k, W, fp8)
+    q, idx, pos, kvc_t, raw_t, L, host = _problem(seed, B, H, Nc, k, W, fp8)
     kvc = _kv_struct(_lib, *kvc_t)
     raw = _kv_struct(_lib, *raw_t)
     scale = 1.0 / math.sqrt(128)
@@ -73,7 +81,8 @@ def _call_both(hcl, _lib, L_, B, H, Nc, k, W, fp8, seed):
                                               lse.data_ptr(), status.data_ptr(), stream))
     torch.cuda.synchronize()
     assert status.item() == 0
-    return need, out, out_ref, lse, lse_ref
+    o_or, l_or = oracle.csa_attn(host["q"], host["okc"], host["idx"], host["okr"], W, host["pos"])
+    return need, out, out_ref, lse, lse_ref, o_or, l_or
 
 
 @pytest.mark.parametrize("fp8", [True, False])
@@ -85,10 +94,12 @@ def test_noalloc_matches_workspace_entry_point_twice(hcl, fp8):
     # split over more blocks than one cluster holds, so the split partials go through the
     # fixed scratch array; then a second, different call
     for seed, (B, H, Nc, k, W) in [(11, (1, 128, 20000, 4096, 128)), (12, (2, 64, 9000, 2048, 128))]:
-        need, out, out_ref, lse, lse_ref = _call_both(hcl, _lib, L_, B, H, Nc, k, W, fp8, seed)
+        need, out, out_ref, lse, lse_ref, o_or, l_or = _call_both(hcl, _lib, L_, B, H, Nc, k, W,
+                                                                  fp8, seed)
         assert 0 < need <= (16 << 20)               # the partials go through the scratch
-        assert (out.float() - out_ref.float()).abs().max().item() <= tol
-        assert (lse - lse_ref).abs().max().item() <= tol
+        assert torch.equal(out, out_ref) and torch.equal(lse, lse_ref)
+        assert np.abs(out.double().cpu().numpy() - o_or).max() <= tol
+        assert np.abs(lse.double().cpu().numpy() - l_or).max() <= tol
 
 
 def test_noalloc_rejects_problems_beyond_the_fixed_scratch(hcl):
