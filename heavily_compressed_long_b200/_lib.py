@@ -30,21 +30,25 @@ KVP = ctypes.POINTER(hcl_kv_t)
 SIGNATURES = {
     "hcl_version": (ctypes.c_char_p, []),
     "hcl_last_error": (ctypes.c_char_p, []),
-    "hcl_csa_compress": (I, [P, P, P, I, I, I, I, I, I, P, I, I, P]),
-    "hcl_hca_compress": (I, [P, P, P, I, I, I, I, I, I, P, I, I, P]),
+    "hcl_csa_compress": (I, [P, P, P, I, I, I, I, I, I, P, I, I, P, F, P]),
+    "hcl_hca_compress": (I, [P, P, P, I, I, I, I, I, I, P, I, I, P, F, P]),
     "hcl_quant_kv_fp8": (I, [P, I64, I, P, P, P, P]),
     "hcl_quant_mxfp4": (I, [P, I64, I, P, P, P]),
     "hcl_csa_index_scores": (I, [I, P, P, P, P, P, I, I, I, I, I, I, P, I, P, I, P, P]),
     "hcl_csa_topk_workspace_bytes": (SZ, [I, I, I, I, I]),
     "hcl_csa_topk": (I, [P, I, I, I, I, P, I, I, P, P, SZ, P, P]),
     "hcl_csa_sparse_attn_workspace_bytes": (SZ, [I, I, I, I, I]),
-    "hcl_csa_sparse_attn": (I, [P, I, I, I, I, KVP, I, P, I, KVP, I, I, P, F, P, P, P, P, SZ, P, P]),
+    "hcl_csa_sparse_attn": (I, [P, I, I, I, I, KVP, I, P, I, KVP, I, I, P, F, P, P, F, P, P, P, SZ,
+                                P, P]),
     "hcl_csa_sparse_attn_noalloc": (I, [P, I, I, I, I, KVP, I, P, I, KVP, I, I, P, F, P, P, P, P, P]),
     "hcl_hca_dense_attn_workspace_bytes": (SZ, [I, I, I, I, I]),
-    "hcl_hca_dense_attn": (I, [P, I, I, I, I, KVP, I, I, KVP, I, I, P, F, P, P, P, P, SZ, P, P]),
+    "hcl_hca_dense_attn": (I, [P, I, I, I, I, KVP, I, I, KVP, I, I, P, F, P, P, F, P, P, P, SZ, P,
+                               P]),
     "hcl_csa_decode_step_workspace_bytes": (SZ, [I, I, I, I, I, I, I, I]),
     "hcl_csa_decode_step": (I, [P, P, P, I, P, P, I, I, I, I, I, I, I, KVP, I, I, I, KVP, I, I,
-                                P, F, P, P, P, P, P, SZ, P, P]),
+                                P, F, P, P, F, P, P, P, P, SZ, P, P]),
+    "hcl_cache_append": (I, [P, P, P, P, I, I, I, P, P, I, KVP, KVP, P, I, I, P, P, I, KVP, P, I,
+                             P, F, P, P]),
     "hcl_selftest_bounded_wait": (I, [P, I, P]),
 }
 

@@ -14,7 +14,7 @@ from ._lib import (HCL_BF16, HCL_FP32, HCL_FP8SPLIT, HCL_MXFP4, check, hcl_kv_t,
 
 __all__ = ["KV", "hcl_csa_compress", "hcl_hca_compress", "hcl_quant_kv_fp8", "hcl_quant_mxfp4",
            "hcl_csa_index_scores", "hcl_csa_topk", "hcl_csa_sparse_attn", "hcl_hca_dense_attn",
-           "hcl_csa_decode_step", "hcl_selftest_bounded_wait", "HCL_BF16", "HCL_FP32",
+           "hcl_csa_decode_step", "hcl_cache_append", "hcl_selftest_bounded_wait", "HCL_BF16", "HCL_FP32",
            "HCL_FP8SPLIT", "HCL_MXFP4"]
 
 
@@ -52,21 +52,26 @@ def _fmt_of(t):
     return HCL_FP32 if t.dtype == torch.float32 else HCL_BF16
 
 
-def hcl_csa_compress(kv, gate, bias, m, out, entry_begin=0, entry_end=None, stream=None):
+def hcl_csa_compress(kv, gate, bias, m, out, entry_begin=0, entry_end=None, gamma=None,
+                     eps=1e-6, stream=None):
+    """gamma (fp32 [d] CUDA tensor): RMSNorm each pooled entry (x / rms(x) * gamma)."""
     B, L, d = kv.shape
     if entry_end is None:
         entry_end = -(-L // m)
     check(lib().hcl_csa_compress(_ptr(kv), _ptr(gate), _ptr(bias), B, L, d, m, entry_begin,
-                                 entry_end, _ptr(out), _fmt_of(out), out.shape[1], _stream(stream)))
+                                 entry_end, _ptr(out), _fmt_of(out), out.shape[1], _ptr(gamma),
+                                 eps, _stream(stream)))
     return out
 
 
-def hcl_hca_compress(kv, gate, bias, m, out, entry_begin=0, entry_end=None, stream=None):
+def hcl_hca_compress(kv, gate, bias, m, out, entry_begin=0, entry_end=None, gamma=None,
+                     eps=1e-6, stream=None):
     B, L, d = kv.shape
     if entry_end is None:
         entry_end = -(-L // m)
     check(lib().hcl_hca_compress(_ptr(kv), _ptr(gate), _ptr(bias), B, L, d, m, entry_begin,
-                                 entry_end, _ptr(out), _fmt_of(out), out.shape[1], _stream(stream)))
+                                 entry_end, _ptr(out), _fmt_of(out), out.shape[1], _ptr(gamma),
+                                 eps, _stream(stream)))
     return out
 
 
@@ -110,7 +115,7 @@ def csa_sparse_attn_workspace_bytes(B, Tq, H, k, W):
 
 
 def hcl_csa_sparse_attn(q, kvc: KV, Nc, idx, raw: KV, L, W, q_pos, out, lse=None, scale=None,
-                        sink=None, ws=None, status=None, stream=None):
+                        sink=None, ws=None, status=None, q_gamma=None, q_eps=1e-6, stream=None):
     B, Tq, H, d = q.shape
     k = idx.shape[-1]
     scale = 1.0 / math.sqrt(d) if scale is None else scale
@@ -118,7 +123,8 @@ def hcl_csa_sparse_attn(q, kvc: KV, Nc, idx, raw: KV, L, W, q_pos, out, lse=None
     if ws is None and need:
         ws = torch.empty(need, dtype=torch.uint8, device=q.device)
     check(lib().hcl_csa_sparse_attn(_ptr(q), B, Tq, H, d, kvc.ref(), Nc, _ptr(idx), k, raw.ref(),
-                                    L, W, _ptr(q_pos), scale, _ptr(sink), _ptr(out), _ptr(lse),
+                                    L, W, _ptr(q_pos), scale, _ptr(sink), _ptr(q_gamma), q_eps,
+                                    _ptr(out), _ptr(lse),
                                     _ptr(ws), 0 if ws is None else ws.numel(), _ptr(status),
                                     _stream(stream)))
     return out
@@ -129,14 +135,15 @@ def hca_dense_attn_workspace_bytes(B, Tq, H, Nh, W):
 
 
 def hcl_hca_dense_attn(q, kvh: KV, Nh, mh, raw: KV, L, W, q_pos, out, lse=None, scale=None,
-                       sink=None, ws=None, status=None, stream=None):
+                       sink=None, ws=None, status=None, q_gamma=None, q_eps=1e-6, stream=None):
     B, Tq, H, d = q.shape
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     need = hca_dense_attn_workspace_bytes(B, Tq, H, Nh, W)
     if ws is None and need:
         ws = torch.empty(need, dtype=torch.uint8, device=q.device)
     check(lib().hcl_hca_dense_attn(_ptr(q), B, Tq, H, d, kvh.ref(), Nh, mh, raw.ref(), L, W,
-                                   _ptr(q_pos), scale, _ptr(sink), _ptr(out), _ptr(lse), _ptr(ws),
+                                   _ptr(q_pos), scale, _ptr(sink), _ptr(q_gamma), q_eps, _ptr(out),
+                                   _ptr(lse), _ptr(ws),
                                    0 if ws is None else ws.numel(), _ptr(status), _stream(stream)))
     return out
 
@@ -147,7 +154,7 @@ def decode_step_workspace_bytes(B, H, HI, Nc, k, W, op_fmt, score_fmt):
 
 def hcl_csa_decode_step(q, qI, w, op_fmt, kI, kvc: KV, Nc, m, k, raw: KV, L, W, q_pos, out,
                         score_fmt=HCL_FP32, kI_sf=None, lse=None, idx_out=None, scale=None,
-                        sink=None, ws=None, status=None, stream=None):
+                        sink=None, ws=None, status=None, q_gamma=None, q_eps=1e-6, stream=None):
     """One CSA decode step (Tq = 1): MXFP4-quantise qI (MXFP4 keys only), score, top-k, attend."""
     B, _, H, d = q.shape
     HI, dI = qI.shape[-2], qI.shape[-1]
@@ -157,10 +164,29 @@ def hcl_csa_decode_step(q, qI, w, op_fmt, kI, kvc: KV, Nc, m, k, raw: KV, L, W, 
         ws = torch.empty(need, dtype=torch.uint8, device=q.device)
     check(lib().hcl_csa_decode_step(_ptr(q), _ptr(qI), _ptr(w), op_fmt, _ptr(kI), _ptr(kI_sf),
                                     kI.shape[1], score_fmt, B, H, HI, dI, d, kvc.ref(), Nc, m, k,
-                                    raw.ref(), L, W, _ptr(q_pos), scale, _ptr(sink), _ptr(out),
-                                    _ptr(lse), _ptr(idx_out), _ptr(ws), ws.numel(), _ptr(status),
+                                    raw.ref(), L, W, _ptr(q_pos), scale, _ptr(sink), _ptr(q_gamma),
+                                    q_eps, _ptr(out), _ptr(lse), _ptr(idx_out), _ptr(ws), ws.numel(),
+                                    _ptr(status),
                                     _stream(stream)))
     return out
+
+
+def hcl_cache_append(kv_new, gate_new, t_new, stage_kv, stage_gate, raw: KV, kvc: KV = None,
+                     bias_csa=None, m=4, kI_new=None, kI=None, kI_sf=None, kvh: KV = None,
+                     bias_hca=None, mh=128, gamma=None, eps=1e-6, stream=None):
+    """Append one token per sequence (kv_new / gate_new bf16 [B, d], t_new int32 [B]) to one
+    layer's cache: staging rings, raw window store, and the CSA (kvc, index keys kI: bf16
+    [B, cap, dI], or MXFP4 packed uint8 [B, cap, dI/2] with kI_sf) or HCA (kvh) entry it
+    completes."""
+    B, d = kv_new.shape
+    kI_fmt = HCL_MXFP4 if kI_sf is not None else HCL_BF16
+    dI = 0 if kI is None else (kI.shape[-1] * (2 if kI_fmt == HCL_MXFP4 else 1))
+    check(lib().hcl_cache_append(_ptr(kv_new), _ptr(gate_new), _ptr(kI_new), _ptr(t_new), B, d, dI,
+                                 _ptr(stage_kv), _ptr(stage_gate), stage_kv.shape[1], raw.ref(),
+                                 None if kvc is None else kvc.ref(), _ptr(bias_csa), m, kI_fmt,
+                                 _ptr(kI), _ptr(kI_sf), 0 if kI is None else kI.shape[1],
+                                 None if kvh is None else kvh.ref(), _ptr(bias_hca), mh,
+                                 _ptr(gamma), eps, None, _stream(stream)))
 
 
 def hcl_selftest_bounded_wait(status, limit_us=1000, stream=None):

@@ -175,7 +175,8 @@ const char* hcl_last_error(void) { return g_err; }
 
 static hcl_status_t compress_common(const void* kv, const void* gate, const float* bias, int B,
                                     int L, int d, int m, int overlap, int e0, int e1, void* out,
-                                    int out_fmt, int out_cap, void* stream, int max_m) {
+                                    int out_fmt, int out_cap, const float* gamma, float eps,
+                                    void* stream, int max_m) {
   HCL_REQUIRE(B >= 0 && L >= 0, "B and L must be non-negative");
   HCL_REQUIRE(d > 0 && d % 8 == 0 && d <= 1024, "d must be a positive multiple of 8, <= 1024");
   HCL_REQUIRE(m >= 1 && m <= max_m, "m must be in [1, %d]", max_m);
@@ -184,25 +185,36 @@ static hcl_status_t compress_common(const void* kv, const void* gate, const floa
               "need 0 <= entry_begin <= entry_end <= min(ceil(L/m)=%lld, out_cap=%d)", n_ent,
               out_cap);
   HCL_REQUIRE(out_fmt == HCL_FP32 || out_fmt == HCL_BF16, "out_fmt must be HCL_FP32 or HCL_BF16");
+  if (gamma != nullptr) {
+    HCL_REQUIRE(eps > 0.f && eps < 1e30f, "eps must be a positive number");
+    // the RMSNorm reduction runs over the d/8 threads of an entry (a power of two <= 32) or
+    // over a 128-thread block (long spans)
+    const int G = d / 8;
+    const bool small = (overlap ? 2 * m : m) <= 16 || 128 % G != 0;
+    if (small && (G > 32 || (G & (G - 1)) != 0))
+      return fail(HCL_ERR_UNSUPPORTED, "RMSNorm epilogue needs d/8 a power of two <= 32 (d=%d)", d);
+  }
   if (e1 == e0 || B == 0) return HCL_OK;
   HCL_REQUIRE(kv && gate && bias && out, "NULL pointer");
   HCL_REQUIRE(aligned16(kv) && aligned16(gate) && aligned16(out), "kv, gate, out must be 16-byte aligned");
   return launch_compress(kv, gate, bias, B, L, d, m, overlap, e0, e1, out, out_fmt, out_cap,
-                         as_stream(stream));
+                         gamma, eps, as_stream(stream));
 }
 
 hcl_status_t hcl_csa_compress(const void* kv, const void* gate, const float* bias, int B, int L,
                               int d, int m, int entry_begin, int entry_end, void* out,
-                              int out_fmt, int out_cap, void* stream) {
+                              int out_fmt, int out_cap, const float* gamma, float eps,
+                              void* stream) {
   return compress_common(kv, gate, bias, B, L, d, m, 1, entry_begin, entry_end, out, out_fmt,
-                         out_cap, stream, 64);
+                         out_cap, gamma, eps, stream, 64);
 }
 
 hcl_status_t hcl_hca_compress(const void* kv, const void* gate, const float* bias, int B, int L,
                               int d, int m, int entry_begin, int entry_end, void* out,
-                              int out_fmt, int out_cap, void* stream) {
+                              int out_fmt, int out_cap, const float* gamma, float eps,
+                              void* stream) {
   return compress_common(kv, gate, bias, B, L, d, m, 0, entry_begin, entry_end, out, out_fmt,
-                         out_cap, stream, 1024);
+                         out_cap, gamma, eps, stream, 1024);
 }
 
 hcl_status_t hcl_quant_kv_fp8(const void* kv, int64_t rows, int d, void* nope, float* scale,
@@ -292,9 +304,9 @@ hcl_status_t hcl_csa_topk(const void* scores, int score_fmt, int B, int Tq, int 
 static hcl_status_t attn_common(int mode, const void* q, int B, int Tq, int H, int d,
                                 const hcl_kv_t* comp, int n_comp, int mh, const int32_t* idx,
                                 int k, const hcl_kv_t* raw, int L, int W, const int32_t* q_pos,
-                                float scale, const float* sink, void* out, float* lse, void* ws,
-                                size_t ws_bytes, int32_t* status, void* stream,
-                                int prewait = 0) {
+                                float scale, const float* sink, const float* q_gamma,
+                                float q_eps, void* out, float* lse, void* ws, size_t ws_bytes,
+                                int32_t* status, void* stream, int prewait = 0) {
   HCL_REQUIRE(B >= 0 && Tq >= 0, "negative size");
   if (d != 128) return fail(HCL_ERR_UNSUPPORTED, "only d == 128 is supported (got %d)", d);
   HCL_REQUIRE(H >= 1 && H <= 128, "H must be in [1, 128]");
@@ -303,6 +315,7 @@ static hcl_status_t attn_common(int mode, const void* q, int B, int Tq, int H, i
   else HCL_REQUIRE(mh >= 1, "mh must be >= 1");
   if ((long long)B * Tq == 0) return HCL_OK;
   HCL_REQUIRE(q && out && q_pos, "NULL pointer");
+  if (q_gamma != nullptr) HCL_REQUIRE(q_eps > 0.f && q_eps < 1e30f, "q_eps must be a positive number");
   HCL_REQUIRE(aligned16(q) && aligned16(out), "q and out must be 16-byte aligned");
   hcl_status_t e = check_kv(comp, d, mode == 0 ? "kvc" : "kvh");
   if (e != HCL_OK) return e;
@@ -317,6 +330,7 @@ static hcl_status_t attn_common(int mode, const void* q, int B, int Tq, int H, i
   a.comp = *comp; a.n_comp = n_comp; a.mh = mh; a.idx = idx; a.k = k;
   a.raw = *raw; a.L = L; a.W = W; a.q_pos = q_pos; a.scale = scale; a.sink = sink;
   a.out = out; a.lse = lse; a.status = status; a.prewait = prewait;
+  a.q_gamma = q_gamma; a.q_eps = q_eps;
   return launch_attn(a, ws, ws_bytes, as_stream(stream));
 }
 
@@ -327,10 +341,10 @@ size_t hcl_csa_sparse_attn_workspace_bytes(int B, int Tq, int H, int k, int W) {
 hcl_status_t hcl_csa_sparse_attn(const void* q, int B, int Tq, int H, int d, const hcl_kv_t* kvc,
                                  int Nc, const int32_t* idx, int k, const hcl_kv_t* raw, int L,
                                  int W, const int32_t* q_pos, float scale, const float* sink,
-                                 void* out, float* lse, void* ws, size_t ws_bytes,
-                                 int32_t* status, void* stream) {
-  return attn_common(0, q, B, Tq, H, d, kvc, Nc, 1, idx, k, raw, L, W, q_pos, scale, sink, out,
-                     lse, ws, ws_bytes, status, stream);
+                                 const float* q_gamma, float q_eps, void* out, float* lse,
+                                 void* ws, size_t ws_bytes, int32_t* status, void* stream) {
+  return attn_common(0, q, B, Tq, H, d, kvc, Nc, 1, idx, k, raw, L, W, q_pos, scale, sink,
+                     q_gamma, q_eps, out, lse, ws, ws_bytes, status, stream);
 }
 
 // The CSA attention with its split-KV partials in the library's fixed scratch array instead
@@ -352,8 +366,9 @@ hcl_status_t hcl_csa_sparse_attn_noalloc(const void* q, int B, int Tq, int H, in
     hcl_status_t e = hcl::noalloc_scratch(&scratch);
     if (e != HCL_OK) return e;
   }
-  return attn_common(0, q, B, Tq, H, d, kvc, Nc, 1, idx, k, raw, L, W, q_pos, scale, sink, out,
-                     lse, scratch, need > 0 ? hcl::NOALLOC_SCRATCH_BYTES : 0, status, stream);
+  return attn_common(0, q, B, Tq, H, d, kvc, Nc, 1, idx, k, raw, L, W, q_pos, scale, sink,
+                     nullptr, 0.f, out, lse, scratch, need > 0 ? hcl::NOALLOC_SCRATCH_BYTES : 0,
+                     status, stream);
 }
 
 size_t hcl_hca_dense_attn_workspace_bytes(int B, int Tq, int H, int Nh, int W) {
@@ -362,11 +377,11 @@ size_t hcl_hca_dense_attn_workspace_bytes(int B, int Tq, int H, int Nh, int W) {
 
 hcl_status_t hcl_hca_dense_attn(const void* q, int B, int Tq, int H, int d, const hcl_kv_t* kvh,
                                 int Nh, int mh, const hcl_kv_t* raw, int L, int W,
-                                const int32_t* q_pos, float scale, const float* sink, void* out,
-                                float* lse, void* ws, size_t ws_bytes, int32_t* status,
-                                void* stream) {
+                                const int32_t* q_pos, float scale, const float* sink,
+                                const float* q_gamma, float q_eps, void* out, float* lse,
+                                void* ws, size_t ws_bytes, int32_t* status, void* stream) {
   return attn_common(1, q, B, Tq, H, d, kvh, Nh, mh, nullptr, 0, raw, L, W, q_pos, scale, sink,
-                     out, lse, ws, ws_bytes, status, stream);
+                     q_gamma, q_eps, out, lse, ws, ws_bytes, status, stream);
 }
 
 // ---- fused decode step -----------------------------------------------------------------
@@ -414,8 +429,9 @@ hcl_status_t hcl_csa_decode_step(const void* q, const void* qI_bf16, const float
                                  int B, int H, int HI, int dI, int d, const hcl_kv_t* kvc,
                                  int Nc, int m, int k, const hcl_kv_t* raw, int L, int W,
                                  const int32_t* q_pos, float scale, const float* sink,
-                                 void* out, float* lse, int32_t* idx_out, void* ws,
-                                 size_t ws_bytes, int32_t* status, void* stream) {
+                                 const float* q_gamma, float q_eps, void* out, float* lse,
+                                 int32_t* idx_out, void* ws, size_t ws_bytes, int32_t* status,
+                                 void* stream) {
   if (dI != 64) return fail(HCL_ERR_UNSUPPORTED, "only dI == 64 is supported");
   const DecodeWs l = decode_ws_layout(B, H, HI, Nc, k, W, op_fmt, score_fmt, dI);
   HCL_REQUIRE(ws != nullptr && aligned16(ws) && ws_bytes >= l.total,
@@ -448,8 +464,55 @@ hcl_status_t hcl_csa_decode_step(const void* q, const void* qI_bf16, const float
   if (e != HCL_OK) return e;
   // the attention's predecessor is the top-k above, which writes neither q, q_pos nor the raw
   // window: the attention may load those before waiting for it
-  return attn_common(0, q, B, 1, H, d, kvc, Nc, 1, idx, k, raw, L, W, q_pos, scale, sink, out,
-                     lse, wsb + l.attn, ws_bytes - l.attn, status, stream, 1);
+  return attn_common(0, q, B, 1, H, d, kvc, Nc, 1, idx, k, raw, L, W, q_pos, scale, sink, q_gamma,
+                     q_eps, out, lse, wsb + l.attn, ws_bytes - l.attn, status, stream, 1);
+}
+
+hcl_status_t hcl_cache_append(const void* kv_new, const void* gate_new, const void* kI_new,
+                              const int32_t* t_new, int B, int d, int dI, void* stage_kv,
+                              void* stage_gate, int stage_cap, const hcl_kv_t* raw,
+                              const hcl_kv_t* kvc, const float* bias_csa, int m, int kI_fmt,
+                              void* kI, void* kI_sf, int kI_cap, const hcl_kv_t* kvh,
+                              const float* bias_hca, int mh, const float* gamma, float eps,
+                              int32_t* status, void* stream) {
+  (void)status;
+  HCL_REQUIRE(B >= 0, "B must be non-negative");
+  if (d != 128) return fail(HCL_ERR_UNSUPPORTED, "cache append: only d == 128 is supported");
+  if (B == 0) return HCL_OK;
+  HCL_REQUIRE(kv_new && gate_new && t_new && stage_kv && stage_gate, "NULL pointer");
+  HCL_REQUIRE(aligned16(kv_new) && aligned16(gate_new) && aligned16(stage_kv) &&
+                  aligned16(stage_gate),
+              "kv_new, gate_new and the staging rings must be 16-byte aligned");
+  hcl_status_t e = check_kv(raw, d, "raw");
+  if (e != HCL_OK) return e;
+  if (raw->fmt == HCL_FP8SPLIT) HCL_REQUIRE(((uintptr_t)raw->data & 7) == 0, "raw: codes must be 8-byte aligned");
+  int need_stage = 1;
+  if (kvc != nullptr) {
+    e = check_kv(kvc, d, "kvc");
+    if (e != HCL_OK) return e;
+    HCL_REQUIRE(m >= 1 && m <= 8, "m must be in [1, 8]");
+    HCL_REQUIRE(bias_csa != nullptr, "bias_csa must be given with kvc");
+    need_stage = 2 * m;
+    if (kI != nullptr) {
+      if (dI != 64) return fail(HCL_ERR_UNSUPPORTED, "cache append: only dI == 64 is supported");
+      HCL_REQUIRE(kI_new != nullptr && aligned16(kI_new) && aligned16(kI), "kI_new and kI must be 16-byte aligned");
+      HCL_REQUIRE(kI_cap >= 1, "kI_cap must be positive");
+      HCL_REQUIRE(kI_fmt == HCL_BF16 || (kI_fmt == HCL_MXFP4 && kI_sf != nullptr),
+                  "kI_fmt must be HCL_BF16, or HCL_MXFP4 with kI_sf");
+    }
+  }
+  if (kvh != nullptr) {
+    e = check_kv(kvh, d, "kvh");
+    if (e != HCL_OK) return e;
+    HCL_REQUIRE(mh >= 1 && mh <= 1024, "mh must be in [1, 1024]");
+    HCL_REQUIRE(bias_hca != nullptr, "bias_hca must be given with kvh");
+    if (mh > need_stage) need_stage = mh;
+  }
+  HCL_REQUIRE(stage_cap >= need_stage, "stage_cap must be >= %d (2m and mh)", need_stage);
+  if (gamma != nullptr) HCL_REQUIRE(eps > 0.f && eps < 1e30f, "eps must be a positive number");
+  CacheAppendArgs a{kv_new, gate_new, kI_new, t_new, B, stage_kv, stage_gate, stage_cap, *raw,
+                    kvc, bias_csa, m, kI_fmt, kI, kI_sf, kI_cap, kvh, bias_hca, mh, gamma, eps};
+  return launch_cache_append(a, as_stream(stream));
 }
 
 hcl_status_t hcl_selftest_bounded_wait(int32_t* status, int limit_us, void* stream) {

@@ -49,6 +49,8 @@ struct AttnParams {
   const int32_t* q_pos;
   float scale_log2;
   const float* sink;
+  const float* q_gamma;  // RMSNorm of every query head row (fp32 [d]), or null
+  float q_eps;
   __nv_bfloat16* out;
   float* lse;
   float* ws_o;
@@ -191,6 +193,34 @@ __global__ void __launch_bounds__(NW * 32)
       qa[kk][2] = qrow[0] ? *reinterpret_cast<const uint32_t*>(qrow[0] + c0 + 8) : 0u;
       qa[kk][3] = qrow[1] ? *reinterpret_cast<const uint32_t*>(qrow[1] + c0 + 8) : 0u;
     }
+  }
+  if (p.q_gamma != nullptr) {
+    // RMSNorm of the two query rows [Tripbot §5], fp32, rounded back to the bf16 operand: the
+    // four threads of a quad hold a row's 128 dims (fragment j: row j&1, dims c0 + 8*(j>>1))
+    float ss[2] = {0.f, 0.f};
+#pragma unroll
+    for (int kk = 0; kk < 8; kk++)
+#pragma unroll
+      for (int j = 0; j < 4; j++) {
+        const float lo = __uint_as_float(qa[kk][j] << 16), hi = __uint_as_float(qa[kk][j] & 0xFFFF0000u);
+        ss[j & 1] = fmaf(lo, lo, fmaf(hi, hi, ss[j & 1]));
+      }
+    float rn[2];
+#pragma unroll
+    for (int i = 0; i < 2; i++) {
+      ss[i] += __shfl_xor_sync(0xffffffffu, ss[i], 1);
+      ss[i] += __shfl_xor_sync(0xffffffffu, ss[i], 2);
+      rn[i] = 1.f / sqrtf(ss[i] / float(D) + p.q_eps);
+    }
+#pragma unroll
+    for (int kk = 0; kk < 8; kk++)
+#pragma unroll
+      for (int j = 0; j < 4; j++) {
+        const int c = kk * 16 + tq * 2 + 8 * (j >> 1);
+        const float lo = __uint_as_float(qa[kk][j] << 16), hi = __uint_as_float(qa[kk][j] & 0xFFFF0000u);
+        qa[kk][j] = pack_bf16(lo * rn[j & 1] * __ldg(p.q_gamma + c),
+                              hi * rn[j & 1] * __ldg(p.q_gamma + c + 1));
+      }
   }
 
   // A CSA block whose rows are all window rows needs nothing from the previous kernel (the
@@ -654,11 +684,40 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
   // Q: thread (row, hc) loads dims 64*hc .. 64*hc+63 of head `row` into SW128 half hc
   {
     const uint4* src = reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.H + row) * D) + hc * 8;
+    uint4 qv[8];
 #pragma unroll
-    for (int c = 0; c < 8; c++) {
-      const uint4 v = row < p.H ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-      *reinterpret_cast<uint4*>(sQ + hc * 16384 + row * 128 + ((c ^ (row & 7)) << 4)) = v;
+    for (int c = 0; c < 8; c++) qv[c] = row < p.H ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    if (p.q_gamma != nullptr) {
+      // RMSNorm of the head's query row [Tripbot §5]: the two threads of a row add their
+      // halves' sums of squares through shared memory; fp32, rounded back to bf16
+      float ss = 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; c++) {
+        const uint32_t w4[4] = {qv[c].x, qv[c].y, qv[c].z, qv[c].w};
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+          const float lo = __uint_as_float(w4[j] << 16), hi = __uint_as_float(w4[j] & 0xFFFF0000u);
+          ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+        }
+      }
+      xch[tid] = ss;
+      __syncthreads();
+      const float rn = 1.f / sqrtf((xch[row] + xch[row + TC_ROWS]) / float(D) + p.q_eps);
+#pragma unroll
+      for (int c = 0; c < 8; c++) {
+        uint32_t w4[4] = {qv[c].x, qv[c].y, qv[c].z, qv[c].w};
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+          const int dim = hc * 64 + c * 8 + 2 * j;
+          const float lo = __uint_as_float(w4[j] << 16), hi = __uint_as_float(w4[j] & 0xFFFF0000u);
+          w4[j] = pack_bf16(lo * rn * __ldg(p.q_gamma + dim), hi * rn * __ldg(p.q_gamma + dim + 1));
+        }
+        qv[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
     }
+#pragma unroll
+    for (int c = 0; c < 8; c++)
+      *reinterpret_cast<uint4*>(sQ + hc * 16384 + row * 128 + ((c ^ (row & 7)) << 4)) = qv[c];
   }
   if (early_ok && !early) pdl_enter();
 
@@ -960,10 +1019,19 @@ struct Plan {
 
 constexpr int MAX_CLUSTER = 16;
 
-// Blocks: one per (sequence, query group, split).  Splits spread a long row list over the
-// SMs when there are few groups; when the splits of a group fit one cluster (<= 16 blocks)
-// and there are enough groups for ~half the SMs, they merge through DSMEM (no workspace, no
-// merge launch); otherwise through the caller's workspace and a merge kernel.
+// Blocks: one per (sequence, query group, split).  The split of a query group's row list --
+// and so the order in which partial results are merged -- is a function of the per-sequence
+// shape only (queries per sequence, heads, list length), never of the batch size or of the
+// device: a sequence's output is then bitwise the same whatever batch it is decoded in
+// (batch-invariant kernels, [Tripbot §8 infrastructure table]).  A sequence with few query
+// groups (decode) splits its list into pieces of SPLIT_CHUNKS chunks so that its rows spread
+// over several SMs; with many groups every group is one block.  Splits of a group merge in a
+// cluster through DSMEM when they fit one (<= 16 blocks; no workspace, no merge launch),
+// otherwise through the caller's workspace and a merge kernel; both merge the splits of a row
+// in split order.
+constexpr int SPLIT_CHUNKS = 2;
+constexpr int FEW_GROUPS = 32;
+
 Plan make_plan(int mode, int B, int Tq, int H, int list_max) {
   Plan pl;
   pl.G = mode == 0 ? 1 : std::max(1, 128 / H);
@@ -973,18 +1041,12 @@ Plan make_plan(int mode, int B, int Tq, int H, int list_max) {
   pl.rows_pad = pl.NW * 16;
   pl.n_groups = (Tq + pl.G - 1) / pl.G;
   pl.n_chunks_max = std::max(1, (list_max + KVB - 1) / KVB);
-  const long long blocks = (long long)B * pl.n_groups;
-  const long long target = 2LL * num_sms();
-  int splits = (int)std::max(1LL, std::min<long long>(pl.n_chunks_max, (target + blocks - 1) / blocks));
-  pl.cmerge = 0;
-  if (splits > 1 && (splits <= MAX_CLUSTER || blocks * MAX_CLUSTER * 2 >= num_sms())) {
-    splits = std::min(splits, MAX_CLUSTER);
-    pl.cmerge = 1;
-  }
-  pl.cps = (pl.n_chunks_max + splits - 1) / splits;
+  pl.cps = pl.n_groups >= FEW_GROUPS ? pl.n_chunks_max : SPLIT_CHUNKS;
   pl.splits = (pl.n_chunks_max + pl.cps - 1) / pl.cps;
-  if (pl.splits == 1) pl.cmerge = 0;
-  // few clusters of 8-warp blocks leave SMs idle: halve the rows per block instead
+  pl.cmerge = pl.splits > 1 && pl.splits <= MAX_CLUSTER;
+  // few clusters of 8-warp blocks leave SMs idle: halve the rows per block instead (each
+  // (query, head) row's arithmetic is the same in either shape, so the bits do not change)
+  const long long blocks = (long long)B * pl.n_groups;
   pl.hsplit = 1;
   if (pl.cmerge && pl.NW == 8 && blocks * pl.splits * 2 <= num_sms()) {
     pl.hsplit = 2;
@@ -1104,6 +1166,8 @@ hcl_status_t launch_attn(const AttnArgs& a, void* ws, size_t ws_bytes, cudaStrea
   p.q_pos = a.q_pos;
   p.scale_log2 = a.scale * LOG2E;
   p.sink = a.sink;
+  p.q_gamma = a.q_gamma;
+  p.q_eps = a.q_eps;
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.lse = a.lse;
   p.G = pl.G; p.n_groups = pl.n_groups; p.splits = pl.splits; p.cps = pl.cps;

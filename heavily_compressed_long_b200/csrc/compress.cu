@@ -7,45 +7,26 @@
 // token t_j (slots outside [0, L) dropped):
 //     out[i, c] = sum_j softmax_j(gate[t_j, c] + bias[j]) * kv[t_j, c]
 //
-// HBM-streaming kernel: each thread owns 8 channels (one 16-byte load of kv and of gate per
-// token row, coalesced along d) and keeps an online (max, sum, weighted sum) softmax in fp32.
-// Small spans (CSA: 2m <= 16) give each entry to one group of d/8 threads; long spans (HCA)
-// split the slots over the 128 threads of a block and merge the partial softmaxes in shared
-// memory.
+// HBM-streaming kernels: each thread owns 8 channels (one 16-byte load of kv and of gate per
+// token row, coalesced along d) and keeps an online (max, sum, weighted sum) softmax in fp32
+// (pool.cuh).  Small spans give each entry to one group of d/8 threads; the CSA span 2m = 8 is
+// a compile-time span, so all 16 row loads of an entry are in flight before the arithmetic
+// (a slot-by-slot loop waits one memory latency per slot).  Long spans (HCA) split the slots
+// over the 128 threads of a block, four slots' loads in flight per thread, and merge the
+// partial softmaxes in shared memory.
+//
+// Optional RMSNorm epilogue [Tripbot §5: queries and compressed KV entries are RMS-normalised,
+// so attention needs no extra QK normalisation]: with gamma given, every pooled entry c is
+// written as c / sqrt(mean_ch(c^2) + eps) * gamma, in fp32 before the output rounding (so
+// before any later quantisation of the cache).
 #include <cuda_bf16.h>
 
 #include "hcl_common.cuh"
 #include "hcl_internal.h"
+#include "pool.cuh"
 
 namespace hcl {
 namespace {
-
-struct Online8 {
-  float mx[8], sum[8], acc[8];
-  __device__ void init() {
-#pragma unroll
-    for (int c = 0; c < 8; c++) { mx[c] = -INFINITY; sum[c] = 0.f; acc[c] = 0.f; }
-  }
-  __device__ void add(const uint4& xv, const uint4& gv, float b) {
-    const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(&xv);
-    const __nv_bfloat16* g = reinterpret_cast<const __nv_bfloat16*>(&gv);
-#pragma unroll
-    for (int c = 0; c < 8; c++) {
-      float z = bf2f(g[c]) + b;
-      float xc = bf2f(x[c]);
-      if (z > mx[c]) {
-        float r = __expf(mx[c] - z);  // exp(-inf) = 0 on the first slot
-        sum[c] = sum[c] * r + 1.f;
-        acc[c] = acc[c] * r + xc;
-        mx[c] = z;
-      } else {
-        float e = __expf(z - mx[c]);
-        sum[c] += e;
-        acc[c] += e * xc;
-      }
-    }
-  }
-};
 
 __device__ __forceinline__ void store8(void* out, int out_fmt, size_t off, const float* v) {
   if (out_fmt == HCL_FP32) {
@@ -61,87 +42,66 @@ __device__ __forceinline__ void store8(void* out, int out_fmt, size_t off, const
   }
 }
 
-// One group of G = d/8 threads per entry.
+// One group of G = d/8 threads per entry; SPAN > 0: compile-time span, else `span`.
+template <int SPAN>
 __global__ void compress_small_kernel(const __nv_bfloat16* __restrict__ kv,
                                       const __nv_bfloat16* __restrict__ gate,
                                       const float* __restrict__ bias, int B, int L, int d,
                                       int m, int span, int first_off, int e0, int e1, void* out,
-                                      int out_fmt, int out_cap) {
+                                      int out_fmt, int out_cap, const float* __restrict__ gamma,
+                                      float eps) {
   const int G = d >> 3;
   const long long n_ent = (long long)(e1 - e0) * B;
   const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long item = gt / G;
   const int chunk = int(gt % G);
-  if (item >= n_ent) return;
+  if (item >= n_ent) return;  // whole groups only (G divides the block)
   const int b = int(item / (e1 - e0));
   const int i = e0 + int(item % (e1 - e0));
   const long long first = (long long)m * i + first_off;
-  Online8 s;
-  s.init();
-  for (int j = 0; j < span; j++) {
-    long long t = first + j;
-    if (t < 0 || t >= L) continue;
-    size_t off = ((size_t)b * L + t) * d + chunk * 8;
-    uint4 xv = __ldg(reinterpret_cast<const uint4*>(kv + off));
-    uint4 gv = __ldg(reinterpret_cast<const uint4*>(gate + off));
-    s.add(xv, gv, __ldg(bias + j));
-  }
+  const __nv_bfloat16* kvb = kv + (size_t)b * L * d;
+  const __nv_bfloat16* gb = gate + (size_t)b * L * d;
+  auto row = [&](int j, const __nv_bfloat16*& kp, const __nv_bfloat16*& gp) {
+    const long long t = first + j;
+    if (t < 0 || t >= L) return false;
+    kp = kvb + (size_t)t * d;
+    gp = gb + (size_t)t * d;
+    return true;
+  };
   float v[8];
-#pragma unroll
-  for (int c = 0; c < 8; c++) v[c] = s.sum[c] > 0.f ? s.acc[c] / s.sum[c] : 0.f;
+  if (SPAN > 0) pool8_span<(SPAN > 0 ? SPAN : 1)>(row, bias, chunk, v);
+  else pool8_any(row, bias, span, chunk, v);
+  if (gamma != nullptr) rmsnorm8_group(v, G, d, chunk, gamma, eps);
   store8(out, out_fmt, ((size_t)b * out_cap + i) * d + chunk * 8, v);
 }
 
-// One block of 128 threads per entry; the span is split over 128/G slot streams.
+// One block of 128 threads per entry (pool_long_block).
 __global__ void __launch_bounds__(128) compress_long_kernel(
     const __nv_bfloat16* __restrict__ kv, const __nv_bfloat16* __restrict__ gate,
     const float* __restrict__ bias, int B, int L, int d, int m, int span, int e0, int e1,
-    void* out, int out_fmt, int out_cap) {
-  extern __shared__ float sm[];  // [streams][3][d]
-  const int G = d >> 3;
-  const int streams = 128 / G;
-  const int chunk = threadIdx.x % G;
-  const int stream = threadIdx.x / G;
+    void* out, int out_fmt, int out_cap, const float* __restrict__ gamma, float eps) {
+  extern __shared__ float sm[];  // [streams][3][d], then 4 floats for the RMSNorm reduction
   const int b = blockIdx.x / (e1 - e0);
   const int i = e0 + blockIdx.x % (e1 - e0);
   const long long first = (long long)m * i;
-  Online8 s;
-  s.init();
-  if (stream < streams) {
-    for (int j = stream; j < span; j += streams) {
-      long long t = first + j;
-      if (t < 0 || t >= L) continue;
-      size_t off = ((size_t)b * L + t) * d + chunk * 8;
-      uint4 xv = __ldg(reinterpret_cast<const uint4*>(kv + off));
-      uint4 gv = __ldg(reinterpret_cast<const uint4*>(gate + off));
-      s.add(xv, gv, __ldg(bias + j));
-    }
-    float* base = sm + (size_t)stream * 3 * d;
+  const __nv_bfloat16* kvb = kv + (size_t)b * L * d;
+  const __nv_bfloat16* gb = gate + (size_t)b * L * d;
+  auto row = [&](int j, const __nv_bfloat16*& kp, const __nv_bfloat16*& gp) {
+    const long long t = first + j;
+    if (t < 0 || t >= L) return false;
+    kp = kvb + (size_t)t * d;
+    gp = gb + (size_t)t * d;
+    return true;
+  };
+  float vals[8];
+  pool_long_block(row, bias, span, d, sm, gamma, eps, vals);
 #pragma unroll
-    for (int c = 0; c < 8; c++) {
-      base[chunk * 8 + c] = s.mx[c];
-      base[d + chunk * 8 + c] = s.sum[c];
-      base[2 * d + chunk * 8 + c] = s.acc[c];
-    }
-  }
-  __syncthreads();
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    float M = -INFINITY;
-    for (int q = 0; q < streams; q++) M = fmaxf(M, sm[(size_t)q * 3 * d + c]);
-    float S = 0.f, A = 0.f;
-    if (M > -INFINITY) {
-      for (int q = 0; q < streams; q++) {
-        const float* base = sm + (size_t)q * 3 * d;
-        if (base[c] == -INFINITY) continue;
-        float r = __expf(base[c] - M);
-        S += base[d + c] * r;
-        A += base[2 * d + c] * r;
-      }
-    }
-    float v = S > 0.f ? A / S : 0.f;
-    size_t o = ((size_t)b * out_cap + i) * d + c;
-    if (out_fmt == HCL_FP32) static_cast<float*>(out)[o] = v;
-    else static_cast<__nv_bfloat16*>(out)[o] = __float2bfloat16_rn(v);
+  for (int u = 0; u < 8; u++) {
+    const int c = threadIdx.x + u * 128;
+    if (c >= d) continue;
+    const size_t o = ((size_t)b * out_cap + i) * d + c;
+    if (out_fmt == HCL_FP32) static_cast<float*>(out)[o] = vals[u];
+    else static_cast<__nv_bfloat16*>(out)[o] = __float2bfloat16_rn(vals[u]);
   }
 }
 
@@ -149,25 +109,32 @@ __global__ void __launch_bounds__(128) compress_long_kernel(
 
 hcl_status_t launch_compress(const void* kv, const void* gate, const float* bias, int B, int L,
                              int d, int m, int overlap, int e0, int e1, void* out, int out_fmt,
-                             int out_cap, cudaStream_t st) {
+                             int out_cap, const float* gamma, float eps, cudaStream_t st) {
   if (e1 <= e0 || B == 0) return HCL_OK;
   const int span = overlap ? 2 * m : m;
   const int G = d / 8;
   auto kvp = static_cast<const __nv_bfloat16*>(kv);
   auto gp = static_cast<const __nv_bfloat16*>(gate);
   if (span <= 16 || 128 % G != 0) {
-    long long threads = (long long)(e1 - e0) * B * G;
-    int blk = 256;
-    long long grid = (threads + blk - 1) / blk;
-    compress_small_kernel<<<(unsigned)grid, blk, 0, st>>>(kvp, gp, bias, B, L, d, m, span,
-                                                          overlap ? -m : 0, e0, e1, out, out_fmt,
-                                                          out_cap);
+    const long long threads = (long long)(e1 - e0) * B * G;
+    // whole groups per block: a multiple of G threads (G <= 128)
+    const int blk = (256 / G) * G;
+    const long long grid = (threads + blk - 1) / blk;
+    const int first_off = overlap ? -m : 0;
+    if (span == 8)
+      compress_small_kernel<8><<<(unsigned)grid, blk, 0, st>>>(kvp, gp, bias, B, L, d, m, span,
+                                                                first_off, e0, e1, out, out_fmt,
+                                                                out_cap, gamma, eps);
+    else
+      compress_small_kernel<0><<<(unsigned)grid, blk, 0, st>>>(kvp, gp, bias, B, L, d, m, span,
+                                                                first_off, e0, e1, out, out_fmt,
+                                                                out_cap, gamma, eps);
   } else {
     const int streams = 128 / G;
-    size_t smem = (size_t)streams * 3 * d * sizeof(float);
-    long long grid = (long long)(e1 - e0) * B;
+    const size_t smem = ((size_t)streams * 3 * d + 4) * sizeof(float);
+    const long long grid = (long long)(e1 - e0) * B;
     compress_long_kernel<<<(unsigned)grid, 128, smem, st>>>(kvp, gp, bias, B, L, d, m, span, e0,
-                                                            e1, out, out_fmt, out_cap);
+                                                            e1, out, out_fmt, out_cap, gamma, eps);
   }
   return check_launch("compress");
 }

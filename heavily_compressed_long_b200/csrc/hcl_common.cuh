@@ -31,6 +31,13 @@ __device__ __forceinline__ void report(int32_t* status, int code) {
 __device__ __forceinline__ float bf2f(__nv_bfloat16 v) { return __bfloat162float(v); }
 __device__ __forceinline__ float bfbits2f(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
 
+// Two fp32 -> two E4M3 (round to nearest even, saturate to the finite range), lo in byte 0.
+__device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -70,9 +70,10 @@ EncodeTiledFn encode_tiled();
 
 // ---- launchers (each validates nothing; the extern "C" layer does) ----
 
+// gamma (fp32 [d]) non-null: RMSNorm epilogue with epsilon eps.
 hcl_status_t launch_compress(const void* kv, const void* gate, const float* bias, int B, int L,
                              int d, int m, int overlap, int e0, int e1, void* out, int out_fmt,
-                             int out_cap, cudaStream_t st);
+                             int out_cap, const float* gamma, float eps, cudaStream_t st);
 
 hcl_status_t launch_quant_kv_fp8(const void* kv, int64_t rows, int d, void* nope, float* scale,
                                  void* rope, cudaStream_t st);
@@ -143,10 +144,38 @@ struct AttnArgs {
   float* lse;
   int32_t* status;
   int prewait = 0;  // 1: q, q_pos and raw do not come from the previous kernel in the stream
+  const float* q_gamma = nullptr;  // RMSNorm of the query rows (fp32 [d]), or null
+  float q_eps = 0.f;
 };
 // n = k (CSA) or Nh (HCA)
 size_t attn_workspace_bytes(int mode, int B, int Tq, int H, int n, int W);
 hcl_status_t launch_attn(const AttnArgs& a, void* ws, size_t ws_bytes, cudaStream_t st);
+
+// Decode-time cache append (one token per sequence); kvc / kvh null: no CSA / HCA store.
+struct CacheAppendArgs {
+  const void* kv_new;
+  const void* gate_new;
+  const void* kI_new;
+  const int32_t* t_new;
+  int B;
+  void* stage_kv;
+  void* stage_gate;
+  int stage_cap;
+  hcl_kv_t raw;
+  const hcl_kv_t* kvc;
+  const float* bias_csa;
+  int m;
+  int kI_fmt;
+  void* kI;
+  void* kI_sf;
+  int kI_cap;
+  const hcl_kv_t* kvh;
+  const float* bias_hca;
+  int mh;
+  const float* gamma;
+  float eps;
+};
+hcl_status_t launch_cache_append(const CacheAppendArgs& a, cudaStream_t st);
 
 // Fixed device scratch of hcl_csa_sparse_attn_noalloc (split-KV partials), and its device
 // address on the current device (looked up once per device).

@@ -14,13 +14,6 @@
 namespace hcl {
 namespace {
 
-// Two fp32 -> two E4M3 (round to nearest even, saturate to the finite range), lo in byte 0.
-__device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
 // One group of d/8 threads per row: the first half of the group holds dims 0..d/2-1.
 __global__ void quant_kv_fp8_kernel(const __nv_bfloat16* __restrict__ kv, long long rows, int d,
                                     uint8_t* __restrict__ nope, float* __restrict__ scale,

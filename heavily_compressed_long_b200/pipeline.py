@@ -17,8 +17,10 @@ class CsaDecode:
     packed [B,cap,dI/2] + kI_sf [B,cap,dI/32]; kvc / raw: api.KV stores; q_pos [B,1] int32."""
 
     def __init__(self, q, qI, w, kI, kvc: KV, Nc, raw: KV, L, W, q_pos, m=4, k=1024,
-                 op_fmt=HCL_BF16, score_fmt=HCL_FP32, kI_sf=None, sink=None):
+                 op_fmt=HCL_BF16, score_fmt=HCL_FP32, kI_sf=None, sink=None, q_gamma=None,
+                 q_eps=1e-6):
         self.q, self.qI, self.w, self.kI, self.kI_sf = q, qI, w, kI, kI_sf
+        self.q_gamma, self.q_eps = q_gamma, q_eps
         self.kvc, self.raw, self.Nc, self.L, self.W, self.q_pos = kvc, raw, Nc, L, W, q_pos
         self.m, self.k, self.op_fmt, self.score_fmt, self.sink = m, k, op_fmt, score_fmt, sink
         B, _, H, d = q.shape
@@ -60,7 +62,8 @@ class CsaDecode:
                          stream=stream)
         api.hcl_csa_sparse_attn(self.q, self.kvc, self.Nc, self.idx, self.raw, self.L, self.W,
                                 self.q_pos, self.out, lse=self.lse, sink=self.sink,
-                                ws=self.attn_ws, status=self.status, stream=stream)
+                                ws=self.attn_ws, status=self.status, q_gamma=self.q_gamma,
+                                q_eps=self.q_eps, stream=stream)
         return self.out
 
     def step(self, stream=None):
@@ -69,7 +72,8 @@ class CsaDecode:
                                 self.m, self.k, self.raw, self.L, self.W, self.q_pos, self.out,
                                 score_fmt=self.score_fmt, kI_sf=self.kI_sf, lse=self.lse,
                                 idx_out=self.idx, sink=self.sink, ws=self.step_ws,
-                                status=self.status, stream=stream)
+                                status=self.status, q_gamma=self.q_gamma, q_eps=self.q_eps,
+                                stream=stream)
         return self.out
 
 
@@ -77,9 +81,10 @@ class HcaLayer:
     """HCA attention over the compressed entries plus the raw window for Tq queries per
     sequence (a prefill chunk, or Tq = 1 for decode); optionally compresses entries first."""
 
-    def __init__(self, q, kvh: KV, Nh, mh, raw: KV, L, W, q_pos, sink=None):
+    def __init__(self, q, kvh: KV, Nh, mh, raw: KV, L, W, q_pos, sink=None, q_gamma=None,
+                 q_eps=1e-6):
         self.q, self.kvh, self.Nh, self.mh, self.raw, self.L, self.W = q, kvh, Nh, mh, raw, L, W
-        self.q_pos, self.sink = q_pos, sink
+        self.q_pos, self.sink, self.q_gamma, self.q_eps = q_pos, sink, q_gamma, q_eps
         B, Tq, H, d = q.shape
         self.out = torch.empty(B, Tq, H, d, dtype=torch.bfloat16, device=q.device)
         self.lse = torch.empty(B, Tq, H, dtype=torch.float32, device=q.device)
@@ -90,7 +95,8 @@ class HcaLayer:
     def step(self, stream=None):
         api.hcl_hca_dense_attn(self.q, self.kvh, self.Nh, self.mh, self.raw, self.L, self.W,
                                self.q_pos, self.out, lse=self.lse, sink=self.sink, ws=self.ws,
-                               status=self.status, stream=stream)
+                               status=self.status, q_gamma=self.q_gamma, q_eps=self.q_eps,
+                               stream=stream)
         return self.out
 
 

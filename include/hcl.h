@@ -100,16 +100,23 @@ HCL_API const char* hcl_last_error(void);
  * kv, gate: bf16 [B, L, d]; bias: fp32 [2m]; out: [B, out_cap, d] in out_fmt (HCL_FP32 or
  * HCL_BF16), entry i written at row i.  Requires 0 <= entry_begin <= entry_end <=
  * min(ceil(L/m), out_cap), d % 8 == 0, 1 <= m <= 64.  Accumulates in fp32.
+ * RMSNorm of the entries [Tripbot §5: compressed KV entries are RMS-normalised]: with gamma
+ * (fp32 [d]) given, each pooled entry c is written as c / sqrt(mean_ch(c^2) + eps) * gamma,
+ * computed in fp32 before the output rounding (NULL: no normalisation; eps >= 0).  With
+ * gamma, d/8 must be a power of two <= 32 (d = 8 .. 256); otherwise HCL_ERR_UNSUPPORTED.
  */
 HCL_API hcl_status_t hcl_csa_compress(const void* kv, const void* gate, const float* bias, int B, int L,
                               int d, int m, int entry_begin, int entry_end, void* out,
-                              int out_fmt, int out_cap, void* stream);
+                              int out_fmt, int out_cap, const float* gamma, float eps,
+                              void* stream);
 
 /* a2 -- HCA compressor [Tripbot §3.2; CSDN §1.2]: as above with span m (no overlap):
- * entry i pools tokens m*i .. m*i+m-1; bias: fp32 [m]; 1 <= m <= 1024. */
+ * entry i pools tokens m*i .. m*i+m-1; bias: fp32 [m]; 1 <= m <= 1024; the same optional
+ * RMSNorm epilogue (gamma, eps). */
 HCL_API hcl_status_t hcl_hca_compress(const void* kv, const void* gate, const float* bias, int B, int L,
                               int d, int m, int entry_begin, int entry_end, void* out,
-                              int out_fmt, int out_cap, void* stream);
+                              int out_fmt, int out_cap, const float* gamma, float eps,
+                              void* stream);
 
 /* ---------------------------------------------------------------------------------------
  * a3 -- cache quantisers [CSDN §1.4; Austery infra].
@@ -165,6 +172,10 @@ HCL_API hcl_status_t hcl_csa_topk(const void* scores, int score_fmt, int B, int 
  *     z_j = scale * q[b,t,h,:] . row_j;  out = sum_j softmax(z)_j row_j;  lse = log sum exp z
  * With a sink (fp32 [H] logits, or NULL) the softmax denominator also has exp(sink[h]) and
  * the sink contributes no value.  No rows and no sink: out = 0, lse = -inf.
+ * Query RMSNorm [Tripbot §5: queries are RMS-normalised before attention]: with q_gamma
+ * (fp32 [d]) given, every query head row is used as q / sqrt(mean(q^2) + q_eps) * q_gamma,
+ * computed in fp32 and rounded to bf16 (the tensor-core operand) before the dot products
+ * (NULL: q as given; q_eps > 0).
  *   q bf16 [B, Tq, H, d]; idx int32 [B, Tq, k] (entries < Nc; -1 = none); out bf16
  *   [B, Tq, H, d]; lse fp32 [B, Tq, H] or NULL.  d == 128, 1 <= H <= 128.
  *   ws: hcl_csa_sparse_attn_workspace_bytes() bytes (split-KV partial results).
@@ -174,12 +185,13 @@ HCL_API size_t hcl_csa_sparse_attn_workspace_bytes(int B, int Tq, int H, int k, 
 HCL_API hcl_status_t hcl_csa_sparse_attn(const void* q, int B, int Tq, int H, int d, const hcl_kv_t* kvc,
                                  int Nc, const int32_t* idx, int k, const hcl_kv_t* raw, int L,
                                  int W, const int32_t* q_pos, float scale, const float* sink,
-                                 void* out, float* lse, void* ws, size_t ws_bytes,
-                                 int32_t* status, void* stream);
+                                 const float* q_gamma, float q_eps, void* out, float* lse,
+                                 void* ws, size_t ws_bytes, int32_t* status, void* stream);
 
 /* ---------------------------------------------------------------------------------------
  * hcl_csa_sparse_attn_noalloc -- the CSA attention above for callers that cannot allocate
- * device memory.  (The paper has no counterpart; this is a deployment variant.)
+ * device memory (without the query RMSNorm).  (The paper has no counterpart; this is a
+ * deployment variant.)
  * Some callers may not call cudaMalloc at all: serving runtimes that reserve the device's
  * memory up front for their own pool and forbid allocation on the request path (cudaMalloc
  * can synchronise the device and fail once the pool owns the memory), and plugin hosts that
@@ -204,16 +216,17 @@ HCL_API hcl_status_t hcl_csa_sparse_attn_noalloc(const void* q, int B, int Tq, i
                                          void* out, float* lse, int32_t* status, void* stream);
 
 /* ---------------------------------------------------------------------------------------
- * a7 -- HCA attention [Tripbot §3.2, §3.3; CSDN §1.2].  As a6 with J = { kvh entry i :
- * 0 <= i < Nh, mh*(i+1) - 1 <= p } followed by the window: dense, no selection.
+ * a7 -- HCA attention [Tripbot §3.2, §3.3; CSDN §1.2].  As a6 (sink, query RMSNorm) with
+ * J = { kvh entry i : 0 <= i < Nh, mh*(i+1) - 1 <= p } followed by the window: dense, no
+ * selection.
  *   kvh: [B, cap, d] rows (cap >= Nh).  d == 128, 1 <= H <= 128.
  */
 HCL_API size_t hcl_hca_dense_attn_workspace_bytes(int B, int Tq, int H, int Nh, int W);
 HCL_API hcl_status_t hcl_hca_dense_attn(const void* q, int B, int Tq, int H, int d, const hcl_kv_t* kvh,
                                 int Nh, int mh, const hcl_kv_t* raw, int L, int W,
-                                const int32_t* q_pos, float scale, const float* sink, void* out,
-                                float* lse, void* ws, size_t ws_bytes, int32_t* status,
-                                void* stream);
+                                const int32_t* q_pos, float scale, const float* sink,
+                                const float* q_gamma, float q_eps, void* out, float* lse,
+                                void* ws, size_t ws_bytes, int32_t* status, void* stream);
 
 /* ---------------------------------------------------------------------------------------
  * Fused CSA decode step [Tripbot §3.1]: for each sequence, the new query's index queries are
@@ -233,8 +246,46 @@ HCL_API hcl_status_t hcl_csa_decode_step(const void* q, const void* qI_bf16, con
                                  int B, int H, int HI, int dI, int d, const hcl_kv_t* kvc,
                                  int Nc, int m, int k, const hcl_kv_t* raw, int L, int W,
                                  const int32_t* q_pos, float scale, const float* sink,
-                                 void* out, float* lse, int32_t* idx_out, void* ws,
-                                 size_t ws_bytes, int32_t* status, void* stream);
+                                 const float* q_gamma, float q_eps, void* out, float* lse,
+                                 int32_t* idx_out, void* ws, size_t ws_bytes, int32_t* status,
+                                 void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Decode-time cache maintenance [Yanbaoke §5 KV cache management: a heterogeneous KV cache;
+ * Austery's talk notes, infrastructure section].  Appends one new raw token per sequence to
+ * one layer's cache, on `stream`, before that step's attention reads it:
+ *   kv_new, gate_new: bf16 [B, d], the token's KV row and gate logits; t_new: int32 [B], its
+ *   absolute position (< 0: the sequence appends nothing this step).
+ *   stage_kv, stage_gate: bf16 [B, stage_cap, d], caller-owned staging rings holding the token
+ *   rows the compressors still need; token u lives at slot u mod stage_cap.  stage_cap >= 2m
+ *   (with kvc) and >= mh (with kvh); before the first call the rings must hold the tokens
+ *   before t_new that the next entries pool (the last 2m - 1 / mh - 1 tokens).
+ *   raw: the raw sliding-window store (hcl_kv_t, HCL_BF16 or HCL_FP8SPLIT); token t is written
+ *   at slot t mod raw->cap (split rows: E4M3 codes with scale amax/448 and the bf16 RoPE half,
+ *   bit-identical to hcl_quant_kv_fp8).
+ *   kvc (or NULL, an HCA layer): the CSA entry store.  When (t+1) % m == 0, entry i = t/m is
+ *   pooled from tokens m(i-1) .. m*i+m-1 with bias_csa (fp32 [2m]) exactly as
+ *   hcl_csa_compress computes it, optionally RMS-normalised (gamma, eps as in
+ *   hcl_csa_compress), rounded to bf16 and written at slot i mod kvc->cap (split rows
+ *   quantised as above).  With kI non-NULL the entry's index key kI_new (bf16 [B, dI]) is
+ *   written at slot i mod kI_cap of kI: HCL_BF16 rows [B, kI_cap, dI], or HCL_MXFP4 packed
+ *   [B, kI_cap, dI/2] + kI_sf E8M0 [B, kI_cap, dI/32] (bit-identical to hcl_quant_mxfp4).
+ *   1 <= m <= 8; dI == 64.
+ *   kvh (or NULL, a CSA layer): the HCA entry store.  When (t+1) % mh == 0, entry i = t/mh is
+ *   pooled from tokens mh*i .. mh*i+mh-1 with bias_hca (fp32 [mh]) as hcl_hca_compress
+ *   computes it (and normalised with gamma), written at slot i mod kvh->cap.  1 <= mh <= 1024.
+ * d == 128.  The call writes through the store pointers of raw, kvc and kvh (their `const`
+ * only means the attention calls read them).  Sequences are independent; two calls that
+ * overlap on the GPU on the same cache race.  status: unused (may be NULL).
+ */
+HCL_API hcl_status_t hcl_cache_append(const void* kv_new, const void* gate_new,
+                                      const void* kI_new, const int32_t* t_new, int B, int d,
+                                      int dI, void* stage_kv, void* stage_gate, int stage_cap,
+                                      const hcl_kv_t* raw, const hcl_kv_t* kvc,
+                                      const float* bias_csa, int m, int kI_fmt, void* kI,
+                                      void* kI_sf, int kI_cap, const hcl_kv_t* kvh,
+                                      const float* bias_hca, int mh, const float* gamma,
+                                      float eps, int32_t* status, void* stream);
 
 /* ---------------------------------------------------------------------------------------
  * Failure-detection self-test: launches one block whose bounded wait on an mbarrier that

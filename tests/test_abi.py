@@ -69,7 +69,8 @@ def test_host_validation_without_device(libhcl):
     rc = L.hcl_csa_topk(fake, libhcl.HCL_FP32, 1, 1, 100, fake, 4, 5000, fake, None, 0, None, None)
     assert rc == libhcl.HCL_ERR_INVALID_ARG
     # compressor: entry range beyond ceil(L/m)
-    rc = L.hcl_csa_compress(fake, fake, fake, 1, 40, 128, 4, 0, 11, fake, libhcl.HCL_FP32, 64, None)
+    rc = L.hcl_csa_compress(fake, fake, fake, 1, 40, 128, 4, 0, 11, fake, libhcl.HCL_FP32, 64, None,
+                            0.0, None)
     assert rc == libhcl.HCL_ERR_INVALID_ARG
     # misaligned pointer
     rc = L.hcl_quant_kv_fp8(ctypes.c_void_p((1 << 20) + 4), 4, 128, fake, fake, fake, None)
@@ -77,11 +78,11 @@ def test_host_validation_without_device(libhcl):
     # attention: d != 128 unsupported; kv descriptor format check
     kv = libhcl.hcl_kv_t(libhcl.HCL_BF16, 16, fake.value, None, None)
     rc = L.hcl_csa_sparse_attn(fake, 1, 1, 8, 64, ctypes.byref(kv), 16, fake, 4, ctypes.byref(kv),
-                               64, 8, fake, 0.1, None, fake, None, None, 0, None, None)
+                               64, 8, fake, 0.1, None, None, 0.0, fake, None, None, 0, None, None)
     assert rc == libhcl.HCL_ERR_UNSUPPORTED
     bad = libhcl.hcl_kv_t(7, 16, fake.value, None, None)
     rc = L.hcl_csa_sparse_attn(fake, 1, 1, 8, 128, ctypes.byref(bad), 16, fake, 4, ctypes.byref(kv),
-                               64, 8, fake, 0.1, None, fake, None, None, 0, None, None)
+                               64, 8, fake, 0.1, None, None, 0.0, fake, None, None, 0, None, None)
     assert rc == libhcl.HCL_ERR_INVALID_ARG
     # empty problems are a no-op success
     assert L.hcl_quant_mxfp4(None, 0, 64, None, None, None) == libhcl.HCL_OK

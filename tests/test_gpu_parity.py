@@ -85,6 +85,28 @@ def test_compress(hcl, B, L, m, overlap):
     assert bf16_out_ratio(as_f64(out16), ref) <= 1.0
 
 
+@pytest.mark.parametrize("B,L,m,overlap", [(1, 4096, 4, True), (2, 1027, 4, True),
+                                           (2, 128 * 37 + 5, 128, False)])
+def test_compress_rmsnorm(hcl, B, L, m, overlap):
+    """The compressor's RMSNorm epilogue against or_rmsnorm applied to or_compress (entries
+    normalised after pooling, before the output rounding)."""
+    d, eps = 128, 1e-6
+    x, g = rbf16(B, L, d), rbf16(B, L, d)
+    span = 2 * m if overlap else m
+    bias = torch.from_numpy((RNG.standard_normal(span) * 0.1).astype(np.float32))
+    gamma = torch.from_numpy((1.0 + 0.25 * RNG.standard_normal(d)).astype(np.float32))
+    ref = oracle.rmsnorm(oracle.compress(x, g, bias, m, overlap), gamma, eps)
+    n = ref.shape[1]
+    fn = hcl.hcl_csa_compress if overlap else hcl.hcl_hca_compress
+    out32 = torch.empty(B, n, d, device="cuda")
+    fn(cuda(x), cuda(g), cuda(bias), m, out32, gamma=cuda(gamma), eps=eps)
+    out16 = torch.empty(B, n, d, dtype=torch.bfloat16, device="cuda")
+    fn(cuda(x), cuda(g), cuda(bias), m, out16, gamma=cuda(gamma), eps=eps)
+    torch.cuda.synchronize()
+    assert rel_rowwise(as_f64(out32), ref) <= 1e-3
+    assert bf16_out_ratio(as_f64(out16), ref) <= 1.0
+
+
 def test_compress_entry_range(hcl):
     B, L, d = 1, 2000, 128
     x, g = rbf16(B, L, d), rbf16(B, L, d)
@@ -312,6 +334,57 @@ def test_csa_attn(hcl, B, Tq, H, Nc, k, W, fp8, sink):
     assert np.abs(as_f64(lse) - l_ref).max() <= tol
 
 
+def _normed_q(q, gamma, eps):
+    """The oracle's RMSNorm of every query head row, rounded to bf16 (the attention's operand
+    precision), as a bf16 tensor."""
+    qn = oracle.round_bf16(oracle.rmsnorm(q, gamma, eps))
+    return torch.from_numpy(qn.astype(np.float32)).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("B,Tq,H,Nc,k,W,fp8", [
+    (1, 1, 8, 1024, 64, 64, False),             # cfg-1 shape
+    (2, 1, 128, 9000, 1024, 128, True),         # cfg-4 shape (tcgen05 decode kernel)
+    (1, 3, 16, 700, 100, 37, False),            # several queries (mma.sync kernel)
+])
+def test_csa_attn_query_rmsnorm(hcl, B, Tq, H, Nc, k, W, fp8):
+    """Attention on RMS-normalised queries: the oracle normalises q (fp64, then bf16) and
+    attends; the kernels normalise in their query load."""
+    d, L, eps = 128, 4 * Nc + 11, 1e-6
+    ent, raw = rbf16(B, Nc, d), rbf16(B, L, d)
+    q = rbf16(B, Tq, H, d, std=3.0)
+    gamma = torch.from_numpy((1.0 + 0.25 * RNG.standard_normal(d)).astype(np.float32))
+    pos = torch.from_numpy(RNG.integers(L - 300, L, (B, Tq)).astype(np.int32))
+    idx = np.stack([[np.sort(RNG.choice(Nc, k, replace=False)) for _ in range(Tq)] for _ in range(B)]).astype(np.int32)
+    okc, gkc, okr, gkr = _kv_pair(ent, raw, fp8)
+    o_ref, l_ref = oracle.csa_attn(_normed_q(q, gamma, eps), okc, idx, okr, W, pos)
+    out = torch.empty(B, Tq, H, d, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, Tq, H, device="cuda")
+    hcl.hcl_csa_sparse_attn(cuda(q), gkc, Nc, cuda(torch.from_numpy(idx)), gkr, L, W, cuda(pos), out,
+                            lse=lse, q_gamma=cuda(gamma), q_eps=eps)
+    torch.cuda.synchronize()
+    tol = 5e-2 if fp8 else 2e-2
+    assert np.abs(as_f64(out) - o_ref).max() <= tol
+    assert np.abs(as_f64(lse) - l_ref).max() <= tol
+
+
+def test_hca_attn_query_rmsnorm(hcl):
+    B, Tq, H, L, W, d, mh, eps = 2, 40, 16, 128 * 30 + 9, 128, 128, 128, 1e-6
+    Nh = -(-L // mh)
+    ent, raw = rbf16(B, Nh, d), rbf16(B, L, d)
+    q = rbf16(B, Tq, H, d, std=0.5)
+    gamma = torch.from_numpy((1.0 + 0.25 * RNG.standard_normal(d)).astype(np.float32))
+    pos = torch.arange(L - Tq, L, dtype=torch.int32).repeat(B, 1).contiguous()
+    okc, gkc, okr, gkr = _kv_pair(ent, raw, False)
+    o_ref, l_ref = oracle.hca_attn(_normed_q(q, gamma, eps), okc, Nh, mh, okr, W, pos)
+    out = torch.empty(B, Tq, H, d, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, Tq, H, device="cuda")
+    hcl.hcl_hca_dense_attn(cuda(q), gkc, Nh, mh, gkr, L, W, cuda(pos), out, lse=lse,
+                           q_gamma=cuda(gamma), q_eps=eps)
+    torch.cuda.synchronize()
+    assert np.abs(as_f64(out) - o_ref).max() <= 2e-2
+    assert np.abs(as_f64(lse) - l_ref).max() <= 2e-2
+
+
 @pytest.mark.parametrize("B,Tq,H,L,W,fp8", [(2, 64, 16, 128 * 40, 128, False),
                                             (2, 1, 16, 128 * 40 + 77, 128, False),
                                             (1, 37, 64, 128 * 20 + 3, 128, False),
@@ -397,18 +470,19 @@ def test_invalid_arguments_rejected(hcl):
 # =========================================================================================
 # fused decode step: MXFP4 keys + bf16 scores select from the indexer's per-16-entry summaries
 
-@pytest.mark.parametrize("B,Nc,k,nvis,ties,plant", [
-    (3, 70000, 1024, (70000, 5000, 700), False, None),   # the last row has fewer than k visible
-    (2, 40000, 512, (40000, 39999), True, None),          # many equal scores, visibility mid-group
-    (1, 4096, 1024, (1030,), True, None),                 # just above k visible
-    (2, 262144, 1024, (262144, 131075), False, None),     # full decode length
+@pytest.mark.parametrize("B,Nc,k,nvis,ties,plant,qnorm", [
+    (3, 70000, 1024, (70000, 5000, 700), False, None, False),  # the last row: fewer than k visible
+    (2, 40000, 512, (40000, 39999), True, None, False),   # many equal scores, visibility mid-group
+    (1, 4096, 1024, (1030,), True, None, False),          # just above k visible
+    (2, 262144, 1024, (262144, 131075), False, None, False),   # full decode length
+    (2, 262144, 1024, (262144, 262143), False, None, True),    # with RMS-normalised queries
     # keys doubled in the groups the top-k samples (every 16th group) of the first P*16
     # groups: the sampled lower bound overshoots, so the exact k-th largest maximum is taken;
     # P = 200 keeps the multi-candidate groups within the shared-memory pool, P = 1024 does not
-    (1, 262144, 1024, (262144,), False, (200, 2.0)),
-    (1, 262144, 1024, (262144,), False, (1024, 2.0)),
+    (1, 262144, 1024, (262144,), False, (200, 2.0), False),
+    (1, 262144, 1024, (262144,), False, (1024, 2.0), False),
 ])
-def test_decode_step_group_maxima(hcl, B, Nc, k, nvis, ties, plant):
+def test_decode_step_group_maxima(hcl, B, Nc, k, nvis, ties, plant, qnorm):
     """The fused step's top-k (group summaries lower bound): the GPU's bf16 scores against the
     oracle's scores of the same MXFP4 operands (quantised by the oracle); the selection against
     the oracle's top-k with the ambiguity band and, exactly, against the oracle's top-k of the
@@ -445,8 +519,11 @@ def test_decode_step_group_maxima(hcl, B, Nc, k, nvis, ties, plant):
     q, qI = rbf16(B, 1, H, d), rbf16(B, 1, HI, 64)
     w = torch.from_numpy(RNG.random((B, 1, HI)).astype(np.float32))
     pos = torch.tensor([[4 * v - 1] for v in nvis], dtype=torch.int32)
+    gamma = (torch.from_numpy((1.0 + 0.25 * RNG.standard_normal(d)).astype(np.float32))
+             if qnorm else None)
     pipe = CsaDecode(cuda(q), cuda(qI), cuda(w), kp, KV(cn, cs, cr), Nc, KV(rn, rs, rr), L, W,
-                     cuda(pos), m=4, k=k, op_fmt=HCL_MXFP4, score_fmt=HCL_BF16, kI_sf=ks)
+                     cuda(pos), m=4, k=k, op_fmt=HCL_MXFP4, score_fmt=HCL_BF16, kI_sf=ks,
+                     q_gamma=None if gamma is None else cuda(gamma))
     pipe.step_parts()
     torch.cuda.synchronize()
     kpo, kso = oracle.quant_mxfp4(kb)
@@ -462,7 +539,8 @@ def test_decode_step_group_maxima(hcl, B, Nc, k, nvis, ties, plant):
     assert np.array_equal(gidx, want)
     okc = oracle.KV(oracle.FMT_FP8SPLIT, *_split3(oracle.quant_kv_fp8(ent), Nc))
     okr = oracle.KV(oracle.FMT_FP8SPLIT, *_split3(oracle.quant_kv_fp8(raw), W))
-    o_ref, l_ref = oracle.csa_attn(q, okc, gidx, okr, W, pos)
+    o_ref, l_ref = oracle.csa_attn(q if gamma is None else _normed_q(q, gamma, 1e-6), okc, gidx,
+                                   okr, W, pos)
     assert np.abs(as_f64(pipe.out) - o_ref).max() <= 5e-2
     assert np.abs(as_f64(pipe.lse) - l_ref).max() <= 5e-2
     out1, idx1 = pipe.out.clone(), pipe.idx.clone()

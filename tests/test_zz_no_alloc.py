@@ -70,7 +70,7 @@ def _call_both(hcl, _lib, L_, B, H, Nc, k, W, fp8, seed):
     lse_ref = torch.empty(B, 1, H, dtype=torch.float32, device="cuda")
     _lib.check(L_.hcl_csa_sparse_attn(q.data_ptr(), B, 1, H, 128, ctypes.byref(kvc), Nc,
                                       idx.data_ptr(), k, ctypes.byref(raw), L, W, pos.data_ptr(),
-                                      scale, None, out_ref.data_ptr(), lse_ref.data_ptr(),
+                                      scale, None, None, 0.0, out_ref.data_ptr(), lse_ref.data_ptr(),
                                       ws.data_ptr(), ws.numel(), status.data_ptr(), stream))
     # the allocation-free entry point
     out = torch.empty_like(out_ref)
@@ -105,7 +105,7 @@ def test_noalloc_matches_workspace_entry_point_twice(hcl, fp8):
 def test_noalloc_rejects_problems_beyond_the_fixed_scratch(hcl):
     from heavily_compressed_long_b200 import _lib
     L_ = _lib.lib()
-    B, H, k, W = 4, 128, 4096, 128          # 4 long selections: 264 split partials > 16 MiB
+    B, H, k, W = 8, 128, 4096, 128          # 8 long selections: 264 split partials > 16 MiB
     need = L_.hcl_csa_sparse_attn_workspace_bytes(B, 1, H, k, W)
     assert need > (16 << 20)
     fake = ctypes.c_void_p(1 << 30)
