@@ -298,7 +298,9 @@ def run_hcl(args, rank, world, local_rank):
     stream = torch.cuda.Stream(device)
     torch.cuda.synchronize()
 
-    # eager warm-up (attributes, first-launch costs), then capture one graph per input set
+    # eager warm-up (attributes, first-launch costs), then capture one graph per input set and
+    # one graph of a whole cycle (one step on every set, in order), so that a run of K steps
+    # is K // n_sets cycle replays plus single-step replays: few host launches per step
     with torch.cuda.stream(stream):
         for p in sets:
             p.step(stream=stream)
@@ -309,7 +311,18 @@ def run_hcl(args, rank, world, local_rank):
         with torch.cuda.graph(gr, stream=stream):
             p.step(stream=stream)
         graphs.append(gr)
+    cycle = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(cycle, stream=stream):
+        for p in sets:
+            p.step(stream=stream)
     torch.cuda.synchronize()
+
+    def run_steps(n):
+        """n decode steps, rotating over the input sets from set 0."""
+        for _ in range(n // n_sets):
+            cycle.replay()
+        for i in range(n % n_sets):
+            graphs[i].replay()
 
     def barrier():
         if world > 1:
@@ -320,8 +333,7 @@ def run_hcl(args, rank, world, local_rank):
 
     K, Wm = args.steps, args.warmup
     with torch.cuda.stream(stream):
-        for i in range(Wm):
-            graphs[i % n_sets].replay()
+        run_steps(Wm)
     torch.cuda.synchronize()
 
     sampler = ClockSampler(local_rank) if rank == 0 else None
@@ -333,8 +345,7 @@ def run_hcl(args, rank, world, local_rank):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     with torch.cuda.stream(stream):
-        for i in range(K):
-            graphs[i % n_sets].replay()
+        run_steps(K)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -407,6 +418,12 @@ def run_hcl(args, rank, world, local_rank):
     barrier()
     e2e_ms = maxv(x0.elapsed_time(x1) / n_e2e)
     clocks = sampler.stop() if sampler else None
+    extra = {}
+    if rank == 0 and world == 1 and not args.no_extra:
+        extra["cache_append"] = measure_cache_append(sets[0], device, stream)
+        del sets[1:]                      # room for the prefill workload
+        torch.cuda.empty_cache()
+        extra["prefill"] = measure_prefill(device, stream)
     status = int(sum(int(p.status.item()) for p in sets))
 
     # CPU baseline: the oracle on the host cores, a bounded sample (rank 0, N = 1 only)
@@ -453,12 +470,115 @@ def run_hcl(args, rank, world, local_rank):
             "device_status": status,
             "clocks": clocks,
         }
+        line.update(extra)
         if cpu:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)
     for gr in graphs:
         del gr
     graphs.clear()
+    del cycle
+
+
+def _time_ms(fn, stream, reps, warm=2):
+    """Average device time of fn() (enqueued on `stream`) over reps calls, CUDA events."""
+    import torch
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def measure_cache_append(p, device, stream, steps=128):
+    """Per-step cost of the decode-time cache append of a CSA layer for the decode workload's
+    sequences (raw window and entries as split FP8 rows, MXFP4 index keys; one CSA entry every
+    4 tokens), B tokens per step: one launch, graph-replayed over `steps` consecutive positions."""
+    import torch
+    from heavily_compressed_long_b200 import api
+    B, d = p.B, p.q.shape[-1]
+    g = torch.Generator(device=device)
+    g.manual_seed(11)
+    stage_kv = torch.randn(B, 128, d, generator=g, device=device).to(torch.bfloat16)
+    stage_g = torch.randn(B, 128, d, generator=g, device=device).to(torch.bfloat16)
+    kv_new = torch.randn(steps, B, d, generator=g, device=device).to(torch.bfloat16)
+    g_new = torch.randn(steps, B, d, generator=g, device=device).to(torch.bfloat16)
+    kI_new = torch.randn(steps, B, 64, generator=g, device=device).to(torch.bfloat16)
+    bias = 0.1 * torch.randn(8, generator=g, device=device)
+    t0 = p.L
+    ts = [torch.full((B,), t0 + s, dtype=torch.int32, device=device) for s in range(steps)]
+
+    def run_all():
+        for s in range(steps):
+            api.hcl_cache_append(kv_new[s], g_new[s], ts[s], stage_kv, stage_g, p.raw, kvc=p.kvc,
+                                 bias_csa=bias, m=p.m, kI_new=kI_new[s], kI=p.kI, kI_sf=p.kI_sf,
+                                 stream=stream)
+
+    with torch.cuda.stream(stream):
+        run_all()
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr, stream=stream):
+        run_all()
+    ms = _time_ms(gr.replay, stream, 3, warm=1) / steps
+    del gr
+    return {"us_per_step": ms * 1e3, "sequences": B, "launches_per_step": 1,
+            "what": "hcl_cache_append: raw window row + staging rings every step, CSA entry "
+                    "(split FP8) + MXFP4 index key every 4th step"}
+
+
+def measure_prefill(device, stream):
+    """The chunked-prefill workload (4096 new tokens on a 262144-token context, 64 heads, CSA
+    top-1024 + HCA, 128-token window): the prefill indexer alone (TFLOP/s vs the measured bf16
+    dense peak), the HCA prefill attention alone, and the whole CSA/HCA layer pair (ms)."""
+    import torch
+    from heavily_compressed_long_b200 import api
+    from heavily_compressed_long_b200.api import HCL_BF16, KV
+    from heavily_compressed_long_b200.pipeline import HcaLayer, PairPrefill
+    from synth.configs import PAIR_PREFILL as cfg
+    g = torch.Generator(device=device)
+    g.manual_seed(cfg.seed)
+    L, d, Tq, H, HI, dI, Nc, Nh = cfg.L, cfg.d, cfg.Tq, cfg.H, cfg.HI, cfg.dI, cfg.Nc, cfg.Nh
+    bf = lambda *sh: torch.randn(*sh, generator=g, device=device).to(torch.bfloat16)
+    kv, gate = bf(1, L, d), bf(1, L, d)
+    q_csa, q_hca = bf(1, Tq, H, d), bf(1, Tq, H, d)
+    qI, kI = bf(1, Tq, HI, dI), bf(1, Nc, dI)
+    w = torch.rand(1, Tq, HI, generator=g, device=device)
+    b_csa = 0.1 * torch.randn(2 * cfg.m, generator=g, device=device)
+    b_hca = 0.1 * torch.randn(cfg.mh, generator=g, device=device)
+    pos = torch.arange(cfg.first_pos, cfg.first_pos + Tq, dtype=torch.int32, device=device).unsqueeze(0).contiguous()
+    comp_c = torch.zeros(1, Nc, d, dtype=torch.bfloat16, device=device)
+    comp_h = torch.zeros(1, Nh, d, dtype=torch.bfloat16, device=device)
+    pp = PairPrefill(kv, gate, b_csa, b_hca, comp_c, comp_h, q_csa, q_hca, qI, w, kI, pos,
+                     cfg.first_pos, m=cfg.m, mh=cfg.mh, k=cfg.k, W=cfg.W, score_fmt=HCL_BF16)
+    with torch.cuda.stream(stream):
+        pp.compress_prior(stream=stream)
+    torch.cuda.synchronize()
+    pair_ms = _time_ms(lambda: pp.step(stream=stream), stream, 5)
+    idx_ms = _time_ms(lambda: api.hcl_csa_index_scores(HCL_BF16, qI, w, kI, pos, cfg.m, pp.scores,
+                                                       stream=stream), stream, 10)
+    hca = HcaLayer(q_hca, KV(comp_h), Nh, cfg.mh, KV(kv), L, cfg.W, pos)
+    hca_ms = _time_ms(lambda: hca.step(stream=stream), stream, 10)
+    peak = bf16_peak()
+    idx_flops = 2.0 * Tq * HI * dI * Nc
+    rows = sum(min(Nh, (p_ + 1) // cfg.mh) + min(cfg.W, p_ + 1) for p_ in range(cfg.first_pos, cfg.first_pos + Tq))
+    hca_flops = 4.0 * H * d * rows
+    return {"workload": cfg.name,
+            "layer_pair_ms": pair_ms,
+            "indexer": {"ms": idx_ms, "tflops": idx_flops / idx_ms / 1e9,
+                        "frac_of_bf16_peak": idx_flops / idx_ms / 1e9 / peak,
+                        "flops": idx_flops, "note": "dense 4096 x 66560 x 16 heads x 64, incl. masked tiles"},
+            "hca_attention": {"ms": hca_ms, "tflops": hca_flops / hca_ms / 1e9,
+                              "frac_of_bf16_peak": hca_flops / hca_ms / 1e9 / peak, "flops": hca_flops,
+                              "note": "4 flops per (query, head, visible row, dim)"},
+            "peak_tflops": peak, "peak_source": "MEASURED_PEAKS.json bf16_tflops (burst)"}
 
 
 def run_prefill_indexer(args, local_rank):
@@ -664,6 +784,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--cpu-frac", type=float, default=1.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the cache-append and prefill measurements added to the line")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

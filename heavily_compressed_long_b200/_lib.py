@@ -45,10 +45,14 @@ SIGNATURES = {
     "hcl_hca_dense_attn": (I, [P, I, I, I, I, KVP, I, I, KVP, I, I, P, F, P, P, F, P, P, P, SZ, P,
                                P]),
     "hcl_csa_decode_step_workspace_bytes": (SZ, [I, I, I, I, I, I, I, I]),
+    "hcl_csa_decode_step_kernels": (I, [I, I, I, I, I, I, I, I, I]),
     "hcl_csa_decode_step": (I, [P, P, P, I, P, P, I, I, I, I, I, I, I, KVP, I, I, I, KVP, I, I,
                                 P, F, P, P, F, P, P, P, P, SZ, P, P]),
     "hcl_cache_append": (I, [P, P, P, P, I, I, I, P, P, I, KVP, KVP, P, I, I, P, P, I, KVP, P, I,
                              P, F, P, P]),
+    "hcl_cp_candidates": (I, [P, I, P, I, I, I, I, P, P, P, P]),
+    "hcl_cp_own": (I, [P, P, I, I, I, I, I, P, P, P]),
+    "hcl_lse_merge": (I, [P, P, I, I64, I, I, P, P, P, P]),
     "hcl_selftest_bounded_wait": (I, [P, I, P]),
 }
 

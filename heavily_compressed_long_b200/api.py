@@ -189,5 +189,32 @@ def hcl_cache_append(kv_new, gate_new, t_new, stage_kv, stage_gate, raw: KV, kvc
                                  _ptr(gamma), eps, None, _stream(stream)))
 
 
+def hcl_cp_candidates(scores, idx, e0, cand_scores, cand_idx, status=None, stream=None):
+    """Local top-k (idx [B, 1, k]) over a rank's scores [B, 1, Nc_local] -> (fp32 score, global
+    index) candidates [B, k]."""
+    B, _, Nc_local = scores.shape
+    k = idx.shape[-1]
+    check(lib().hcl_cp_candidates(_ptr(scores), _fmt_of(scores), _ptr(idx), B, Nc_local, k, e0,
+                                  _ptr(cand_scores), _ptr(cand_idx), _ptr(status), _stream(stream)))
+
+
+def hcl_cp_own(pos, gathered_idx, e0, e1, sel_out, own_out, stream=None):
+    """pos [B, 1, k] selected positions in the gathered list gathered_idx [B, n] -> global
+    selection sel_out [B, 1, k] and this rank's local share own_out [B, 1, k]."""
+    B, n = gathered_idx.shape
+    k = pos.shape[-1]
+    check(lib().hcl_cp_own(_ptr(pos), _ptr(gathered_idx), B, n, k, e0, e1, _ptr(sel_out),
+                           _ptr(own_out), _stream(stream)))
+
+
+def hcl_lse_merge(o_parts, lse_parts, out, lse_out=None, sink=None, stream=None):
+    """o_parts bf16 [G, B, Tq, H, d], lse_parts fp32 [G, B, Tq, H] -> out [B, Tq, H, d]."""
+    G = o_parts.shape[0]
+    H, d = o_parts.shape[-2], o_parts.shape[-1]
+    rows = lse_parts[0].numel()
+    check(lib().hcl_lse_merge(_ptr(o_parts), _ptr(lse_parts), G, rows, d, H, _ptr(sink), _ptr(out),
+                              _ptr(lse_out), _stream(stream)))
+
+
 def hcl_selftest_bounded_wait(status, limit_us=1000, stream=None):
     check(lib().hcl_selftest_bounded_wait(_ptr(status), limit_us, _stream(stream)))

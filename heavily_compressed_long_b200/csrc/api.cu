@@ -424,6 +424,16 @@ size_t hcl_csa_decode_step_workspace_bytes(int B, int H, int HI, int Nc, int k, 
   return decode_ws_layout(B, H, HI, Nc, k, W, op_fmt, score_fmt, 64).total;
 }
 
+int hcl_csa_decode_step_kernels(int B, int H, int HI, int Nc, int k, int W, int op_fmt,
+                                int score_fmt, int kv_fmt) {
+  (void)HI;
+  if (B <= 0) return 0;
+  if (decode_uses_gmax(op_fmt, score_fmt, Nc) && hcl::select_attn_supported(Nc, H, k, W, kv_fmt))
+    return 2;  // indexer, then selection + attention
+  const size_t ws = hcl::attn_workspace_bytes(0, B, 1, H, k, W);
+  return 3 + (ws > 0 ? 1 : 0);  // indexer, top-k, attention (+ split merge)
+}
+
 hcl_status_t hcl_csa_decode_step(const void* q, const void* qI_bf16, const float* w, int op_fmt,
                                  const void* kI, const void* kI_sf, int kI_cap, int score_fmt,
                                  int B, int H, int HI, int dI, int d, const hcl_kv_t* kvc,
@@ -453,6 +463,20 @@ hcl_status_t hcl_csa_decode_step(const void* q, const void* qI_bf16, const float
                           kI_cap, q_pos, m, scores, score_fmt, status, stream);
   if (e != HCL_OK) return e;
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(wsb + l.idx);
+  if (gmax != nullptr && kvc != nullptr && raw != nullptr && kvc->fmt == raw->fmt &&
+      hcl::select_attn_supported(Nc, H, k, W, kvc->fmt) && d == 128) {
+    // selection and attention in one cluster kernel per sequence (it reads q, q_pos and the
+    // raw window before waiting for the indexer, which writes none of them)
+    e = check_kv(kvc, d, "kvc");
+    if (e != HCL_OK) return e;
+    e = check_kv(raw, d, "raw");
+    if (e != HCL_OK) return e;
+    HCL_REQUIRE(q && out && q_pos && aligned16(q) && aligned16(out), "q, out (16-byte aligned) and q_pos are required");
+    if (q_gamma != nullptr) HCL_REQUIRE(q_eps > 0.f && q_eps < 1e30f, "q_eps must be a positive number");
+    SelectAttnArgs sa{scores, gmax, g2nd, garg, B, Nc, q_pos, m, k, idx, q, H, *kvc, *raw, W,
+                      scale, sink, q_gamma, q_eps, out, lse, status};
+    return launch_select_attn(sa, as_stream(stream));
+  }
   // the top-k's predecessor is the indexer above, which does not write q_pos
   if (gmax != nullptr) {
     HCL_REQUIRE(k >= 1 && k <= 4096, "k must be in [1, 4096]");
@@ -513,6 +537,36 @@ hcl_status_t hcl_cache_append(const void* kv_new, const void* gate_new, const vo
   CacheAppendArgs a{kv_new, gate_new, kI_new, t_new, B, stage_kv, stage_gate, stage_cap, *raw,
                     kvc, bias_csa, m, kI_fmt, kI, kI_sf, kI_cap, kvh, bias_hca, mh, gamma, eps};
   return launch_cache_append(a, as_stream(stream));
+}
+
+hcl_status_t hcl_cp_candidates(const void* scores, int score_fmt, const int32_t* idx, int B,
+                               int Nc_local, int k, int e0, float* cand_scores,
+                               int32_t* cand_idx, int32_t* status, void* stream) {
+  HCL_REQUIRE(score_fmt == HCL_FP32 || score_fmt == HCL_BF16, "score_fmt must be HCL_FP32 or HCL_BF16");
+  HCL_REQUIRE(B >= 0 && Nc_local >= 0 && k >= 1 && e0 >= 0, "invalid size");
+  if (B == 0) return HCL_OK;
+  HCL_REQUIRE(idx && cand_scores && cand_idx && (scores || Nc_local == 0), "NULL pointer");
+  return launch_cp_candidates(scores, score_fmt, idx, B, Nc_local, k, e0, cand_scores, cand_idx,
+                              status, as_stream(stream));
+}
+
+hcl_status_t hcl_cp_own(const int32_t* pos, const int32_t* gathered_idx, int B, int n, int k,
+                        int e0, int e1, int32_t* sel_out, int32_t* own_out, void* stream) {
+  HCL_REQUIRE(B >= 0 && n >= 0 && k >= 1 && 0 <= e0 && e0 <= e1, "invalid size");
+  if (B == 0) return HCL_OK;
+  HCL_REQUIRE(pos && gathered_idx && sel_out && own_out, "NULL pointer");
+  return launch_cp_own(pos, gathered_idx, B, n, k, e0, e1, sel_out, own_out, as_stream(stream));
+}
+
+hcl_status_t hcl_lse_merge(const void* o_parts, const float* lse_parts, int G, int64_t rows, int d,
+                           int H, const float* sink, void* out, float* lse_out, void* stream) {
+  HCL_REQUIRE(G >= 1 && rows >= 0 && H >= 1, "invalid size");
+  HCL_REQUIRE(d >= 2 && d % 2 == 0 && d <= 1024, "d must be even, <= 1024");
+  if (rows == 0) return HCL_OK;
+  HCL_REQUIRE(o_parts && lse_parts && out, "NULL pointer");
+  HCL_REQUIRE(((uintptr_t)o_parts & 3) == 0 && ((uintptr_t)out & 3) == 0, "o_parts and out must be 4-byte aligned");
+  return launch_lse_merge(o_parts, lse_parts, G, (long long)rows, d, H, sink, out, lse_out,
+                          as_stream(stream));
 }
 
 hcl_status_t hcl_selftest_bounded_wait(int32_t* status, int limit_us, void* stream) {

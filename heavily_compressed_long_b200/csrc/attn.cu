@@ -1187,6 +1187,7 @@ hcl_status_t launch_attn(const AttnArgs& a, void* ws, size_t ws_bytes, cudaStrea
     p.ws_o = static_cast<float*>(ws);
     p.ws_lse = p.ws_o + items * pl.rows_pad * D;
   }
+  if (hca_flash_usable(a)) return launch_hca_flash(a, st);
   if (tc_usable(a, pl)) {
     return a.comp.fmt == HCL_FP8SPLIT ? launch_tc<HCL_FP8SPLIT>(p, st) : launch_tc<HCL_BF16>(p, st);
   }

@@ -1,0 +1,418 @@
+// attn_flash.cu -- HCA dense attention for prefill chunks on tcgen05 tensor cores.
+//
+// [Tripbot §3.2; CSDN §1.2] HCA attends densely over every compressed entry visible to the
+// query (entry i of ratio m' is visible at position p when m'(i+1) - 1 <= p) and [Tripbot §3.3]
+// over the raw tokens of its sliding window, under one softmax (scale, optional sink); each
+// row is both key and value of the one shared KV head.
+//
+// Design (B200): one block of 256 threads per query group: G = floor(128 / H) consecutive
+// queries x H heads = up to 128 (query, head) rows = the UMMA M dimension = 128 TMEM lanes, two
+// threads per row.  The group's KV list is the visible-entry prefix of its last query followed
+// by the union of its queries' windows; it is processed in rounds of two 64-row chunks gathered
+// with cp.async (split FP8 rows widened to bf16 with their scale).  Per round S = Q K^T (N = 64
+// per chunk) and O = P V (V read as the MN-major operand of the same SW128 tile) accumulate in
+// TMEM; the softmax runs in registers with each row's own causal mask (for query q: the list
+// rows [0, visible entries of q) and the window rows of q -- two index intervals, turned into
+// bit masks), online across rounds: O of a round is added to the register accumulator after
+// rescaling by the change of the running maximum.  Two blocks fit per SM (about 106 KB of
+// shared memory, 256 TMEM columns each), so one block's gather overlaps the other's MMAs.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "hcl_common.cuh"
+#include "hcl_internal.h"
+
+namespace hcl {
+namespace {
+
+constexpr int FA_THREADS = 256;
+constexpr int FA_ROWS = 128;
+constexpr int FA_D = 128;
+constexpr int FA_CH = 64;
+constexpr int FA_RCH = 2;
+constexpr float FA_LOG2E = 1.4426950408889634f;
+constexpr float FA_LN2 = 0.6931471805599453f;
+
+struct FaParams {
+  const __nv_bfloat16* q;   // [B, Tq, H, 128]
+  int B, Tq, H, G, n_groups;
+  hcl_kv_t comp, raw;
+  int Nh, mh, W;
+  const int32_t* q_pos;
+  float scale_log2;
+  const float* sink;
+  const float* q_gamma;
+  float q_eps;
+  __nv_bfloat16* out;
+  float* lse;
+  int32_t* status;
+  long long limit;
+};
+
+struct FaOff {
+  static constexpr uint32_t Q = 0;
+  static constexpr uint32_t KV = 32768;
+  static constexpr uint32_t P = KV + FA_RCH * 16384;
+  static constexpr uint32_t STG = P + FA_RCH * 16384;
+  static constexpr uint32_t SCL = STG + FA_RCH * 4096;
+  static constexpr uint32_t XCH = SCL + FA_RCH * 256;
+  static constexpr uint32_t BAR = XCH + 2 * FA_THREADS * 4;
+  static constexpr uint32_t TOTAL = BAR + 32;
+};
+
+__device__ __forceinline__ uint32_t fa_pack(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint32_t fa_e4m3x2(uint16_t codes, float scale) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(codes));
+  const float2 f = __half22float2(*reinterpret_cast<__half2*>(&h2));
+  return fa_pack(f.x * scale, f.y * scale);
+}
+
+// Bits j (0..31) of the columns c0 + j inside [lo, hi).
+__device__ __forceinline__ uint32_t range_bits(int c0, int lo, int hi) {
+  const int a = max(lo - c0, 0), e = min(hi - c0, 32);
+  if (a >= e) return 0u;
+  const uint32_t upto = e >= 32 ? 0xFFFFFFFFu : ((1u << e) - 1u);
+  const uint32_t from = a <= 0 ? 0xFFFFFFFFu : ~((1u << a) - 1u);
+  return upto & from;
+}
+
+template <int KVFMT>
+__global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
+  extern __shared__ __align__(1024) uint8_t fa_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fa_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int row = tid & (FA_ROWS - 1), hc = tid / FA_ROWS;
+  const int grp = blockIdx.x % p.n_groups, b = blockIdx.x / p.n_groups;
+  const int t0 = grp * p.G;
+  const int gq = min(p.G, p.Tq - t0);
+  float* xch = reinterpret_cast<float*>(sm + FaOff::XCH);
+  uint64_t* bar_s = reinterpret_cast<uint64_t*>(sm + FaOff::BAR);
+  uint64_t* bar_o = bar_s + 1;
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + FaOff::BAR + 16);
+  if (tid == 0) {
+    mbar_init(bar_s, 1);
+    mbar_init(bar_o, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(sTmem, 256);
+    tmem_relinquish();
+  }
+  pdl_enter();
+  // this thread's (query, head) row and its visibility intervals
+  const int qi = row / p.H, hh = row % p.H;
+  const bool rv = qi < gq;
+  const int my_p = rv ? p.q_pos[(size_t)b * p.Tq + t0 + qi] : -1;
+  int pmin = 0x7fffffff, pmax = -1;
+  for (int i = 0; i < gq; i++) {
+    const int pp = p.q_pos[(size_t)b * p.Tq + t0 + i];
+    pmin = min(pmin, pp);
+    pmax = max(pmax, pp);
+  }
+  const int n_a = pmax < 0 ? 0 : min(p.Nh, (pmax + 1) / p.mh);
+  const int raw_lo = pmin - p.W + 1;
+  const int n_raw = (p.W > 0 && pmax >= 0) ? max(0, pmax - raw_lo + 1) : 0;
+  const int total = n_a + n_raw;
+  // list rows visible to this row: entries [0, nv_e) and window rows [w_lo, w_hi)
+  const int nv_e = my_p < 0 ? 0 : min(n_a, (my_p + 1) / p.mh);
+  int w_lo = 0, w_hi = 0;
+  if (rv && my_p >= 0 && p.W > 0) {
+    const int u_lo = max(0, my_p - p.W + 1);
+    w_lo = n_a + (u_lo - raw_lo);
+    w_hi = n_a + (my_p - raw_lo) + 1;
+  }
+
+  // Q rows (query qi, head hh) -> SW128 halves, optionally RMS-normalised
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(
+                           p.q + (((size_t)b * p.Tq + t0 + (rv ? qi : 0)) * p.H + hh) * FA_D) + hc * 8;
+    uint4 qv[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) qv[i] = rv ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+    if (p.q_gamma != nullptr) {
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        const uint32_t w4[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+          const float lo = __uint_as_float(w4[j] << 16), hi = __uint_as_float(w4[j] & 0xFFFF0000u);
+          ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+        }
+      }
+      xch[tid] = ss;
+      __syncthreads();
+      const float rn = 1.f / sqrtf((xch[row] + xch[row + FA_ROWS]) / float(FA_D) + p.q_eps);
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        uint32_t w4[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+          const int dim = hc * 64 + i * 8 + 2 * j;
+          const float lo = __uint_as_float(w4[j] << 16), hi = __uint_as_float(w4[j] & 0xFFFF0000u);
+          w4[j] = fa_pack(lo * rn * __ldg(p.q_gamma + dim), hi * rn * __ldg(p.q_gamma + dim + 1));
+        }
+        qv[i] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
+      __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 8; i++)
+      *reinterpret_cast<uint4*>(sm + FaOff::Q + hc * 16384 + row * 128 + ((i ^ (row & 7)) << 4)) = qv[i];
+  }
+
+  tc_fence_after();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *sTmem;
+  const uint32_t ocol = FA_RCH * FA_CH;
+  const uint32_t trow = tbase + (uint32_t((warp & 3) * 32) << 16);
+  float o_acc[64];
+#pragma unroll
+  for (int i = 0; i < 64; i++) o_acc[i] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+  bool ok = true;
+  const int nrounds = (total + FA_RCH * FA_CH - 1) / (FA_RCH * FA_CH);
+  for (int rd = 0; rd < nrounds; rd++) {
+    const int r0 = rd * FA_RCH * FA_CH;
+    const int nr = min(FA_RCH * FA_CH, total - r0);
+    const int nch = (nr + FA_CH - 1) / FA_CH;
+    // gather: list row r0 + jj -> KV row jj (rows past nr: zeros)
+    constexpr int PIECES = KVFMT == HCL_BF16 ? 16 : 13;
+    for (int u = tid; u < nch * FA_CH * PIECES; u += FA_THREADS) {
+      const int jj = u / PIECES, pc = u % PIECES;
+      const int ch = jj / FA_CH, r = jj % FA_CH;
+      const int e = r0 + jj;
+      long long slot = -1;
+      const hcl_kv_t* st = &p.comp;
+      if (jj < nr) {
+        if (e < n_a) {
+          slot = (long long)b * p.comp.cap + (e % p.comp.cap);
+        } else {
+          const long long tok = (long long)raw_lo + (e - n_a);
+          if (tok >= 0) { st = &p.raw; slot = (long long)b * p.raw.cap + tok % p.raw.cap; }
+        }
+      }
+      uint8_t* kv = sm + FaOff::KV + ch * 16384;
+      if (KVFMT == HCL_BF16) {
+        uint8_t* dst = kv + (pc >> 3) * 8192 + r * 128 + (((pc & 7) ^ (r & 7)) << 4);
+        if (slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st->data) + slot * 256 + pc * 16);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+      } else if (pc < 8) {
+        uint8_t* dst = kv + 8192 + r * 128 + ((pc ^ (r & 7)) << 4);
+        if (slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st->rope) + slot * 128 + pc * 16);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+      } else if (pc < 12) {
+        uint8_t* dst = sm + FaOff::STG + (ch * FA_CH + r) * 64 + (pc - 8) * 16;
+        if (slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st->data) + slot * 64 + (pc - 8) * 16);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+      } else {
+        float* dst = reinterpret_cast<float*>(sm + FaOff::SCL) + ch * FA_CH + r;
+        if (slot >= 0)
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)),
+                       "l"(st->scale + slot)
+                       : "memory");
+        else *dst = 0.f;
+      }
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    if (KVFMT == HCL_FP8SPLIT) {
+      for (int u = tid; u < nch * FA_CH * 8; u += FA_THREADS) {
+        const int jj = u >> 3, cc = u & 7, ch = jj / FA_CH, r = jj % FA_CH;
+        const uint2 codes = *reinterpret_cast<const uint2*>(sm + FaOff::STG + (ch * FA_CH + r) * 64 + cc * 8);
+        const float sc = reinterpret_cast<const float*>(sm + FaOff::SCL)[ch * FA_CH + r];
+        uint4 v;
+        v.x = fa_e4m3x2(uint16_t(codes.x & 0xffff), sc);
+        v.y = fa_e4m3x2(uint16_t(codes.x >> 16), sc);
+        v.z = fa_e4m3x2(uint16_t(codes.y & 0xffff), sc);
+        v.w = fa_e4m3x2(uint16_t(codes.y >> 16), sc);
+        *reinterpret_cast<uint4*>(sm + FaOff::KV + ch * 16384 + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
+      }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+      const uint32_t aq = smem_u32(sm + FaOff::Q);
+      for (int ch = 0; ch < nch; ch++) {
+        const uint32_t ak = smem_u32(sm + FaOff::KV + ch * 16384);
+#pragma unroll
+        for (int ks = 0; ks < 8; ks++) {
+          const uint32_t h = ks >> 2, kk = ks & 3;
+          umma_bf16(tbase + ch * FA_CH, make_sdesc(aq + h * 16384 + kk * 32, 16, 1024, SMEM_SWIZZLE_128B),
+                    make_sdesc(ak + h * 8192 + kk * 32, 16, 1024, SMEM_SWIZZLE_128B),
+                    idesc_bf16(128, FA_CH), ks > 0 ? 1u : 0u);
+        }
+      }
+      umma_commit(bar_s);
+    }
+    ok = ok && mbar_wait(bar_s, rd & 1, p.limit, nullptr);
+    tc_fence_after();
+    // two passes over this thread's 32 columns of each chunk: maximum, then exponentials
+    // (the columns are read from TMEM twice instead of being held in registers)
+    uint32_t vb[FA_RCH];
+    float lmax = -INFINITY;
+#pragma unroll
+    for (int ch = 0; ch < FA_RCH; ch++) {
+      vb[ch] = 0u;
+      if (ch < nch && rv) {
+        const int c0 = r0 + ch * FA_CH + hc * 32;
+        vb[ch] = (range_bits(c0, 0, nv_e) | range_bits(c0, w_lo, w_hi)) &
+                 range_bits(c0, r0, r0 + nr);
+      }
+      if (ch < nch) {
+        uint32_t sv[32];
+        tmem_ld16(trow + ch * FA_CH + hc * 32, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
+        tmem_ld16(trow + ch * FA_CH + hc * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; j++)
+          if ((vb[ch] >> j) & 1u) lmax = fmaxf(lmax, __uint_as_float(sv[j]) * p.scale_log2);
+      }
+    }
+    xch[tid] = lmax;
+    __syncthreads();
+    const float m_new = fmaxf(m_run, fmaxf(xch[row], xch[row + FA_ROWS]));
+    const float muse = m_new == -INFINITY ? 0.f : m_new;
+    float lsum = 0.f;
+#pragma unroll
+    for (int ch = 0; ch < FA_RCH; ch++)
+      if (ch < nch) {
+        uint32_t sv[32];
+        tmem_ld16(trow + ch * FA_CH + hc * 32, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
+        tmem_ld16(trow + ch * FA_CH + hc * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+        tmem_ld_wait();
+        uint8_t* prow = sm + FaOff::P + ch * 16384 + row * 128;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; q4++) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int i = 0; i < 8; i += 2) {
+            const int j = q4 * 8 + i;
+            const float p0 = ((vb[ch] >> j) & 1u) ? exp2f(__uint_as_float(sv[j]) * p.scale_log2 - muse) : 0.f;
+            const float p1 = ((vb[ch] >> (j + 1)) & 1u) ? exp2f(__uint_as_float(sv[j + 1]) * p.scale_log2 - muse) : 0.f;
+            lsum += p0 + p1;
+            pk[i >> 1] = fa_pack(p0, p1);
+          }
+          *reinterpret_cast<uint4*>(prow + (((hc * 4 + q4) ^ (row & 7)) << 4)) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+      for (int ch = 0; ch < nch; ch++) {
+        const uint32_t ap = smem_u32(sm + FaOff::P + ch * 16384);
+        const uint32_t av = smem_u32(sm + FaOff::KV + ch * 16384);
+#pragma unroll
+        for (int ks = 0; ks < 4; ks++)
+          umma_bf16(tbase + ocol, make_sdesc(ap + ks * 32, 16, 1024, SMEM_SWIZZLE_128B),
+                    make_sdesc(av + ks * 2048, 8192, 1024, SMEM_SWIZZLE_128B),
+                    idesc_bf16(128, FA_D) | (1u << 16), (ch > 0 || ks > 0) ? 1u : 0u);
+      }
+      umma_commit(bar_o);
+    }
+    ok = ok && mbar_wait(bar_o, rd & 1, p.limit, nullptr);
+    tc_fence_after();
+    {
+      const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - m_new);
+#pragma unroll
+      for (int q4 = 0; q4 < 4; q4++) {
+        uint32_t r16[16];
+        tmem_ld16(trow + ocol + hc * 64 + q4 * 16, r16);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; i++)
+          o_acc[q4 * 16 + i] = o_acc[q4 * 16 + i] * alpha + __uint_as_float(r16[i]);
+      }
+      l_run = l_run * alpha + lsum;
+      m_run = m_new;
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+  if (!ok) report(p.status, HCL_ERR_TIMEOUT);
+  xch[FA_THREADS + tid] = l_run;
+  __syncthreads();
+  float l2 = xch[FA_THREADS + row] + xch[FA_THREADS + row + FA_ROWS];
+  float m2 = m_run;
+  float f = l2 > 0.f ? 1.f / l2 : 0.f;
+  if (p.sink) {
+    const float s2 = p.sink[hh] * FA_LOG2E;
+    const float mm = fmaxf(m2, s2);
+    const float fa = l2 > 0.f ? exp2f(m2 - mm) : 0.f;
+    const float l3 = l2 * fa + exp2f(s2 - mm);
+    f = l3 > 0.f ? fa / l3 : 0.f;
+    l2 = l3;
+    m2 = mm;
+  }
+  if (rv) {
+    const size_t orow = ((size_t)b * p.Tq + t0 + qi) * p.H + hh;
+    __nv_bfloat16* dst = p.out + orow * FA_D + hc * 64;
+#pragma unroll
+    for (int i = 0; i < 64; i += 8)
+      *reinterpret_cast<uint4*>(dst + i) =
+          make_uint4(fa_pack(o_acc[i] * f, o_acc[i + 1] * f), fa_pack(o_acc[i + 2] * f, o_acc[i + 3] * f),
+                     fa_pack(o_acc[i + 4] * f, o_acc[i + 5] * f), fa_pack(o_acc[i + 6] * f, o_acc[i + 7] * f));
+    if (hc == 0 && p.lse) p.lse[orow] = l2 > 0.f ? (m2 + log2f(l2)) * FA_LN2 : -INFINITY;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 256);
+  }
+}
+
+template <int KVFMT>
+hcl_status_t launch_flash_t(const FaParams& p, cudaStream_t st) {
+  auto kern = hca_flash_kernel<KVFMT>;
+  const int smem = (int)FaOff::TOTAL + 1024;
+  hcl_status_t e = set_kernel_attrs(reinterpret_cast<const void*>(kern), smem, false);
+  if (e != HCL_OK) return e;
+  return check_cuda(launch_pdl(kern, dim3((unsigned)((long long)p.B * p.n_groups)),
+                               dim3(FA_THREADS), (size_t)smem, st, 1, p),
+                    "hca flash attention launch");
+}
+
+}  // namespace
+
+bool hca_flash_usable(const AttnArgs& a) {
+  if (a.mode != 1 || a.H > FA_ROWS || a.d != FA_D) return false;
+  const int G = std::max(1, FA_ROWS / a.H);
+  const int n_groups = (a.Tq + G - 1) / G;
+  return n_groups >= 32 && (a.comp.fmt == HCL_BF16 || a.comp.fmt == HCL_FP8SPLIT);
+}
+
+hcl_status_t launch_hca_flash(const AttnArgs& a, cudaStream_t st) {
+  FaParams p;
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.B = a.B; p.Tq = a.Tq; p.H = a.H;
+  p.G = std::min(std::max(1, FA_ROWS / a.H), a.Tq);
+  p.n_groups = (a.Tq + p.G - 1) / p.G;
+  p.comp = a.comp; p.raw = a.raw;
+  p.Nh = a.n_comp; p.mh = a.mh; p.W = a.W;
+  p.q_pos = a.q_pos;
+  p.scale_log2 = a.scale * FA_LOG2E;
+  p.sink = a.sink;
+  p.q_gamma = a.q_gamma;
+  p.q_eps = a.q_eps;
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.lse = a.lse;
+  p.status = a.status;
+  p.limit = wait_limit_cycles();
+  return a.comp.fmt == HCL_FP8SPLIT ? launch_flash_t<HCL_FP8SPLIT>(p, st) : launch_flash_t<HCL_BF16>(p, st);
+}
+
+}  // namespace hcl

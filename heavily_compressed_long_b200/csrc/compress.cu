@@ -9,11 +9,8 @@
 //
 // HBM-streaming kernels: each thread owns 8 channels (one 16-byte load of kv and of gate per
 // token row, coalesced along d) and keeps an online (max, sum, weighted sum) softmax in fp32
-// (pool.cuh).  Small spans give each entry to one group of d/8 threads; the CSA span 2m = 8 is
-// a compile-time span, so all 16 row loads of an entry are in flight before the arithmetic
-// (a slot-by-slot loop waits one memory latency per slot).  Long spans (HCA) split the slots
-// over the 128 threads of a block, four slots' loads in flight per thread, and merge the
-// partial softmaxes in shared memory.
+// (pool.cuh).  Small spans give each entry to one group of d/8 threads; long spans (HCA) split
+// the slots over the 128 threads of a block and merge the partial softmaxes in shared memory.
 //
 // Optional RMSNorm epilogue [Tripbot §5: queries and compressed KV entries are RMS-normalised,
 // so attention needs no extra QK normalisation]: with gamma given, every pooled entry c is
@@ -121,14 +118,9 @@ hcl_status_t launch_compress(const void* kv, const void* gate, const float* bias
     const int blk = (256 / G) * G;
     const long long grid = (threads + blk - 1) / blk;
     const int first_off = overlap ? -m : 0;
-    if (span == 8)
-      compress_small_kernel<8><<<(unsigned)grid, blk, 0, st>>>(kvp, gp, bias, B, L, d, m, span,
-                                                                first_off, e0, e1, out, out_fmt,
-                                                                out_cap, gamma, eps);
-    else
-      compress_small_kernel<0><<<(unsigned)grid, blk, 0, st>>>(kvp, gp, bias, B, L, d, m, span,
-                                                                first_off, e0, e1, out, out_fmt,
-                                                                out_cap, gamma, eps);
+    compress_small_kernel<0><<<(unsigned)grid, blk, 0, st>>>(kvp, gp, bias, B, L, d, m, span,
+                                                              first_off, e0, e1, out, out_fmt,
+                                                              out_cap, gamma, eps);
   } else {
     const int streams = 128 / G;
     const size_t smem = ((size_t)streams * 3 * d + 4) * sizeof(float);

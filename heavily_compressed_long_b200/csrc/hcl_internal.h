@@ -125,6 +125,33 @@ bool topk_gmax_supported(int Nc);
 hcl_status_t launch_topk_gmax(const TopkArgs& a, const uint16_t* gmax, const uint16_t* g2nd,
                               const uint8_t* garg, cudaStream_t st);
 
+// Fused decode selection + attention (MXFP4 keys, bf16 scores with the indexer's group
+// summaries): one cluster of CTAs per sequence selects the top-k from the summaries and
+// attends over its share of the selected entries and the window.
+struct SelectAttnArgs {
+  const void* scores;        // bf16 [B, Nc]
+  const uint16_t* gmax;      // [B, gmax_row_stride(Nc)]
+  const uint16_t* g2nd;
+  const uint8_t* garg;
+  int B, Nc;
+  const int32_t* q_pos;
+  int m, k;
+  int32_t* idx;              // [B, k]
+  const void* q;             // bf16 [B, H, 128]
+  int H;
+  hcl_kv_t comp, raw;
+  int W;
+  float scale;
+  const float* sink;
+  const float* q_gamma;
+  float q_eps;
+  void* out;
+  float* lse;
+  int32_t* status;
+};
+bool select_attn_supported(int Nc, int H, int k, int W, int comp_fmt);
+hcl_status_t launch_select_attn(const SelectAttnArgs& a, cudaStream_t st);
+
 // One attention launch: CSA (selected entries + window) or HCA (visible entries + window).
 struct AttnArgs {
   int mode;  // 0 = CSA, 1 = HCA
@@ -149,6 +176,9 @@ struct AttnArgs {
 };
 // n = k (CSA) or Nh (HCA)
 size_t attn_workspace_bytes(int mode, int B, int Tq, int H, int n, int W);
+// HCA prefill (many query groups, no KV split) on tcgen05 (attn_flash.cu).
+bool hca_flash_usable(const AttnArgs& a);
+hcl_status_t launch_hca_flash(const AttnArgs& a, cudaStream_t st);
 hcl_status_t launch_attn(const AttnArgs& a, void* ws, size_t ws_bytes, cudaStream_t st);
 
 // Decode-time cache append (one token per sequence); kvc / kvh null: no CSA / HCA store.
@@ -176,6 +206,15 @@ struct CacheAppendArgs {
   float eps;
 };
 hcl_status_t launch_cache_append(const CacheAppendArgs& a, cudaStream_t st);
+
+// Context-parallel decode data steps (cp.cu).
+hcl_status_t launch_cp_candidates(const void* scores, int score_fmt, const int32_t* idx, int B,
+                                  int Nc_local, int k, int e0, float* cand_s, int32_t* cand_i,
+                                  int32_t* status, cudaStream_t st);
+hcl_status_t launch_cp_own(const int32_t* pos, const int32_t* gidx, int B, int n, int k, int e0,
+                           int e1, int32_t* sel_out, int32_t* own_out, cudaStream_t st);
+hcl_status_t launch_lse_merge(const void* o, const float* lse, int G, long long rows, int d, int H,
+                              const float* sink, void* out, float* lse_out, cudaStream_t st);
 
 // Fixed device scratch of hcl_csa_sparse_attn_noalloc (split-KV partials), and its device
 // address on the current device (looked up once per device).

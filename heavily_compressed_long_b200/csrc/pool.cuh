@@ -122,7 +122,7 @@ __device__ __forceinline__ void rmsnorm8_group(float (&v)[8], int G, int d, int 
 
 // Long spans (HCA): one entry per block of 128 threads.  Thread t works on channel chunk
 // t % G (G = d/8) of slot stream t / G; stream s takes slots s, s + S, s + 2S, ... (S = 128/G
-// streams), four slots' loads in flight at a time; the streams' partial softmaxes are merged
+// streams); the streams' partial softmaxes are merged
 // through shared memory `sm` ([S][3][d] floats, then 4 floats).  On return thread t holds, for
 // channels c = t + 128u (u < MAXV, c < d), the entry in vals[u] -- RMS-normalised with gamma.
 // All 128 threads must call it.
@@ -138,23 +138,13 @@ __device__ __forceinline__ void pool_long_block(RowFn row, const float* __restri
   Online8 s;
   s.init();
   if (stream < streams) {
-    for (int j0 = stream; j0 < span; j0 += 4 * streams) {
-      uint4 xv[4], gv[4];
-      bool ok[4];
-#pragma unroll
-      for (int u = 0; u < 4; u++) {
-        const int j = j0 + u * streams;
-        const __nv_bfloat16* kp;
-        const __nv_bfloat16* gp;
-        ok[u] = j < span && row(j, kp, gp);
-        if (ok[u]) {
-          xv[u] = ld_row16<NC>(kp, chunk);
-          gv[u] = ld_row16<NC>(gp, chunk);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; u++)
-        if (ok[u]) s.add(xv[u], gv[u], __ldg(bias + j0 + u * streams));
+    for (int j = stream; j < span; j += streams) {
+      const __nv_bfloat16* kp;
+      const __nv_bfloat16* gp;
+      if (!row(j, kp, gp)) continue;
+      const uint4 xv = ld_row16<NC>(kp, chunk);
+      const uint4 gv = ld_row16<NC>(gp, chunk);
+      s.add(xv, gv, __ldg(bias + j));
     }
     float* base = sm + (size_t)stream * 3 * d;
 #pragma unroll

@@ -42,10 +42,14 @@ class CsaDecode:
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
 
     def launches_per_step(self, fused=True):
-        """Kernels one step launches: indexer, top-k, attention (+ split merge), and with
-        step_parts() a separate q_I quantisation for MXFP4 keys (fused into the indexer by
-        the C-ABI decode step)."""
-        n = 3 + (1 if (self.op_fmt == HCL_MXFP4 and not fused) else 0)
+        """Kernels one step launches: the fused C-ABI step as the library reports it, or with
+        step_parts() indexer, top-k, attention (+ split merge) and, for MXFP4 keys, a separate
+        q_I quantisation."""
+        if fused:
+            return api.lib().hcl_csa_decode_step_kernels(self.B, self.H, self.HI, self.Nc, self.k,
+                                                         self.W, self.op_fmt, self.score_fmt,
+                                                         self.kvc.fmt)
+        n = 3 + (1 if self.op_fmt == HCL_MXFP4 else 0)
         need = api.csa_sparse_attn_workspace_bytes(self.B, 1, self.H, self.k, self.W)
         return n + (1 if need else 0)
 

@@ -232,7 +232,9 @@ HCL_API hcl_status_t hcl_hca_dense_attn(const void* q, int B, int Tq, int H, int
  * Fused CSA decode step [Tripbot §3.1]: for each sequence, the new query's index queries are
  * quantised (MXFP4 operands only), scored against all entries, the top-k kept, and
  * attention run over them plus the window -- a4 -> a5 -> a6 enqueued back to back on
- * `stream`.  Arguments as in the individual calls; qI_bf16 is the unquantised bf16 index
+ * `stream`; with MXFP4 keys and bf16 scores a5 and a6 run as one kernel (a cluster per
+ * sequence selects from the indexer's group summaries and attends over its share of the
+ * selection), whose selection equals hcl_csa_topk's bit for bit.  Arguments as in the individual calls; qI_bf16 is the unquantised bf16 index
  * query [B, 1, HI, dI]; Tq == 1.  ws: hcl_csa_decode_step_workspace_bytes() bytes; it holds
  * the scores and, with MXFP4 operands and bf16 scores, a 5-byte summary per 16-entry group
  * (largest and second largest score as order-preserving keys, position of the largest) that
@@ -241,6 +243,12 @@ HCL_API hcl_status_t hcl_hca_dense_attn(const void* q, int B, int Tq, int H, int
  */
 HCL_API size_t hcl_csa_decode_step_workspace_bytes(int B, int H, int HI, int Nc, int k, int W,
                                            int op_fmt, int score_fmt);
+/* The number of kernels one hcl_csa_decode_step call with these shapes and formats launches
+ * (kv_fmt: the compressed / raw store format): 2 with MXFP4 keys and bf16 scores (the indexer,
+ * then selection and attention in one cluster kernel per sequence), otherwise 3 or 4 (indexer,
+ * top-k, attention, and a split merge when the attention needs a workspace). */
+HCL_API int hcl_csa_decode_step_kernels(int B, int H, int HI, int Nc, int k, int W, int op_fmt,
+                                        int score_fmt, int kv_fmt);
 HCL_API hcl_status_t hcl_csa_decode_step(const void* q, const void* qI_bf16, const float* w, int op_fmt,
                                  const void* kI, const void* kI_sf, int kI_cap, int score_fmt,
                                  int B, int H, int HI, int dI, int d, const hcl_kv_t* kvc,
@@ -286,6 +294,38 @@ HCL_API hcl_status_t hcl_cache_append(const void* kv_new, const void* gate_new,
                                       void* kI_sf, int kI_cap, const hcl_kv_t* kvh,
                                       const float* bias_hca, int mh, const float* gamma,
                                       float eps, int32_t* status, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Context-parallel CSA decode [Austery's talk notes, infrastructure section: context
+ * parallelism]: one sequence's compressed entries sharded over ranks, rank r holding entries
+ * [e0, e1).  The ranks' collectives (all-gathers) are issued by the caller between these
+ * calls; the data steps are:
+ *   hcl_cp_candidates: a rank's local top-k (idx int32 [B, k], ascending local indices, -1
+ *     padded, as hcl_csa_topk writes them over the rank's scores [B, Nc_local] in score_fmt)
+ *     -> candidates: cand_scores fp32 [B, k] (the bf16 / fp32 score, exactly) and cand_idx
+ *     int32 [B, k] = e0 + local index (padding: -inf and -1).  Gathered in rank order the
+ *     candidates are in ascending global index order, so the k best of the gathered list
+ *     (hcl_csa_topk over the n = ranks * k scores, visible count n: q_pos = n - 1 with m = 1)
+ *     are the global top-k with ties to the lower global index.
+ *   hcl_cp_own: pos int32 [B, k] (the ascending positions hcl_csa_topk selected in the gathered
+ *     list) and gathered_idx int32 [B, n] -> sel_out int32 [B, k], the selected global indices,
+ *     ascending, -1 padded; own_out int32 [B, k], those in [e0, e1) as local indices (minus e0),
+ *     ascending, -1 padded -- the rank's share of the attention, to pass to
+ *     hcl_csa_sparse_attn over its slice (the window on the rank holding the last tokens).
+ *   hcl_lse_merge: the ranks' partial attention outputs o_parts bf16 [G, rows, d] and
+ *     lse_parts fp32 [G, rows] (natural log; rows = B * Tq * H, head h = row % H) ->
+ *     out bf16 [rows, d] = sum_r w_r o_r / sum_r w_r with w_r = exp(lse_r - M), and lse_out
+ *     fp32 [rows] (or NULL) = M + log sum_r w_r, M the largest lse; a sink (fp32 [H] logits or
+ *     NULL) adds exp(sink[h] - M) to the denominator only.  Partials with lse = -inf weigh 0.
+ */
+HCL_API hcl_status_t hcl_cp_candidates(const void* scores, int score_fmt, const int32_t* idx, int B,
+                                       int Nc_local, int k, int e0, float* cand_scores,
+                                       int32_t* cand_idx, int32_t* status, void* stream);
+HCL_API hcl_status_t hcl_cp_own(const int32_t* pos, const int32_t* gathered_idx, int B, int n, int k,
+                                int e0, int e1, int32_t* sel_out, int32_t* own_out, void* stream);
+HCL_API hcl_status_t hcl_lse_merge(const void* o_parts, const float* lse_parts, int G, int64_t rows,
+                                   int d, int H, const float* sink, void* out, float* lse_out,
+                                   void* stream);
 
 /* ---------------------------------------------------------------------------------------
  * Failure-detection self-test: launches one block whose bounded wait on an mbarrier that

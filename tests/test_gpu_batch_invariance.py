@@ -44,6 +44,7 @@ def _run(cfg, seqs, fused):
 
 @pytest.mark.parametrize("fused", [True, False])
 def test_csa_decode_128k_batch_invariant(hcl, fused):
+    """bf16 index operands, fp32 scores: the separate top-k and attention kernels."""
     cfg = CSA_128K
     full = _run(cfg, list(range(32)), fused)
     seven = _run(cfg, list(range(7)), fused)
@@ -52,3 +53,40 @@ def test_csa_decode_128k_batch_invariant(hcl, fused):
         assert torch.equal(a[:7], b)
     for a, b in zip(full, one):
         assert torch.equal(a[:1], b)
+
+
+def _run_mxfp4(cfg, seqs):
+    """The 1M-decode path's formats (MXFP4 keys, bf16 scores, FP8 split KV rows) through the fused
+    step, whose selection and attention run as one cluster kernel per sequence."""
+    from heavily_compressed_long_b200 import api
+    from heavily_compressed_long_b200.api import HCL_BF16, HCL_MXFP4
+    B, L, W, Nc = len(seqs), cfg.L, cfg.W, cfg.Nc
+    dev = "cuda"
+    kp = torch.empty(B, Nc, 32, dtype=torch.uint8, device=dev)
+    ks = torch.empty(B, Nc, 2, dtype=torch.uint8, device=dev)
+    cn = torch.empty(B, Nc, 64, dtype=torch.uint8, device=dev)
+    cs = torch.empty(B, Nc, dtype=torch.float32, device=dev)
+    cr = torch.empty(B, Nc, 64, dtype=torch.bfloat16, device=dev)
+    api.hcl_quant_mxfp4(cuda(gen.index_keys(cfg, seqs)), kp, ks)
+    api.hcl_quant_kv_fp8(cuda(gen.comp_kv(cfg, seqs, Nc)), cn, cs, cr)
+    rn = torch.empty(B, W, 64, dtype=torch.uint8, device=dev)
+    rs = torch.empty(B, W, dtype=torch.float32, device=dev)
+    rr = torch.empty(B, W, 64, dtype=torch.bfloat16, device=dev)
+    api.hcl_quant_kv_fp8(cuda(gen.raw_kv(cfg, seqs, L - W, L)), rn, rs, rr)
+    q, qI, w = gen.queries(cfg, seqs), gen.index_queries(cfg, seqs), gen.head_weights(cfg, seqs)
+    pos = gen.query_positions(cfg, B)
+    pipe = CsaDecode(cuda(q), cuda(qI), cuda(w), kp, KV(cn, cs, cr), Nc, KV(rn, rs, rr), L, W,
+                     cuda(pos), m=cfg.m, k=cfg.k, op_fmt=HCL_MXFP4, score_fmt=HCL_BF16, kI_sf=ks)
+    pipe.step()
+    torch.cuda.synchronize()
+    assert pipe.status.item() == 0
+    return pipe.idx.cpu(), pipe.out.cpu(), pipe.lse.cpu()
+
+
+def test_csa_decode_mxfp4_batch_invariant(hcl):
+    from synth.configs import CSA_1M, scaled
+    cfg = scaled(CSA_1M, L=4 * 70000)
+    full = _run_mxfp4(cfg, [0, 1, 2])
+    one = _run_mxfp4(cfg, [1])
+    for a, b in zip(full, one):
+        assert torch.equal(a[1:2], b)
