@@ -120,6 +120,49 @@ __device__ __forceinline__ void rmsnorm8_group(float (&v)[8], int G, int d, int 
   for (int c = 0; c < 8; c++) v[c] = v[c] * r * __ldg(gamma + chunk * 8 + c);
 }
 
+// The second half of a long-span pooling (see pool_long_block): thread t of a block of 128
+// merges, for channels c = t + 128u (c < d), the S stream partials (max, sum, weighted sum)
+// that sm holds ([S][3][d] floats, then 4 floats of scratch) into the entry value vals[u],
+// RMS-normalised with gamma when given.  All 128 threads must call it.
+__device__ __forceinline__ void merge_streams_block(float* sm, int streams, int d,
+                                                    const float* __restrict__ gamma, float eps,
+                                                    float (&vals)[8]) {
+  float ss = 0.f;
+#pragma unroll
+  for (int u = 0; u < 8; u++) {
+    const int c = threadIdx.x + u * 128;
+    vals[u] = 0.f;
+    if (c >= d) continue;
+    float M = -INFINITY;
+    for (int q = 0; q < streams; q++) M = fmaxf(M, sm[(size_t)q * 3 * d + c]);
+    float S = 0.f, A = 0.f;
+    if (M > -INFINITY) {
+      for (int q = 0; q < streams; q++) {
+        const float* base = sm + (size_t)q * 3 * d;
+        if (base[c] == -INFINITY) continue;
+        const float r = __expf(base[c] - M);
+        S += base[d + c] * r;
+        A += base[2 * d + c] * r;
+      }
+    }
+    vals[u] = S > 0.f ? A / S : 0.f;
+    ss = fmaf(vals[u], vals[u], ss);
+  }
+  if (gamma != nullptr) {
+    float* red = sm + (size_t)streams * 3 * d;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    const float rn = 1.f / sqrtf((red[0] + red[1] + red[2] + red[3]) / float(d) + eps);
+#pragma unroll
+    for (int u = 0; u < 8; u++) {
+      const int c = threadIdx.x + u * 128;
+      if (c < d) vals[u] = vals[u] * rn * __ldg(gamma + c);
+    }
+  }
+}
+
 // Long spans (HCA): one entry per block of 128 threads.  Thread t works on channel chunk
 // t % G (G = d/8) of slot stream t / G; stream s takes slots s, s + S, s + 2S, ... (S = 128/G
 // streams); the streams' partial softmaxes are merged
@@ -155,40 +198,7 @@ __device__ __forceinline__ void pool_long_block(RowFn row, const float* __restri
     }
   }
   __syncthreads();
-  float ss = 0.f;
-#pragma unroll
-  for (int u = 0; u < 8; u++) {
-    const int c = threadIdx.x + u * 128;
-    vals[u] = 0.f;
-    if (c >= d) continue;
-    float M = -INFINITY;
-    for (int q = 0; q < streams; q++) M = fmaxf(M, sm[(size_t)q * 3 * d + c]);
-    float S = 0.f, A = 0.f;
-    if (M > -INFINITY) {
-      for (int q = 0; q < streams; q++) {
-        const float* base = sm + (size_t)q * 3 * d;
-        if (base[c] == -INFINITY) continue;
-        const float r = __expf(base[c] - M);
-        S += base[d + c] * r;
-        A += base[2 * d + c] * r;
-      }
-    }
-    vals[u] = S > 0.f ? A / S : 0.f;
-    ss = fmaf(vals[u], vals[u], ss);
-  }
-  if (gamma != nullptr) {
-    float* red = sm + (size_t)streams * 3 * d;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-    __syncthreads();
-    const float rn = 1.f / sqrtf((red[0] + red[1] + red[2] + red[3]) / float(d) + eps);
-#pragma unroll
-    for (int u = 0; u < 8; u++) {
-      const int c = threadIdx.x + u * 128;
-      if (c < d) vals[u] = vals[u] * rn * __ldg(gamma + c);
-    }
-  }
+  merge_streams_block(sm, streams, d, gamma, eps, vals);
 }
 
 }  // namespace hcl
