@@ -816,6 +816,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
     }
     umma_commit(bar_s);
   }
+  __syncwarp();   // warp 0 reconverges before waiting (the issuing lane is not left behind)
   bool ok = nch == 0 || mbar_wait(bar_s, 0, limit, nullptr);
   if (!ok) report(p.status, HCL_ERR_TIMEOUT);
   tc_fence_after();
@@ -909,6 +910,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
     }
     umma_commit(bar_o);
   }
+  __syncwarp();
   ok = nch == 0 || mbar_wait(bar_o, 0, limit, nullptr);
   if (!ok) report(p.status, HCL_ERR_TIMEOUT);
   __syncthreads();               // the partial sums

@@ -255,6 +255,7 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
       }
       umma_commit(bar_s);
     }
+    __syncwarp();   // warp 0 reconverges before waiting (the issuing lane is not left behind)
     ok = ok && mbar_wait(bar_s, rd & 1, p.limit, nullptr);
     tc_fence_after();
     // two passes over this thread's 32 columns of each chunk: maximum, then exponentials
@@ -323,6 +324,7 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
       }
       umma_commit(bar_o);
     }
+    __syncwarp();
     ok = ok && mbar_wait(bar_o, rd & 1, p.limit, nullptr);
     tc_fence_after();
     {

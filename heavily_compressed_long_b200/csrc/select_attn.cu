@@ -11,14 +11,17 @@
 // contiguous range of G groups and a share of the window rows.
 //   1. Before the indexer finishes (programmatic dependent launch), every CTA loads the
 //      query heads (optionally RMS-normalised) and starts gathering its window rows.
-//   2. L = the k-th largest group maximum, exactly, by a two-digit (8 + 8 bit) radix search
-//      whose per-digit counts every CTA pulls from the cluster's shared memory.  L is a lower
-//      bound of the k-th largest score (the maxima are scores of distinct entries).
+//   2. L = the k-th largest group maximum, exactly, by a two-digit (8 + 8 bit) radix search:
+//      every CTA pushes its per-digit counts into every CTA's shared memory (remote stores),
+//      one cluster barrier per digit, and adds the copies locally.  L is a lower bound of the
+//      k-th largest score (the maxima are scores of distinct entries).
 //   3. Each CTA lists its candidates, the entries with key >= L (a group whose second largest
 //      is below L gives its single candidate from the summary; the others' scores are read),
-//      in index order.  One cluster barrier, then every CTA pulls all candidate keys (about k
-//      of them) and finds the exact k-th largest key T and the ties to take locally, and --
-//      from the keys of the CTAs before it -- the output positions of its own selected entries.
+//      in index order, and pushes their keys (about k / S) to every CTA.  After one cluster
+//      barrier every CTA holds all candidate keys and finds locally the exact k-th largest key
+//      T, the ties to take and -- from the keys of the CTAs before it -- the output positions
+//      of its own selected entries.  (Only remote stores cross CTAs: a remote load costs a
+//      full round trip, a store is paid for at the barrier.)
 //   4. Each CTA writes its part of the selected indices (ascending overall) and attends over
 //      its own rows: S = Q K^T and O = P V on tcgen05 (heads = M = 128 TMEM lanes, rows in
 //      chunks of 64, two chunks per round, online softmax across rounds in registers).
@@ -46,10 +49,11 @@ constexpr int SA_ROWS = 128;      // heads per CTA = UMMA M = TMEM lanes
 constexpr int SA_D = 128;
 constexpr int SA_CH = 64;         // KV rows per chunk (UMMA N of S = Q K^T)
 constexpr int SA_RCH = 2;         // chunks per round
-constexpr int SA_MAXS = 16;       // largest cluster the code handles
-constexpr int SA_USE_S = 8;       // CTAs per sequence used (portable cluster size)
-constexpr int SA_CAND_CAP = 1024; // candidates a CTA may list
+constexpr int SA_USE_S = 8;       // CTAs per sequence, at most (portable cluster size)
+constexpr int SA_MAXS = SA_USE_S;
 constexpr int SA_ALL_CAP = 4096;  // candidates of the whole cluster
+constexpr int SA_CAPS = SA_ALL_CAP / SA_USE_S;   // candidates a CTA may list and push
+constexpr int SA_CAND_CAP = SA_CAPS;
 constexpr int SA_MAX_ROWS = 4096 + 256;  // a CTA's row list: selected entries + window share
 constexpr float SA_LOG2E = 1.4426950408889634f;
 constexpr float SA_LN2 = 0.6931471805599453f;
@@ -87,23 +91,27 @@ struct SaOff {
   static constexpr uint32_t SCL = STG + SA_RCH * 4096;    // row scales
   static constexpr uint32_t ROWS = SCL + SA_RCH * 256;    // row list
   static constexpr uint32_t CAND = ROWS + SA_MAX_ROWS * 4;     // key << 16 | local entry
-  static constexpr uint32_t ALLK = CAND + SA_CAND_CAP * 4;     // pulled keys (u16)
-  static constexpr uint32_t HA = ALLK + SA_ALL_CAP * 2;        // 256-bin digit counts
+  static constexpr uint32_t ALLK = CAND + SA_CAND_CAP * 4;     // pushed keys [S][SA_CAPS] u16
+  static constexpr uint32_t HA = ALLK + SA_ALL_CAP * 2;        // 256-bin digit counts (local)
   static constexpr uint32_t HB = HA + 1024;
   static constexpr uint32_t HC = HB + 1024;
-  static constexpr uint32_t XCH = HC + 1024;                   // [2][256] floats
+  static constexpr uint32_t RA = HC + 1024;                    // pushed counts [S][256] u16
+  static constexpr uint32_t RB = RA + SA_USE_S * 512;
+  static constexpr uint32_t XCH = RB + SA_USE_S * 512;         // [2][256] floats
   static constexpr uint32_t META = XCH + 2048;                 // 64 u32 of scalars
   static constexpr uint32_t BAR = META + 256;                  // 2 mbarriers + TMEM address
   static constexpr uint32_t VIS = BAR + 32;                    // row visibility bits of a round
   static constexpr uint32_t RECV = VIS + 64;                   // merge: rpo x S x 128 floats
-  static constexpr uint32_t RECV_BYTES = (SA_ROWS + SA_MAXS) * SA_D * 4;
+  static constexpr uint32_t RECV_BYTES = (SA_ROWS + SA_USE_S) * SA_D * 4;
   static constexpr uint32_t RLSE = RECV + RECV_BYTES;
-  static constexpr uint32_t TOTAL = RLSE + (SA_ROWS + SA_MAXS) * 4;
+  static constexpr uint32_t TOTAL = RLSE + (SA_ROWS + SA_USE_S) * 4;
 };
 
 // meta words
 enum : int { M_NCAND = 0, M_OVF = 1, M_T = 2, M_ABOVE = 3, M_FOUND = 4, M_L = 5, M_NSEL = 6,
-             M_CNTG = 7, M_CNTE = 8, M_TMP = 16 };
+             M_CNTG = 7, M_CNTE = 8, M_TMP = 16,
+             M_IN_CAND = 32,   // pushed by CTA r: [32 + 2r] candidates, [33 + 2r] overflow
+             M_IN_CNT = 48 };  // pushed by CTA r: [48 + 2r] keys > T, [49 + 2r] keys == T
 
 __device__ __forceinline__ uint32_t okey(uint16_t bits) {
   return uint32_t(bits ^ ((bits & 0x8000u) ? 0xFFFFu : 0x8000u));
@@ -189,36 +197,44 @@ __device__ __forceinline__ void find_digit(const uint32_t* cnt, uint32_t target,
   if (lane == 0) meta[M_FOUND] = any ? 1u : 0u;
 }
 
-// Sum over the cluster's CTAs of word threadIdx.x of array `a` (in every CTA's shared memory):
-// the remote loads of all sources are issued before any is used.
-__device__ __forceinline__ uint32_t pull_sum(cg::cluster_group& cl, uint32_t* a, int S) {
-  uint32_t v[SA_MAXS];
+// Every CTA of the cluster receives this CTA's count v (< 2^16) of digit threadIdx.x in slot
+// [c][threadIdx.x] of its `recv` (remote stores, made visible by the next cluster barrier).
+__device__ __forceinline__ void push16(cg::cluster_group& cl, uint16_t* recv, uint32_t v, int S,
+                                       int c) {
 #pragma unroll
-  for (int r = 0; r < SA_MAXS; r++) v[r] = r < S ? cl.map_shared_rank(a, r)[threadIdx.x] : 0u;
+  for (int r = 0; r < SA_MAXS; r++)
+    if (r < S) cl.map_shared_rank(recv, r)[c * 256 + threadIdx.x] = uint16_t(v);
+}
+
+__device__ __forceinline__ uint32_t sum16(const uint16_t* recv, int S) {
   uint32_t s = 0;
 #pragma unroll
-  for (int r = 0; r < SA_MAXS; r++) s += v[r];
+  for (int r = 0; r < SA_MAXS; r++)
+    if (r < S) s += recv[r * 256 + threadIdx.x];
   return s;
 }
 
 // Cluster-wide selection of the target-th largest 16-bit key among the keys the CTAs
 // enumerate (for_each(f) calls f(key, valid) a uniform number of times per thread).  Two
-// digits of 8 bits; each CTA counts its own keys into hA / hB and pulls the cluster's counts
-// after a cluster barrier.  Returns found (false: fewer than target keys), T and the number of
-// keys > T.  Uses two cluster barriers; hA / hB must not be read remotely by an earlier call
-// after its second barrier.
+// digits of 8 bits; each CTA counts its own keys (hA / hB) and pushes the counts to every CTA
+// (rA / rB, [S][256] u16: per-CTA counts stay below 2^16), one cluster barrier per digit, then
+// every CTA adds the S copies locally.  Returns found (false: fewer than target keys), T and
+// the number of keys > T.  Two cluster barriers; a later call may push into rA / rB only after
+// a barrier that follows this call's last local read of them.
 template <class ForEach>
 __device__ bool cluster_select16(cg::cluster_group& cl, ForEach for_each, uint32_t target,
-                                 uint32_t* hA, uint32_t* hB, uint32_t* meta, uint32_t* tot,
-                                 uint32_t& T, uint32_t& above) {
+                                 uint32_t* hA, uint32_t* hB, uint16_t* rA, uint16_t* rB,
+                                 uint32_t* meta, uint32_t* tot, uint32_t& T, uint32_t& above) {
   const int tid = threadIdx.x;
-  const int S = (int)cl.num_blocks();
+  const int S = (int)cl.num_blocks(), c = (int)cl.block_rank();
   hA[tid] = 0u;
   hB[tid] = 0u;
   __syncthreads();
   for_each([&](uint32_t key, bool valid) { hist_inc(hA, key >> 8, valid); });
+  __syncthreads();
+  push16(cl, rA, hA[tid], S, c);
   cl.sync();
-  tot[tid] = pull_sum(cl, hA, S);
+  tot[tid] = sum16(rA, S);
   __syncthreads();
   find_digit(tot, target, meta);
   __syncthreads();
@@ -229,8 +245,10 @@ __device__ bool cluster_select16(cg::cluster_group& cl, ForEach for_each, uint32
   const uint32_t hi = meta[M_T], ab_hi = meta[M_ABOVE];
   __syncthreads();
   for_each([&](uint32_t key, bool valid) { hist_inc(hB, key & 255u, valid && (key >> 8) == hi); });
+  __syncthreads();
+  push16(cl, rB, hB[tid], S, c);
   cl.sync();
-  tot[tid] = pull_sum(cl, hB, S);
+  tot[tid] = sum16(rB, S);
   __syncthreads();
   find_digit(tot, target - ab_hi, meta);
   __syncthreads();
@@ -273,6 +291,8 @@ __global__ void __launch_bounds__(SA_THREADS, 1) select_attn_kernel(SaParams p) 
   uint32_t* hA = reinterpret_cast<uint32_t*>(sm + SaOff::HA);
   uint32_t* hB = reinterpret_cast<uint32_t*>(sm + SaOff::HB);
   uint32_t* hC = reinterpret_cast<uint32_t*>(sm + SaOff::HC);
+  uint16_t* rA = reinterpret_cast<uint16_t*>(sm + SaOff::RA);
+  uint16_t* rB = reinterpret_cast<uint16_t*>(sm + SaOff::RB);
   float* xch = reinterpret_cast<float*>(sm + SaOff::XCH);
   uint32_t* meta = reinterpret_cast<uint32_t*>(sm + SaOff::META);
   uint64_t* bar_s = reinterpret_cast<uint64_t*>(sm + SaOff::BAR);
@@ -428,7 +448,7 @@ __global__ void __launch_bounds__(SA_THREADS, 1) select_attn_kernel(SaParams p) 
           for (int i = 0; i < 16; i++)
             if (i < p.gpt) f(mx[i], mx[i] != 0u);
         },
-        (uint32_t)k, hA, hB, meta, hC, L, ab);
+        (uint32_t)k, hA, hB, rA, rB, meta, hC, L, ab);
     if (!haveL || L == 0u) L = 1u;   // fewer than k groups: every visible entry is a candidate
 
     // ---- 3. candidates (key >= L) in index order -------------------------------------
@@ -444,7 +464,7 @@ __global__ void __launch_bounds__(SA_THREADS, 1) select_attn_kernel(SaParams p) 
     }
     uint32_t ncta;
     uint32_t off = scan256(nmine, tmp, ncta);
-    const bool ovf_local = ncta > (uint32_t)SA_CAND_CAP;
+    const bool ovf_local = ncta > (uint32_t)SA_CAPS;
     if (!ovf_local) {
 #pragma unroll
       for (int i = 0; i < 16; i++) {
@@ -458,64 +478,50 @@ __global__ void __launch_bounds__(SA_THREADS, 1) select_attn_kernel(SaParams p) 
           if (kk[j] >= L) cand[off++] = (kk[j] << 16) | (lg + j);
       }
     }
-    if (tid == 0) { meta[M_NCAND] = ncta; meta[M_OVF] = ovf_local ? 1u : 0u; }
-    cl.sync();
-    // every CTA pulls the cluster's candidate counts (lane r of warp 0 reads CTA r) ...
-    uint32_t* srcoff = meta + 32;                        // [SA_MAXS + 1] key offsets per source
-    if (warp == 0) {
-      uint32_t n = 0, o = 0;
-      if (lane < S) {
-        const uint32_t* mr = cl.map_shared_rank(meta, lane);
-        n = mr[M_NCAND];
-        o = mr[M_OVF];
-      }
-      uint32_t inc = n;
-#pragma unroll
-      for (int d2 = 1; d2 < 32; d2 <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, d2);
-        if (lane >= d2) inc += y;
-      }
-      const unsigned anyo = __ballot_sync(0xffffffffu, o != 0u);
-      if (lane <= S) srcoff[lane] = inc - n + (lane == S ? 0u : 0u);
-      if (lane == S - 1) srcoff[S] = inc;
-      if (lane == 0) meta[M_TMP + 12] = anyo ? 1u : 0u;
-    }
     __syncthreads();
-    const uint32_t tot_c = srcoff[S], before_c = srcoff[c];
-    bool ovf = meta[M_TMP + 12] != 0u || tot_c > (uint32_t)SA_ALL_CAP;
+    // push this CTA's candidate count, overflow flag and keys to every CTA of the cluster
+    if (tid < S) {
+      uint32_t* dst = cl.map_shared_rank(meta, tid) + M_IN_CAND + 2 * c;
+      dst[0] = ncta;
+      dst[1] = ovf_local ? 1u : 0u;
+    }
+    if (!ovf_local) {
+      for (uint32_t j = tid; j < ncta; j += SA_THREADS) {
+        const uint16_t key = uint16_t(cand[j] >> 16);
+#pragma unroll
+        for (int r = 0; r < SA_MAXS; r++)
+          if (r < S) cl.map_shared_rank(allk, r)[c * SA_CAPS + j] = key;
+      }
+    }
+    cl.sync();
+    uint32_t tot_c = 0, before_c = 0;
+    bool ovf = false;
+    for (int r = 0; r < S; r++) {
+      const uint32_t n = meta[M_IN_CAND + 2 * r];
+      ovf |= meta[M_IN_CAND + 2 * r + 1] != 0u;
+      if (r < c) before_c += n;
+      tot_c += n;
+    }
     uint32_t T = 0u, above = 0u, gt_before = 0u, eq_before = 0u;
-    bool exact_path = !ovf;
+    const bool exact_path = !ovf;
     if (exact_path) {
-      // pull the keys: CTA r's candidates go to allk[off_r ...]
-      // ... and keys: key j of the cluster's list comes from the source whose offset range
-      // holds it; up to SA_ALL_CAP / 256 loads per thread, all in flight together
+      // ---- the exact k-th largest of the candidate keys (local two-digit search over the
+      // pushed segments: CTA r's keys in allk[r * SA_CAPS, + n_r)) -----------------------
       constexpr int PER = SA_ALL_CAP / SA_THREADS;
-      uint32_t kv_[PER];
-#pragma unroll
-      for (int it = 0; it < PER; it++) {
-        const uint32_t j = uint32_t(it * SA_THREADS + tid);
-        kv_[it] = 0u;
-        if (j < tot_c) {
-          int r = 0;
-#pragma unroll
-          for (int q2 = 1; q2 < SA_MAXS; q2++) r += (q2 < S && srcoff[q2] <= j) ? 1 : 0;
-          kv_[it] = cl.map_shared_rank(cand, r)[j - srcoff[r]];
-        }
-      }
-#pragma unroll
-      for (int it = 0; it < PER; it++) {
-        const uint32_t j = uint32_t(it * SA_THREADS + tid);
-        if (j < tot_c) allk[j] = uint16_t(kv_[it] >> 16);
-      }
+      auto slot_key = [&](int it, uint32_t& key) {
+        const int q2 = it * SA_THREADS + tid;
+        const int r = q2 / SA_CAPS, j = q2 % SA_CAPS;
+        const bool v = r < S && (uint32_t)j < meta[M_IN_CAND + 2 * min(r, S - 1)];
+        key = v ? allk[q2] : 0u;
+        return v;
+      };
+      hA[tid] = 0u;
       __syncthreads();
-      // ---- the exact k-th largest of the candidate keys (local two-digit search) -------
-      hA[tid] = 0u;   // safe: the last remote reads of hA happened before the barrier above
-      __syncthreads();
-      const int per = (int)((tot_c + SA_THREADS - 1) / SA_THREADS);
-      for (int it = 0; it < per; it++) {
-        const uint32_t j = uint32_t(it * SA_THREADS + tid);
-        const uint32_t key = j < tot_c ? allk[j] : 0u;
-        hist_inc(hA, key >> 8, j < tot_c);
+#pragma unroll 4
+      for (int it = 0; it < PER; it++) {
+        uint32_t key;
+        const bool v = slot_key(it, key);
+        hist_inc(hA, key >> 8, v);
       }
       __syncthreads();
       find_digit(hA, (uint32_t)k, meta);
@@ -524,10 +530,11 @@ __global__ void __launch_bounds__(SA_THREADS, 1) select_attn_kernel(SaParams p) 
       __syncthreads();
       hA[tid] = 0u;
       __syncthreads();
-      for (int it = 0; it < per; it++) {
-        const uint32_t j = uint32_t(it * SA_THREADS + tid);
-        const uint32_t key = j < tot_c ? allk[j] : 0u;
-        hist_inc(hA, key & 255u, j < tot_c && (key >> 8) == hi);
+#pragma unroll 4
+      for (int it = 0; it < PER; it++) {
+        uint32_t key;
+        const bool v = slot_key(it, key);
+        hist_inc(hA, key & 255u, v && (key >> 8) == hi);
       }
       __syncthreads();
       find_digit(hA, (uint32_t)k - ab_hi, meta);
@@ -536,9 +543,11 @@ __global__ void __launch_bounds__(SA_THREADS, 1) select_attn_kernel(SaParams p) 
       above = ab_hi + meta[M_ABOVE];
       // keys > T and == T among the candidates of the CTAs before this one
       uint32_t g = 0, e = 0;
-      for (uint32_t j = tid; j < before_c; j += SA_THREADS) {
-        g += allk[j] > T;
-        e += allk[j] == T;
+#pragma unroll 4
+      for (int it = 0; it < PER; it++) {
+        uint32_t key;
+        const int q2 = it * SA_THREADS + tid;
+        if (slot_key(it, key) && q2 / SA_CAPS < c) { g += key > T; e += key == T; }
       }
       uint32_t tg, te;
       scan256(g, tmp, tg);
@@ -557,9 +566,9 @@ __global__ void __launch_bounds__(SA_THREADS, 1) select_attn_kernel(SaParams p) 
               for (int j = 0; j < 16; j++) f(any ? kk[j] : 0u, any && kk[j] != 0u);
             }
           },
-          (uint32_t)k, hA, hB, meta, hC, T, above);
+          (uint32_t)k, hA, hB, rA, rB, meta, hC, T, above);
       if (!ok) report(p.status, HCL_ERR_DEVICE_FAULT);   // cannot happen: nvis > k
-      // this CTA's counts of > T and == T, published, then the counts of the CTAs before it
+      // this CTA's counts of > T and == T, pushed to every CTA, then those of the CTAs before
       uint32_t g = 0, e = 0;
       for (int i = 0; i < p.gpt; i++) {
         if (g0 + i >= ngv) break;
@@ -571,25 +580,19 @@ __global__ void __launch_bounds__(SA_THREADS, 1) select_attn_kernel(SaParams p) 
       uint32_t tg, te;
       scan256(g, tmp, tg);
       scan256(e, tmp, te);
-      if (tid == 0) { meta[M_CNTG] = tg; meta[M_CNTE] = te; }
+      if (tid < S) {
+        uint32_t* dst = cl.map_shared_rank(meta, tid) + M_IN_CNT + 2 * c;
+        dst[0] = tg;
+        dst[1] = te;
+      }
       cl.sync();
       uint32_t gb2 = 0, eb2 = 0;
-      if (warp == 0) {
-        if (lane < c) {
-          const uint32_t* mr = cl.map_shared_rank(meta, lane);
-          gb2 = mr[M_CNTG];
-          eb2 = mr[M_CNTE];
-        }
-#pragma unroll
-        for (int d2 = 16; d2 > 0; d2 >>= 1) {
-          gb2 += __shfl_xor_sync(0xffffffffu, gb2, d2);
-          eb2 += __shfl_xor_sync(0xffffffffu, eb2, d2);
-        }
-        if (lane == 0) { meta[M_TMP + 13] = gb2; meta[M_TMP + 14] = eb2; }
+      for (int r = 0; r < c; r++) {
+        gb2 += meta[M_IN_CNT + 2 * r];
+        eb2 += meta[M_IN_CNT + 2 * r + 1];
       }
-      __syncthreads();
-      gt_before = meta[M_TMP + 13];
-      eq_before = meta[M_TMP + 14];
+      gt_before = gb2;
+      eq_before = eb2;
     }
     const uint32_t krem = (uint32_t)k - above;
     const uint32_t base_slot = gt_before + min(eq_before, krem);
@@ -777,6 +780,7 @@ __global__ void __launch_bounds__(SA_THREADS, 1) select_attn_kernel(SaParams p) 
       }
       umma_commit(bar_s);
     }
+    __syncwarp();   // warp 0 reconverges before waiting (the issuing lane is not left behind)
     ok = ok && mbar_wait(bar_s, rd & 1, p.limit, nullptr);
     tc_fence_after();
     // softmax of the round: this thread holds columns 32*hc .. 32*hc+31 of every chunk
@@ -839,6 +843,7 @@ __global__ void __launch_bounds__(SA_THREADS, 1) select_attn_kernel(SaParams p) 
       }
       umma_commit(bar_o);
     }
+    __syncwarp();
     ok = ok && mbar_wait(bar_o, rd & 1, p.limit, nullptr);
     tc_fence_after();
     {
