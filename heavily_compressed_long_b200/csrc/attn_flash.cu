@@ -1,9 +1,10 @@
-// attn_flash.cu -- HCA dense attention for prefill chunks on tcgen05 tensor cores.
+// attn_flash.cu -- prefill attention on tcgen05 tensor cores (HCA dense, CSA selected).
 //
 // [Tripbot §3.2; CSDN §1.2] HCA attends densely over every compressed entry visible to the
 // query (entry i of ratio m' is visible at position p when m'(i+1) - 1 <= p) and [Tripbot §3.3]
 // over the raw tokens of its sliding window, under one softmax (scale, optional sink); each
-// row is both key and value of the one shared KV head.
+// row is both key and value of the one shared KV head.  [Tripbot §3.1 step 2] CSA attends
+// over the query's own top-k entries plus the same window.
 //
 // Design (B200): one block of 256 threads per query group: G = floor(128 / H) consecutive
 // queries x H heads = up to 128 (query, head) rows = the UMMA M dimension = 128 TMEM lanes, two
@@ -16,6 +17,12 @@
 // bit masks), online across rounds: O of a round is added to the register accumulator after
 // rescaling by the change of the running maximum.  Two blocks fit per SM (about 106 KB of
 // shared memory, 256 TMEM columns each), so one block's gather overlaps the other's MMAs.
+//
+// CSA prefill (every query has its own selection) uses the same kernel with G = 128 / H
+// queries per block (2 at H = 64): the KV list is the concatenation of the G queries' lists
+// (selected entries, then window) and each row's mask keeps its own query's segment, so the
+// MMAs do G times the useful work -- on the tensor pipe, which has the room, and used only for
+// H >= 32.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -35,8 +42,11 @@ constexpr float FA_LOG2E = 1.4426950408889634f;
 constexpr float FA_LN2 = 0.6931471805599453f;
 
 struct FaParams {
+  int mode;                 // 1: HCA (shared visible prefix + window union); 0: CSA segments
   const __nv_bfloat16* q;   // [B, Tq, H, 128]
   int B, Tq, H, G, n_groups;
+  const int32_t* idx;       // CSA: [B, Tq, k]
+  int k;
   hcl_kv_t comp, raw;
   int Nh, mh, W;
   const int32_t* q_pos;
@@ -58,7 +68,7 @@ struct FaOff {
   static constexpr uint32_t SCL = STG + FA_RCH * 4096;
   static constexpr uint32_t XCH = SCL + FA_RCH * 256;
   static constexpr uint32_t BAR = XCH + 2 * FA_THREADS * 4;
-  static constexpr uint32_t TOTAL = BAR + 32;
+  static constexpr uint32_t TOTAL = BAR + 64;
 };
 
 __device__ __forceinline__ uint32_t fa_pack(float lo, float hi) {
@@ -116,18 +126,29 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
     pmin = min(pmin, pp);
     pmax = max(pmax, pp);
   }
+  // HCA list: the visible-entry prefix [0, n_a) of the last query, then window tokens
+  // raw_lo .. raw_lo + n_raw - 1; CSA list: G segments of k + W rows (query i's selection, then
+  // its window)
   const int n_a = pmax < 0 ? 0 : min(p.Nh, (pmax + 1) / p.mh);
   const int raw_lo = pmin - p.W + 1;
   const int n_raw = (p.W > 0 && pmax >= 0) ? max(0, pmax - raw_lo + 1) : 0;
-  const int total = n_a + n_raw;
-  // list rows visible to this row: entries [0, nv_e) and window rows [w_lo, w_hi)
-  const int nv_e = my_p < 0 ? 0 : min(n_a, (my_p + 1) / p.mh);
-  int w_lo = 0, w_hi = 0;
-  if (rv && my_p >= 0 && p.W > 0) {
-    const int u_lo = max(0, my_p - p.W + 1);
-    w_lo = n_a + (u_lo - raw_lo);
-    w_hi = n_a + (my_p - raw_lo) + 1;
+  const int seg = p.k + p.W;
+  const int total = p.mode == 1 ? n_a + n_raw : gq * seg;
+  // list rows visible to this row: HCA: entries [0, nv_e) and window rows [w_lo, w_hi);
+  // CSA: its own segment [w_lo, w_hi) (invalid rows are masked by the round's row bits)
+  int nv_e = 0, w_lo = 0, w_hi = 0;
+  if (p.mode == 1) {
+    nv_e = my_p < 0 ? 0 : min(n_a, (my_p + 1) / p.mh);
+    if (rv && my_p >= 0 && p.W > 0) {
+      const int u_lo = max(0, my_p - p.W + 1);
+      w_lo = n_a + (u_lo - raw_lo);
+      w_hi = n_a + (my_p - raw_lo) + 1;
+    }
+  } else if (rv) {
+    w_lo = qi * seg;
+    w_hi = w_lo + seg;
   }
+  uint32_t* rbits = reinterpret_cast<uint32_t*>(sm + FaOff::BAR + 32);   // 4 words per round
 
   // Q rows (query qi, head hh) -> SW128 halves, optionally RMS-normalised
   {
@@ -193,11 +214,23 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
       long long slot = -1;
       const hcl_kv_t* st = &p.comp;
       if (jj < nr) {
-        if (e < n_a) {
-          slot = (long long)b * p.comp.cap + (e % p.comp.cap);
+        if (p.mode == 1) {
+          if (e < n_a) {
+            slot = (long long)b * p.comp.cap + (e % p.comp.cap);
+          } else {
+            const long long tok = (long long)raw_lo + (e - n_a);
+            if (tok >= 0) { st = &p.raw; slot = (long long)b * p.raw.cap + tok % p.raw.cap; }
+          }
         } else {
-          const long long tok = (long long)raw_lo + (e - n_a);
-          if (tok >= 0) { st = &p.raw; slot = (long long)b * p.raw.cap + tok % p.raw.cap; }
+          const int sq = e / seg, se = e % seg;
+          if (se < p.k) {
+            const int ent = p.idx[((size_t)b * p.Tq + t0 + sq) * p.k + se];
+            if (ent >= 0 && ent < p.Nh) slot = (long long)b * p.comp.cap + (ent % p.comp.cap);
+            else if (ent >= p.Nh || ent < -1) report(p.status, HCL_ERR_DEVICE_FAULT);
+          } else {
+            const long long tok = (long long)p.q_pos[(size_t)b * p.Tq + t0 + sq] - p.W + 1 + (se - p.k);
+            if (tok >= 0) { st = &p.raw; slot = (long long)b * p.raw.cap + tok % p.raw.cap; }
+          }
         }
       }
       uint8_t* kv = sm + FaOff::KV + ch * 16384;
@@ -223,6 +256,22 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
       }
     }
     cp_async_commit();
+    if (p.mode == 0) {
+      // valid list rows of the round (a selected entry, or a window token >= 0)
+      const int jj = tid;
+      bool v = false;
+      if (jj < nr) {
+        const int e = r0 + jj, sq = e / seg, se = e % seg;
+        if (se < p.k) {
+          const int ent = p.idx[((size_t)b * p.Tq + t0 + sq) * p.k + se];
+          v = ent >= 0 && ent < p.Nh;
+        } else {
+          v = (long long)p.q_pos[(size_t)b * p.Tq + t0 + sq] - p.W + 1 + (se - p.k) >= 0;
+        }
+      }
+      const uint32_t bits = __ballot_sync(0xffffffffu, v);
+      if ((tid & 31) == 0 && tid < FA_RCH * FA_CH) rbits[tid >> 5] = bits;
+    }
     cp_async_wait<0>();
     __syncthreads();
     if (KVFMT == HCL_FP8SPLIT) {
@@ -269,6 +318,7 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
         const int c0 = r0 + ch * FA_CH + hc * 32;
         vb[ch] = (range_bits(c0, 0, nv_e) | range_bits(c0, w_lo, w_hi)) &
                  range_bits(c0, r0, r0 + nr);
+        if (p.mode == 0) vb[ch] &= rbits[2 * ch + hc];
       }
       if (ch < nch) {
         uint32_t sv[32];
@@ -391,20 +441,26 @@ hcl_status_t launch_flash_t(const FaParams& p, cudaStream_t st) {
 }  // namespace
 
 bool hca_flash_usable(const AttnArgs& a) {
-  if (a.mode != 1 || a.H > FA_ROWS || a.d != FA_D) return false;
+  if (a.H > FA_ROWS || a.d != FA_D) return false;
+  if (!(a.comp.fmt == HCL_BF16 || a.comp.fmt == HCL_FP8SPLIT)) return false;
   const int G = std::max(1, FA_ROWS / a.H);
   const int n_groups = (a.Tq + G - 1) / G;
-  return n_groups >= 32 && (a.comp.fmt == HCL_BF16 || a.comp.fmt == HCL_FP8SPLIT);
+  if (a.mode == 1) return n_groups >= 32;
+  // CSA: the block's MMAs do G times the useful work; worth it while G <= 4
+  return a.H >= 32 && n_groups >= 32 && a.k >= 1 && a.idx != nullptr;
 }
 
 hcl_status_t launch_hca_flash(const AttnArgs& a, cudaStream_t st) {
   FaParams p;
+  p.mode = a.mode;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.B = a.B; p.Tq = a.Tq; p.H = a.H;
   p.G = std::min(std::max(1, FA_ROWS / a.H), a.Tq);
   p.n_groups = (a.Tq + p.G - 1) / p.G;
+  p.idx = a.idx;
+  p.k = a.mode == 0 ? a.k : 0;
   p.comp = a.comp; p.raw = a.raw;
-  p.Nh = a.n_comp; p.mh = a.mh; p.W = a.W;
+  p.Nh = a.n_comp; p.mh = a.mode == 1 ? a.mh : 1; p.W = a.W;
   p.q_pos = a.q_pos;
   p.scale_log2 = a.scale * FA_LOG2E;
   p.sink = a.sink;

@@ -313,6 +313,10 @@ def hcl_kv(data, scale=None, rope=None):
     (1, 3, 16, 700, 100, 37, False, False),     # ragged list, several queries
     (2, 2, 128, 3000, 64, 0, True, True),       # no window
     (1, 1, 128, 9000, 4096, 128, True, True),   # long list: splits merged via the workspace
+    # prefill chunks (>= 32 groups of 128 / H queries): the tcgen05 flash kernel, each query's
+    # own selection concatenated per block
+    (1, 80, 64, 3000, 256, 64, False, False),
+    (2, 130, 32, 2000, 100, 37, True, True),
 ])
 def test_csa_attn(hcl, B, Tq, H, Nc, k, W, fp8, sink):
     d, L = 128, 4 * Nc + 11
