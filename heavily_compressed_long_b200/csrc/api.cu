@@ -6,9 +6,10 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <algorithm>
+#include <map>
 #include <mutex>
-#include <set>
-#include <tuple>
+#include <utility>
 
 #include "hcl_common.cuh"
 #include "hcl_internal.h"
@@ -88,23 +89,38 @@ unsigned long long current_ctx_id() {
 }
 
 hcl_status_t set_kernel_attrs(const void* kern, int smem, bool nonportable_cluster) {
+  // The maximum dynamic shared memory is one value per kernel and context: it is only ever
+  // raised (a smaller later request must not lower the limit a larger launch relies on).
   static std::mutex mu;
-  static std::set<std::tuple<const void*, unsigned long long, int, bool>> done;
+  static std::map<std::pair<const void*, unsigned long long>, std::pair<int, bool>> done;
   const unsigned long long ctx = current_ctx_id();
   std::lock_guard<std::mutex> lock(mu);
-  if (ctx != 0 && done.count(std::make_tuple(kern, ctx, smem, nonportable_cluster))) return HCL_OK;
+  if (ctx != 0) {
+    auto it = done.find(std::make_pair(kern, ctx));
+    if (it != done.end() && it->second.first >= smem && (it->second.second || !nonportable_cluster))
+      return HCL_OK;
+  }
+  int want = smem;
+  bool cluster = nonportable_cluster;
+  if (ctx != 0) {
+    auto it = done.find(std::make_pair(kern, ctx));
+    if (it != done.end()) {
+      want = std::max(want, it->second.first);
+      cluster = cluster || it->second.second;
+    }
+  }
   hcl_status_t e = check_cuda(
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, want),
       "kernel shared-memory attribute");
   if (e != HCL_OK) return e;
-  if (nonportable_cluster) {
+  if (cluster) {
     e = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1),
                    "kernel cluster attribute");
     if (e != HCL_OK) return e;
   }
   // the attribute call makes a context current if none was; record under its id
   const unsigned long long now = current_ctx_id();
-  if (now != 0) done.insert(std::make_tuple(kern, now, smem, nonportable_cluster));
+  if (now != 0) done[std::make_pair(kern, now)] = std::make_pair(want, cluster);
   return HCL_OK;
 }
 

@@ -287,6 +287,13 @@ hcl_status_t launch_compress(const void* kv, const void* gate, const float* bias
                              int d, int m, int overlap, int e0, int e1, void* out, int out_fmt,
                              int out_cap, const float* gamma, float eps, cudaStream_t st) {
   if (e1 <= e0 || B == 0) return HCL_OK;
+  {
+    // an error left by an earlier runtime call would otherwise be reported as this launch's
+    const cudaError_t stale = cudaGetLastError();
+    if (stale != cudaSuccess)
+      return fail(HCL_ERR_CUDA, "compress: error pending before the launch: %s",
+                  cudaGetErrorString(stale));
+  }
   const int span = overlap ? 2 * m : m;
   const int G = d / 8;
   auto kvp = static_cast<const __nv_bfloat16*>(kv);
@@ -305,7 +312,11 @@ hcl_status_t launch_compress(const void* kv, const void* gate, const float* bias
     csa_compress_staged_kernel<<<grid, CS_THREADS, smem, st>>>(
         kvp, gp, bias, L, d, m, e0, e1, out, out_fmt, out_cap, gamma, eps, tiles_per_seq, n_tiles,
         stage_rows, wait_limit_cycles());
-    return check_launch("compress");
+    const cudaError_t le = cudaGetLastError();
+    if (le != cudaSuccess)
+      return fail(HCL_ERR_CUDA, "staged CSA compress launch (grid %d, %d threads, %d B shared): %s",
+                  grid, CS_THREADS, smem, cudaGetErrorString(le));
+    return HCL_OK;
   }
   if (!overlap && 128 % G == 0 && (size_t)4 * m * d * 2 + ((size_t)(128 / G) * 3 * d + 4) * 4 <= 200 * 1024) {
     // staged HCA path
@@ -320,7 +331,11 @@ hcl_status_t launch_compress(const void* kv, const void* gate, const float* bias
     hca_compress_staged_kernel<<<grid, 128, smem, st>>>(kvp, gp, bias, L, d, m, e0, e1, out,
                                                         out_fmt, out_cap, gamma, eps, n_tiles,
                                                         wait_limit_cycles());
-    return check_launch("compress");
+    const cudaError_t le = cudaGetLastError();
+    if (le != cudaSuccess)
+      return fail(HCL_ERR_CUDA, "staged HCA compress launch (grid %d, 128 threads, %d B shared): %s",
+                  grid, smem, cudaGetErrorString(le));
+    return HCL_OK;
   }
   if (span <= 16 || 128 % G != 0) {
     const long long threads = (long long)(e1 - e0) * B * G;

@@ -53,10 +53,11 @@ int num_sms();
 // reused within a process (a context created after cudaDeviceReset gets a new one), so they
 // key per-context caches safely, unlike device numbers or context handles.
 unsigned long long current_ctx_id();
-// Sets `kern`'s maximum dynamic shared memory to `smem` bytes (and, with nonportable_cluster,
-// allows cluster sizes above 8), once per (kernel, CUDA context, smem): function attributes
-// belong to a context, so every device -- and a context re-created after a reset -- gets its
-// own.  Thread-safe.
+// Makes `kern`'s maximum dynamic shared memory at least `smem` bytes (and, with
+// nonportable_cluster, allows cluster sizes above 8), per (kernel, CUDA context): function
+// attributes belong to a context, so every device -- and a context re-created after a reset --
+// gets its own.  The limit is only ever raised, so launches of one kernel with different
+// shared-memory sizes do not undo each other.  Thread-safe.
 hcl_status_t set_kernel_attrs(const void* kern, int smem, bool nonportable_cluster);
 // Bounded-wait budget for device spin loops, in SM clock cycles (about one second).
 long long wait_limit_cycles();
