@@ -444,8 +444,7 @@ int hcl_csa_decode_step_kernels(int B, int H, int HI, int Nc, int k, int W, int 
                                 int score_fmt, int kv_fmt) {
   (void)HI;
   if (B <= 0) return 0;
-  if (decode_uses_gmax(op_fmt, score_fmt, Nc) && hcl::select_attn_supported(Nc, H, k, W, kv_fmt))
-    return 2;  // indexer, then selection + attention
+  (void)op_fmt; (void)score_fmt; (void)Nc; (void)kv_fmt;
   const size_t ws = hcl::attn_workspace_bytes(0, B, 1, H, k, W);
   return 3 + (ws > 0 ? 1 : 0);  // indexer, top-k, attention (+ split merge)
 }
@@ -479,20 +478,6 @@ hcl_status_t hcl_csa_decode_step(const void* q, const void* qI_bf16, const float
                           kI_cap, q_pos, m, scores, score_fmt, status, stream);
   if (e != HCL_OK) return e;
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(wsb + l.idx);
-  if (gmax != nullptr && kvc != nullptr && raw != nullptr && kvc->fmt == raw->fmt &&
-      hcl::select_attn_supported(Nc, H, k, W, kvc->fmt) && d == 128) {
-    // selection and attention in one cluster kernel per sequence (it reads q, q_pos and the
-    // raw window before waiting for the indexer, which writes none of them)
-    e = check_kv(kvc, d, "kvc");
-    if (e != HCL_OK) return e;
-    e = check_kv(raw, d, "raw");
-    if (e != HCL_OK) return e;
-    HCL_REQUIRE(q && out && q_pos && aligned16(q) && aligned16(out), "q, out (16-byte aligned) and q_pos are required");
-    if (q_gamma != nullptr) HCL_REQUIRE(q_eps > 0.f && q_eps < 1e30f, "q_eps must be a positive number");
-    SelectAttnArgs sa{scores, gmax, g2nd, garg, B, Nc, q_pos, m, k, idx, q, H, *kvc, *raw, W,
-                      scale, sink, q_gamma, q_eps, out, lse, status};
-    return launch_select_attn(sa, as_stream(stream));
-  }
   // the top-k's predecessor is the indexer above, which does not write q_pos
   if (gmax != nullptr) {
     HCL_REQUIRE(k >= 1 && k <= 4096, "k must be in [1, 4096]");

@@ -126,33 +126,6 @@ bool topk_gmax_supported(int Nc);
 hcl_status_t launch_topk_gmax(const TopkArgs& a, const uint16_t* gmax, const uint16_t* g2nd,
                               const uint8_t* garg, cudaStream_t st);
 
-// Fused decode selection + attention (MXFP4 keys, bf16 scores with the indexer's group
-// summaries): one cluster of CTAs per sequence selects the top-k from the summaries and
-// attends over its share of the selected entries and the window.
-struct SelectAttnArgs {
-  const void* scores;        // bf16 [B, Nc]
-  const uint16_t* gmax;      // [B, gmax_row_stride(Nc)]
-  const uint16_t* g2nd;
-  const uint8_t* garg;
-  int B, Nc;
-  const int32_t* q_pos;
-  int m, k;
-  int32_t* idx;              // [B, k]
-  const void* q;             // bf16 [B, H, 128]
-  int H;
-  hcl_kv_t comp, raw;
-  int W;
-  float scale;
-  const float* sink;
-  const float* q_gamma;
-  float q_eps;
-  void* out;
-  float* lse;
-  int32_t* status;
-};
-bool select_attn_supported(int Nc, int H, int k, int W, int comp_fmt);
-hcl_status_t launch_select_attn(const SelectAttnArgs& a, cudaStream_t st);
-
 // One attention launch: CSA (selected entries + window) or HCA (visible entries + window).
 struct AttnArgs {
   int mode;  // 0 = CSA, 1 = HCA

@@ -232,9 +232,7 @@ HCL_API hcl_status_t hcl_hca_dense_attn(const void* q, int B, int Tq, int H, int
  * Fused CSA decode step [Tripbot §3.1]: for each sequence, the new query's index queries are
  * quantised (MXFP4 operands only), scored against all entries, the top-k kept, and
  * attention run over them plus the window -- a4 -> a5 -> a6 enqueued back to back on
- * `stream`; with MXFP4 keys and bf16 scores a5 and a6 run as one kernel (a cluster per
- * sequence selects from the indexer's group summaries and attends over its share of the
- * selection), whose selection equals hcl_csa_topk's bit for bit.  Arguments as in the individual calls; qI_bf16 is the unquantised bf16 index
+ * `stream`.  Arguments as in the individual calls; qI_bf16 is the unquantised bf16 index
  * query [B, 1, HI, dI]; Tq == 1.  ws: hcl_csa_decode_step_workspace_bytes() bytes; it holds
  * the scores and, with MXFP4 operands and bf16 scores, a 5-byte summary per 16-entry group
  * (largest and second largest score as order-preserving keys, position of the largest) that
@@ -244,9 +242,8 @@ HCL_API hcl_status_t hcl_hca_dense_attn(const void* q, int B, int Tq, int H, int
 HCL_API size_t hcl_csa_decode_step_workspace_bytes(int B, int H, int HI, int Nc, int k, int W,
                                            int op_fmt, int score_fmt);
 /* The number of kernels one hcl_csa_decode_step call with these shapes and formats launches
- * (kv_fmt: the compressed / raw store format): 2 with MXFP4 keys and bf16 scores (the indexer,
- * then selection and attention in one cluster kernel per sequence), otherwise 3 or 4 (indexer,
- * top-k, attention, and a split merge when the attention needs a workspace). */
+ * (kv_fmt: the compressed / raw store format): the indexer, the top-k, the attention, and a
+ * split merge when the attention needs a workspace. */
 HCL_API int hcl_csa_decode_step_kernels(int B, int H, int HI, int Nc, int k, int W, int op_fmt,
                                         int score_fmt, int kv_fmt);
 HCL_API hcl_status_t hcl_csa_decode_step(const void* q, const void* qI_bf16, const float* w, int op_fmt,
