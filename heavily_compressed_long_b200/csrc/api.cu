@@ -203,10 +203,10 @@ static hcl_status_t compress_common(const void* kv, const void* gate, const floa
   HCL_REQUIRE(out_fmt == HCL_FP32 || out_fmt == HCL_BF16, "out_fmt must be HCL_FP32 or HCL_BF16");
   if (gamma != nullptr) {
     HCL_REQUIRE(eps > 0.f && eps < 1e30f, "eps must be a positive number");
-    // the RMSNorm reduction runs over the d/8 threads of an entry (a power of two <= 32) or
-    // over a 128-thread block (long spans)
+    // the RMSNorm reduction runs over the d/8 threads of an entry (a power of two <= 32) or,
+    // for HCA with d/8 dividing 256, over a block
     const int G = d / 8;
-    const bool small = (overlap ? 2 * m : m) <= 16 || 128 % G != 0;
+    const bool small = overlap || 256 % G != 0;
     if (small && (G > 32 || (G & (G - 1)) != 0))
       return fail(HCL_ERR_UNSUPPORTED, "RMSNorm epilogue needs d/8 a power of two <= 32 (d=%d)", d);
   }

@@ -10,13 +10,16 @@
 // queries x H heads = up to 128 (query, head) rows = the UMMA M dimension = 128 TMEM lanes, two
 // threads per row.  The group's KV list is the visible-entry prefix of its last query followed
 // by the union of its queries' windows; it is processed in rounds of two 64-row chunks gathered
-// with cp.async (split FP8 rows widened to bf16 with their scale).  Per round S = Q K^T (N = 64
-// per chunk) and O = P V (V read as the MN-major operand of the same SW128 tile) accumulate in
-// TMEM; the softmax runs in registers with each row's own causal mask (for query q: the list
-// rows [0, visible entries of q) and the window rows of q -- two index intervals, turned into
-// bit masks), online across rounds: O of a round is added to the register accumulator after
-// rescaling by the change of the running maximum.  Two blocks fit per SM (about 106 KB of
-// shared memory, 256 TMEM columns each), so one block's gather overlaps the other's MMAs.
+// with cp.async (split FP8 rows widened to bf16 with their scale; each row's store slot is
+// resolved once per round, not per 16-byte piece).  Per round S = Q K^T (N = 64 per chunk) lands
+// in TMEM and O += P V (V read as the MN-major operand of the same SW128 tile) accumulates in
+// TMEM across all rounds; the softmax runs in registers (S read from TMEM once) with each row's
+// own causal mask (for query q: the list rows [0, visible entries of q) and the window rows of
+// q -- two index intervals, turned into bit masks).  The probabilities of a round are taken
+// against a reference maximum that is raised only when the row maximum grows by more than 2^8;
+// only then is O rescaled in TMEM (load, scale, store), so most rounds leave O untouched.  Two
+// blocks fit per SM (about 109 KB of shared memory, 256 TMEM columns each), so one block's
+// gather overlaps the other's MMAs.
 //
 // CSA prefill (every query has its own selection) uses the same kernel with G = 128 / H
 // queries per block (2 at H = 64): the KV list is the concatenation of the G queries' lists
@@ -68,8 +71,19 @@ struct FaOff {
   static constexpr uint32_t SCL = STG + FA_RCH * 4096;
   static constexpr uint32_t XCH = SCL + FA_RCH * 256;
   static constexpr uint32_t BAR = XCH + 2 * FA_THREADS * 4;
-  static constexpr uint32_t TOTAL = BAR + 64;
+  static constexpr uint32_t RS = BAR + 64;                       // FA_RCH * FA_CH row sources
+  static constexpr uint32_t TOTAL = RS + FA_RCH * FA_CH * 16;
 };
+
+struct FaRow {
+  long long slot;   // row slot in its store (-1: no row)
+  int from_raw;
+  int pad;
+};
+
+// Rescale O only when the running maximum grows by more than this (log2 units): until then the
+// probabilities are taken against the stale maximum (values <= 2^8, exact in fp32 sums).
+constexpr float FA_RESCALE_LOG2 = 8.f;
 
 __device__ __forceinline__ uint32_t fa_pack(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -195,9 +209,7 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
   const uint32_t tbase = *sTmem;
   const uint32_t ocol = FA_RCH * FA_CH;
   const uint32_t trow = tbase + (uint32_t((warp & 3) * 32) << 16);
-  float o_acc[64];
-#pragma unroll
-  for (int i = 0; i < 64; i++) o_acc[i] = 0.f;
+  FaRow* rsrc = reinterpret_cast<FaRow*>(sm + FaOff::RS);
   float m_run = -INFINITY, l_run = 0.f;
   bool ok = true;
   const int nrounds = (total + FA_RCH * FA_CH - 1) / (FA_RCH * FA_CH);
@@ -205,73 +217,68 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
     const int r0 = rd * FA_RCH * FA_CH;
     const int nr = min(FA_RCH * FA_CH, total - r0);
     const int nch = (nr + FA_CH - 1) / FA_CH;
-    // gather: list row r0 + jj -> KV row jj (rows past nr: zeros)
-    constexpr int PIECES = KVFMT == HCL_BF16 ? 16 : 13;
-    for (int u = tid; u < nch * FA_CH * PIECES; u += FA_THREADS) {
-      const int jj = u / PIECES, pc = u % PIECES;
-      const int ch = jj / FA_CH, r = jj % FA_CH;
-      const int e = r0 + jj;
-      long long slot = -1;
-      const hcl_kv_t* st = &p.comp;
+    // resolve list row r0 + jj (jj = tid < 128, whole warps 0..3) to its store slot once
+    if (tid < FA_RCH * FA_CH) {
+      const int jj = tid, e = r0 + jj;
+      FaRow rs{-1, 0, 0};
       if (jj < nr) {
         if (p.mode == 1) {
           if (e < n_a) {
-            slot = (long long)b * p.comp.cap + (e % p.comp.cap);
+            rs.slot = (long long)b * p.comp.cap + (e % p.comp.cap);
           } else {
-            const long long tok = (long long)raw_lo + (e - n_a);
-            if (tok >= 0) { st = &p.raw; slot = (long long)b * p.raw.cap + tok % p.raw.cap; }
+            const int tok = raw_lo + (e - n_a);
+            if (tok >= 0) { rs.slot = (long long)b * p.raw.cap + tok % p.raw.cap; rs.from_raw = 1; }
           }
         } else {
-          const int sq = e / seg, se = e % seg;
+          const int sq = e / seg, se = e - sq * seg;
           if (se < p.k) {
             const int ent = p.idx[((size_t)b * p.Tq + t0 + sq) * p.k + se];
-            if (ent >= 0 && ent < p.Nh) slot = (long long)b * p.comp.cap + (ent % p.comp.cap);
+            if (ent >= 0 && ent < p.Nh) rs.slot = (long long)b * p.comp.cap + (ent % p.comp.cap);
             else if (ent >= p.Nh || ent < -1) report(p.status, HCL_ERR_DEVICE_FAULT);
           } else {
-            const long long tok = (long long)p.q_pos[(size_t)b * p.Tq + t0 + sq] - p.W + 1 + (se - p.k);
-            if (tok >= 0) { st = &p.raw; slot = (long long)b * p.raw.cap + tok % p.raw.cap; }
+            const int tok = p.q_pos[(size_t)b * p.Tq + t0 + sq] - p.W + 1 + (se - p.k);
+            if (tok >= 0) { rs.slot = (long long)b * p.raw.cap + tok % p.raw.cap; rs.from_raw = 1; }
           }
         }
       }
+      rsrc[jj] = rs;
+      if (p.mode == 0) {
+        // valid list rows of the round (a selected entry, or a window token >= 0)
+        const uint32_t bits = __ballot_sync(0xffffffffu, rs.slot >= 0);
+        if ((tid & 31) == 0) rbits[tid >> 5] = bits;
+      }
+    }
+    __syncthreads();
+    // gather: list row r0 + jj -> KV row jj (rows past nr: zeros)
+    constexpr int PIECES = KVFMT == HCL_BF16 ? 16 : 13;
+    for (int u = tid; u < nch * FA_CH * PIECES; u += FA_THREADS) {
+      const int jj = u / PIECES, pc = u - jj * PIECES;
+      const int ch = jj / FA_CH, r = jj % FA_CH;
+      const FaRow rs = rsrc[jj];
+      const hcl_kv_t& st = rs.from_raw ? p.raw : p.comp;
       uint8_t* kv = sm + FaOff::KV + ch * 16384;
       if (KVFMT == HCL_BF16) {
         uint8_t* dst = kv + (pc >> 3) * 8192 + r * 128 + (((pc & 7) ^ (r & 7)) << 4);
-        if (slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st->data) + slot * 256 + pc * 16);
+        if (rs.slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.data) + rs.slot * 256 + pc * 16);
         else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
       } else if (pc < 8) {
         uint8_t* dst = kv + 8192 + r * 128 + ((pc ^ (r & 7)) << 4);
-        if (slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st->rope) + slot * 128 + pc * 16);
+        if (rs.slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.rope) + rs.slot * 128 + pc * 16);
         else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
       } else if (pc < 12) {
         uint8_t* dst = sm + FaOff::STG + (ch * FA_CH + r) * 64 + (pc - 8) * 16;
-        if (slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st->data) + slot * 64 + (pc - 8) * 16);
+        if (rs.slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.data) + rs.slot * 64 + (pc - 8) * 16);
         else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
       } else {
         float* dst = reinterpret_cast<float*>(sm + FaOff::SCL) + ch * FA_CH + r;
-        if (slot >= 0)
+        if (rs.slot >= 0)
           asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)),
-                       "l"(st->scale + slot)
+                       "l"(st.scale + rs.slot)
                        : "memory");
         else *dst = 0.f;
       }
     }
     cp_async_commit();
-    if (p.mode == 0) {
-      // valid list rows of the round (a selected entry, or a window token >= 0)
-      const int jj = tid;
-      bool v = false;
-      if (jj < nr) {
-        const int e = r0 + jj, sq = e / seg, se = e % seg;
-        if (se < p.k) {
-          const int ent = p.idx[((size_t)b * p.Tq + t0 + sq) * p.k + se];
-          v = ent >= 0 && ent < p.Nh;
-        } else {
-          v = (long long)p.q_pos[(size_t)b * p.Tq + t0 + sq] - p.W + 1 + (se - p.k) >= 0;
-        }
-      }
-      const uint32_t bits = __ballot_sync(0xffffffffu, v);
-      if ((tid & 31) == 0 && tid < FA_RCH * FA_CH) rbits[tid >> 5] = bits;
-    }
     cp_async_wait<0>();
     __syncthreads();
     if (KVFMT == HCL_FP8SPLIT) {
@@ -307,10 +314,16 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
     __syncwarp();   // warp 0 reconverges before waiting (the issuing lane is not left behind)
     ok = ok && mbar_wait(bar_s, rd & 1, p.limit, nullptr);
     tc_fence_after();
-    // two passes over this thread's 32 columns of each chunk: maximum, then exponentials
-    // (the columns are read from TMEM twice instead of being held in registers)
+    // this thread's 32 columns of each chunk, held in registers for both softmax passes
     uint32_t vb[FA_RCH];
+    uint32_t sv[FA_RCH][32];
     float lmax = -INFINITY;
+#pragma unroll
+    for (int ch = 0; ch < FA_RCH; ch++) {
+      tmem_ld16(trow + ch * FA_CH + hc * 32, *reinterpret_cast<uint32_t(*)[16]>(&sv[ch][0]));
+      tmem_ld16(trow + ch * FA_CH + hc * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[ch][16]));
+    }
+    tmem_ld_wait();
 #pragma unroll
     for (int ch = 0; ch < FA_RCH; ch++) {
       vb[ch] = 0u;
@@ -320,44 +333,55 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
                  range_bits(c0, r0, r0 + nr);
         if (p.mode == 0) vb[ch] &= rbits[2 * ch + hc];
       }
-      if (ch < nch) {
-        uint32_t sv[32];
-        tmem_ld16(trow + ch * FA_CH + hc * 32, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
-        tmem_ld16(trow + ch * FA_CH + hc * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
-        tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; j++)
-          if ((vb[ch] >> j) & 1u) lmax = fmaxf(lmax, __uint_as_float(sv[j]) * p.scale_log2);
-      }
+      for (int j = 0; j < 32; j++)
+        if ((vb[ch] >> j) & 1u) lmax = fmaxf(lmax, __uint_as_float(sv[ch][j]) * p.scale_log2);
     }
     xch[tid] = lmax;
     __syncthreads();
-    const float m_new = fmaxf(m_run, fmaxf(xch[row], xch[row + FA_ROWS]));
+    const float m_cand = fmaxf(m_run, fmaxf(xch[row], xch[row + FA_ROWS]));
+    // the same decision in both threads of a row: a new reference maximum only when it grew by
+    // more than FA_RESCALE_LOG2 (or is the first finite one)
+    const bool grow = m_cand > m_run + FA_RESCALE_LOG2;
+    const float m_new = grow ? m_cand : m_run;
+    const float alpha = (grow && m_run > -INFINITY) ? exp2f(m_run - m_new) : 1.f;
     const float muse = m_new == -INFINITY ? 0.f : m_new;
     float lsum = 0.f;
 #pragma unroll
-    for (int ch = 0; ch < FA_RCH; ch++)
-      if (ch < nch) {
-        uint32_t sv[32];
-        tmem_ld16(trow + ch * FA_CH + hc * 32, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
-        tmem_ld16(trow + ch * FA_CH + hc * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
-        tmem_ld_wait();
-        uint8_t* prow = sm + FaOff::P + ch * 16384 + row * 128;
+    for (int ch = 0; ch < FA_RCH; ch++) {
+      uint8_t* prow = sm + FaOff::P + ch * 16384 + row * 128;
 #pragma unroll
-        for (int q4 = 0; q4 < 4; q4++) {
-          uint32_t pk[4];
+      for (int q4 = 0; q4 < 4; q4++) {
+        uint32_t pk[4];
 #pragma unroll
-          for (int i = 0; i < 8; i += 2) {
-            const int j = q4 * 8 + i;
-            const float p0 = ((vb[ch] >> j) & 1u) ? exp2f(__uint_as_float(sv[j]) * p.scale_log2 - muse) : 0.f;
-            const float p1 = ((vb[ch] >> (j + 1)) & 1u) ? exp2f(__uint_as_float(sv[j + 1]) * p.scale_log2 - muse) : 0.f;
-            lsum += p0 + p1;
-            pk[i >> 1] = fa_pack(p0, p1);
-          }
+        for (int i = 0; i < 8; i += 2) {
+          const int j = q4 * 8 + i;
+          const float p0 = ((vb[ch] >> j) & 1u) ? exp2f(__uint_as_float(sv[ch][j]) * p.scale_log2 - muse) : 0.f;
+          const float p1 = ((vb[ch] >> (j + 1)) & 1u) ? exp2f(__uint_as_float(sv[ch][j + 1]) * p.scale_log2 - muse) : 0.f;
+          lsum += p0 + p1;
+          pk[i >> 1] = fa_pack(p0, p1);
+        }
+        if (ch < nch)
           *reinterpret_cast<uint4*>(prow + (((hc * 4 + q4) ^ (row & 7)) << 4)) =
               make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        }
       }
+    }
+    // O (complete: the previous round's PV was waited for) rescaled in TMEM where the reference
+    // maximum moved; warp-uniform (TMEM loads and stores are warp-collective)
+    if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+      for (int q4 = 0; q4 < 4; q4++) {
+        uint32_t r16[16];
+        tmem_ld16(trow + ocol + hc * 64 + q4 * 16, r16);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; i++) r16[i] = __float_as_uint(__uint_as_float(r16[i]) * alpha);
+        tmem_st16(trow + ocol + hc * 64 + q4 * 16, r16);
+      }
+      tmem_st_wait();
+    }
+    l_run = l_run * alpha + lsum;
+    m_run = m_new;
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -370,29 +394,13 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
         for (int ks = 0; ks < 4; ks++)
           umma_bf16(tbase + ocol, make_sdesc(ap + ks * 32, 16, 1024, SMEM_SWIZZLE_128B),
                     make_sdesc(av + ks * 2048, 8192, 1024, SMEM_SWIZZLE_128B),
-                    idesc_bf16(128, FA_D) | (1u << 16), (ch > 0 || ks > 0) ? 1u : 0u);
+                    idesc_bf16(128, FA_D) | (1u << 16), (rd > 0 || ch > 0 || ks > 0) ? 1u : 0u);
       }
       umma_commit(bar_o);
     }
     __syncwarp();
-    ok = ok && mbar_wait(bar_o, rd & 1, p.limit, nullptr);
+    ok = ok && mbar_wait(bar_o, rd & 1, p.limit, nullptr);   // KV, P and O free again
     tc_fence_after();
-    {
-      const float alpha = m_run == -INFINITY ? 0.f : exp2f(m_run - m_new);
-#pragma unroll
-      for (int q4 = 0; q4 < 4; q4++) {
-        uint32_t r16[16];
-        tmem_ld16(trow + ocol + hc * 64 + q4 * 16, r16);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 16; i++)
-          o_acc[q4 * 16 + i] = o_acc[q4 * 16 + i] * alpha + __uint_as_float(r16[i]);
-      }
-      l_run = l_run * alpha + lsum;
-      m_run = m_new;
-    }
-    tc_fence_before();
-    __syncthreads();
   }
   if (!ok) report(p.status, HCL_ERR_TIMEOUT);
   xch[FA_THREADS + tid] = l_run;
@@ -409,16 +417,29 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
     l2 = l3;
     m2 = mm;
   }
-  if (rv) {
-    const size_t orow = ((size_t)b * p.Tq + t0 + qi) * p.H + hh;
-    __nv_bfloat16* dst = p.out + orow * FA_D + hc * 64;
+  const bool have_o = nrounds > 0;   // else O was never written
+  const size_t orow = ((size_t)b * p.Tq + t0 + qi) * p.H + hh;
 #pragma unroll
-    for (int i = 0; i < 64; i += 8)
-      *reinterpret_cast<uint4*>(dst + i) =
-          make_uint4(fa_pack(o_acc[i] * f, o_acc[i + 1] * f), fa_pack(o_acc[i + 2] * f, o_acc[i + 3] * f),
-                     fa_pack(o_acc[i + 4] * f, o_acc[i + 5] * f), fa_pack(o_acc[i + 6] * f, o_acc[i + 7] * f));
-    if (hc == 0 && p.lse) p.lse[orow] = l2 > 0.f ? (m2 + log2f(l2)) * FA_LN2 : -INFINITY;
+  for (int q4 = 0; q4 < 4; q4++) {
+    uint32_t r16[16];
+    tmem_ld16(trow + ocol + hc * 64 + q4 * 16, r16);
+    tmem_ld_wait();
+    if (!have_o) {
+#pragma unroll
+      for (int i = 0; i < 16; i++) r16[i] = 0u;
+    }
+    if (rv) {
+      __nv_bfloat16* dst = p.out + orow * FA_D + hc * 64 + q4 * 16;
+#pragma unroll
+      for (int i = 0; i < 16; i += 8)
+        *reinterpret_cast<uint4*>(dst + i) = make_uint4(
+            fa_pack(__uint_as_float(r16[i]) * f, __uint_as_float(r16[i + 1]) * f),
+            fa_pack(__uint_as_float(r16[i + 2]) * f, __uint_as_float(r16[i + 3]) * f),
+            fa_pack(__uint_as_float(r16[i + 4]) * f, __uint_as_float(r16[i + 5]) * f),
+            fa_pack(__uint_as_float(r16[i + 6]) * f, __uint_as_float(r16[i + 7]) * f));
+    }
   }
+  if (rv && hc == 0 && p.lse) p.lse[orow] = l2 > 0.f ? (m2 + log2f(l2)) * FA_LN2 : -INFINITY;
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {

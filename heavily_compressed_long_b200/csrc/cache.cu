@@ -95,7 +95,8 @@ __device__ __forceinline__ uint4 pack8_bf16(const float (&v)[8]) {
 }
 
 __global__ void __launch_bounds__(AP_THREADS) cache_append_kernel(AppendParams p) {
-  __shared__ float sm[8 * 3 * AP_D + 4];   // pool_long_block: 8 slot streams x 3 x d, + 4
+  __shared__ float part[3 * 2048];         // stream partials [NS][3][d] (pool.cuh), NS * d = 2048
+  __shared__ float red[4];
   __shared__ float amax2[2];
   pdl_enter();
   const int b = blockIdx.x;
@@ -137,8 +138,7 @@ __global__ void __launch_bounds__(AP_THREADS) cache_append_kernel(AppendParams p
         return staged(t + 1 - span + j, kp, gp);
       };
       if (lane < 16) {
-        if (span == 8) pool8_span<8, false>(row, p.bias_csa, lane, v);
-        else pool8_any<false>(row, p.bias_csa, span, lane, v);
+        pool8_any<false>(row, p.bias_csa, span, lane, v);
         if (p.gamma != nullptr) rmsnorm8_group(v, 16, AP_D, lane, p.gamma, p.eps);
       }
       uint4 pk = make_uint4(0, 0, 0, 0);
@@ -169,8 +169,14 @@ __global__ void __launch_bounds__(AP_THREADS) cache_append_kernel(AppendParams p
     auto row = [&](int j, const __nv_bfloat16*& kp, const __nv_bfloat16*& gp) {
       return staged(t + 1 - p.mh + j, kp, gp);
     };
+    // the batch compressor's 256 threads as 128: thread t takes streams t / 16 and t / 16 + 8
+    constexpr int NS = pool_streams(AP_D), G = AP_D / 8;
+    static_assert(NS * G == 2 * AP_THREADS, "two slot streams per thread");
+    pool_stream_partial<false>(row, p.bias_hca, p.mh, AP_D, tid / G, tid % G, part);
+    pool_stream_partial<false>(row, p.bias_hca, p.mh, AP_D, tid / G + NS / 2, tid % G, part);
+    __syncthreads();
     float vals[8];
-    pool_long_block<false>(row, p.bias_hca, p.mh, AP_D, sm, p.gamma, p.eps, vals);
+    pool_merge_streams(part, AP_D, red, p.gamma, p.eps, vals);
     // thread c holds channel c; round to bf16 as the batch compressor's bf16 output does
     const __nv_bfloat16 xb = __float2bfloat16_rn(vals[0]);
     const long long slot = (long long)b * p.kvh.cap + i % p.kvh.cap;
