@@ -649,7 +649,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
   const int b = blockIdx.x / p.splits;
   const TcOff off = tc_offsets(p.cps, p.splits);
   uint8_t* sQ = sm + off.q;
-  RowSrc* rsrc = reinterpret_cast<RowSrc*>(sm + off.rs);
   uint64_t* bar_s = reinterpret_cast<uint64_t*>(sm + off.bar);
   uint64_t* bar_o = bar_s + 1;
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + off.bar + 16);
@@ -721,63 +720,69 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
   }
   if (early_ok && !early) pdl_enter();
 
-  // rows of the split: resolve, then gather (rope half / bf16 rows straight into the SW128
-  // tile with cp.async, E4M3 codes and scales into staging)
+  // rows of the split: two threads per row resolve the row's store slot and copy their halves
+  // of its 16-byte pieces (rope half / bf16 rows straight into the SW128 tile with cp.async,
+  // E4M3 codes and scales into staging); a warp's ballot gives the validity bits of its 16 rows
   const int nrows = nch * KVB;
-  for (int jj = tid; jj < nrows; jj += TC_THREADS) {
+  for (int j0 = 0; j0 < nrows; j0 += TC_THREADS / 2) {
+    const int jj = j0 + (tid >> 1), half = tid & 1;
     const int e = c_begin * KVB + jj;
-    RowSrc rs{-1, 0};
-    if (e < n_a) {
-      long long ent = p.idx[(size_t)b * p.k + e];
-      if (ent < -1 || ent >= p.n_comp) {
-        report(p.status, HCL_ERR_DEVICE_FAULT);
-        ent = -1;
+    long long slot = -1;
+    bool from_raw = false;
+    if (jj < nrows) {
+      if (e < n_a) {
+        long long ent = p.idx[(size_t)b * p.k + e];
+        if (ent < -1 || ent >= p.n_comp) {
+          if (half == 0) report(p.status, HCL_ERR_DEVICE_FAULT);
+          ent = -1;
+        }
+        if (ent >= 0) slot = (long long)b * p.comp.cap + (ent % p.comp.cap);
+      } else if (e < total) {
+        const long long u = (long long)raw_lo + (e - n_a);
+        if (u >= 0) { slot = (long long)b * p.raw.cap + (u % p.raw.cap); from_raw = true; }
       }
-      if (ent >= 0) rs.slot = (long long)b * p.comp.cap + (ent % p.comp.cap);
-    } else if (e < total) {
-      const long long u = (long long)raw_lo + (e - n_a);
-      if (u >= 0) { rs.slot = (long long)b * p.raw.cap + (u % p.raw.cap); rs.from_raw = 1; }
     }
-    rsrc[jj] = rs;
-  }
-  __syncthreads();
-  // one bit per row of the split (row j of chunk c: word 2c + j/32, bit j%32)
-  for (int w0 = 0; w0 < nrows; w0 += TC_THREADS) {
-    const int jj = w0 + tid;
-    const uint32_t bits = __ballot_sync(0xffffffffu, jj < nrows && rsrc[jj].slot >= 0);
-    if (lane == 0 && jj < nrows) visw[jj >> 5] = bits;
-  }
-  {
-    constexpr int PIECES = KVFMT == HCL_BF16 ? 16 : 13;
-    for (int u = tid; u < nrows * PIECES; u += TC_THREADS) {
-      const int jj = u / PIECES, c = u % PIECES;
-      const int ch = jj / KVB, r = jj % KVB;
-      const RowSrc rs = rsrc[jj];
-      const hcl_kv_t& st = rs.from_raw ? p.raw : p.comp;
-      uint8_t* kv = sm + off.kv + ch * 16384;
-      if (KVFMT == HCL_BF16) {
+    const uint32_t bal = __ballot_sync(0xffffffffu, slot >= 0);
+    uint32_t bits16 = 0;
+#pragma unroll
+    for (int i = 0; i < 16; i++) bits16 |= ((bal >> (2 * i)) & 1u) << i;
+    if (lane == 0 && j0 + 16 * warp < nrows)
+      reinterpret_cast<uint16_t*>(visw)[(j0 >> 4) + warp] = uint16_t(bits16);
+    if (jj >= nrows) continue;
+    const int ch = jj / KVB, r = jj % KVB;
+    const hcl_kv_t& st = from_raw ? p.raw : p.comp;
+    uint8_t* kv = sm + off.kv + ch * 16384;
+    if (KVFMT == HCL_BF16) {
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        const int c = half * 8 + i;
         uint8_t* dst = kv + (c >> 3) * 8192 + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-        if (rs.slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.data) + rs.slot * 256 + c * 16);
+        if (slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.data) + slot * 256 + c * 16);
         else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-      } else if (c < 8) {          // RoPE dims 64..127: the second half, as stored
-        uint8_t* dst = kv + 8192 + r * 128 + ((c ^ (r & 7)) << 4);
-        if (rs.slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.rope) + rs.slot * 128 + c * 16);
-        else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-      } else if (c < 12) {         // E4M3 codes of dims 0..63
-        uint8_t* dst = sm + off.stg + (ch * KVB + r) * 64 + (c - 8) * 16;
-        if (rs.slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.data) + rs.slot * 64 + (c - 8) * 16);
-        else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-      } else {
-        float* dst = reinterpret_cast<float*>(sm + off.scl) + ch * KVB + r;
-        if (rs.slot >= 0)
-          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)),
-                       "l"(st.scale + rs.slot)
-                       : "memory");
-        else *dst = 0.f;
       }
+    } else if (half == 0) {        // RoPE dims 64..127: the second half, as stored
+#pragma unroll
+      for (int c = 0; c < 8; c++) {
+        uint8_t* dst = kv + 8192 + r * 128 + ((c ^ (r & 7)) << 4);
+        if (slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.rope) + slot * 128 + c * 16);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+      }
+    } else {                       // E4M3 codes of dims 0..63 and the row scale
+#pragma unroll
+      for (int c = 0; c < 4; c++) {
+        uint8_t* dst = sm + off.stg + (ch * KVB + r) * 64 + c * 16;
+        if (slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.data) + slot * 64 + c * 16);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+      }
+      float* dst = reinterpret_cast<float*>(sm + off.scl) + ch * KVB + r;
+      if (slot >= 0)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)),
+                     "l"(st.scale + slot)
+                     : "memory");
+      else *dst = 0.f;
     }
-    cp_async_commit();
   }
+  cp_async_commit();
   if (early) pdl_enter();
   cp_async_wait<0>();
   __syncthreads();
@@ -922,8 +927,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
   const float inv_l = l2 > 0.f ? 1.f / l2 : 0.f;
   float* pdst = nullptr;
   if (p.splits > 1) {
+    // row r is merged by block r / rpo (contiguous head blocks: a warp's stores reach one or
+    // two blocks), in its slot r % rpo
     cg::cluster_group cluster = cg::this_cluster();
-    const int owner = row % p.splits, slot = row / p.splits;
+    const int rpo = (TC_ROWS + p.splits - 1) / p.splits;
+    const int owner = row / rpo, slot = row % rpo;
     pdst = cluster.map_shared_rank(recv, owner) + ((size_t)slot * p.splits + split) * D + hc * 64;
     if (hv && hc == 0)
       *(cluster.map_shared_rank(recv_lse, owner) + slot * p.splits + split) =
@@ -974,13 +982,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
     tmem_dealloc(tbase, ncols);
   }
   if (p.splits > 1) {
-    // merge the rows this block owns (row r -> block r % splits, slot r / splits)
+    // merge the rows this block owns (row r -> block r / rpo, slot r % rpo)
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();
     const int S = p.splits;
     const int rpo = (TC_ROWS + S - 1) / S;
     for (int slot = warp; slot < rpo; slot += TC_THREADS / 32) {
-      const int h = split + S * slot;
+      const int h = split * rpo + slot;
       if (h >= p.H) break;
       const float ls = lane < S ? recv_lse[slot * S + lane] : -INFINITY;
       float M = ls;

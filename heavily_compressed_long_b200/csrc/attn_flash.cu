@@ -9,17 +9,18 @@
 // Design (B200): one block of 256 threads per query group: G = floor(128 / H) consecutive
 // queries x H heads = up to 128 (query, head) rows = the UMMA M dimension = 128 TMEM lanes, two
 // threads per row.  The group's KV list is the visible-entry prefix of its last query followed
-// by the union of its queries' windows; it is processed in rounds of two 64-row chunks gathered
-// with cp.async (split FP8 rows widened to bf16 with their scale; each row's store slot is
-// resolved once per round, not per 16-byte piece).  Per round S = Q K^T (N = 64 per chunk) lands
-// in TMEM and O += P V (V read as the MN-major operand of the same SW128 tile) accumulates in
-// TMEM across all rounds; the softmax runs in registers (S read from TMEM once) with each row's
-// own causal mask (for query q: the list rows [0, visible entries of q) and the window rows of
-// q -- two index intervals, turned into bit masks).  The probabilities of a round are taken
-// against a reference maximum that is raised only when the row maximum grows by more than 2^8;
-// only then is O rescaled in TMEM (load, scale, store), so most rounds leave O untouched.  Two
-// blocks fit per SM (about 109 KB of shared memory, 256 TMEM columns each), so one block's
-// gather overlaps the other's MMAs.
+// by the union of its queries' windows; it is processed in rounds of 64 rows.  A round's rows
+// are gathered with cp.async into one of two KV buffers (4 threads per row, each resolving the
+// row's store slot; split FP8 rows widened to bf16 with their scale), so the gather of round
+// r + 1 is in flight while round r runs S = Q K^T (N = 64) into TMEM, its softmax and
+// O += P V (V read as the MN-major operand of the same SW128 tile; O accumulates in TMEM
+// across all rounds).  The softmax runs in registers with each row's own causal mask (for
+// query q: the list rows [0, visible entries of q) and the window rows of q -- two index
+// intervals, turned into bit masks; full 32-column words skip the per-column selects), its
+// probabilities taken against a reference maximum that is raised only when the row maximum
+// grows by more than 2^8, and only then is O rescaled in TMEM (load, scale, store).  Paired
+// fp32 instructions form the exponents and sums.  Two blocks fit per SM (about 92 KB of
+// shared memory, 256 TMEM columns each), so one block's softmax overlaps the other's MMAs.
 //
 // CSA prefill (every query has its own selection) uses the same kernel with G = 128 / H
 // queries per block (2 at H = 64): the KV list is the concatenation of the G queries' lists
@@ -39,8 +40,7 @@ namespace {
 constexpr int FA_THREADS = 256;
 constexpr int FA_ROWS = 128;
 constexpr int FA_D = 128;
-constexpr int FA_CH = 64;
-constexpr int FA_RCH = 2;
+constexpr int FA_CH = 64;        // list rows per round
 constexpr float FA_LOG2E = 1.4426950408889634f;
 constexpr float FA_LN2 = 0.6931471805599453f;
 
@@ -64,21 +64,14 @@ struct FaParams {
 };
 
 struct FaOff {
-  static constexpr uint32_t Q = 0;
-  static constexpr uint32_t KV = 32768;
-  static constexpr uint32_t P = KV + FA_RCH * 16384;
-  static constexpr uint32_t STG = P + FA_RCH * 16384;
-  static constexpr uint32_t SCL = STG + FA_RCH * 4096;
-  static constexpr uint32_t XCH = SCL + FA_RCH * 256;
-  static constexpr uint32_t BAR = XCH + 2 * FA_THREADS * 4;
-  static constexpr uint32_t RS = BAR + 64;                       // FA_RCH * FA_CH row sources
-  static constexpr uint32_t TOTAL = RS + FA_RCH * FA_CH * 16;
-};
-
-struct FaRow {
-  long long slot;   // row slot in its store (-1: no row)
-  int from_raw;
-  int pad;
+  static constexpr uint32_t Q = 0;                          // 2 halves x 128 rows x 128 B
+  static constexpr uint32_t KV = 32768;                     // 2 buffers x (2 halves x 64 rows x 128 B)
+  static constexpr uint32_t P = KV + 2 * 16384;             // 128 rows x 64 bf16
+  static constexpr uint32_t STG = P + 16384;                // 2 buffers x 64 rows x 64 B codes
+  static constexpr uint32_t SCL = STG + 2 * 4096;           // 2 buffers x 64 scales
+  static constexpr uint32_t XCH = SCL + 2 * 256;            // 2 x 256 floats
+  static constexpr uint32_t BAR = XCH + 2 * FA_THREADS * 4; // 2 mbarriers, TMEM base, row bits
+  static constexpr uint32_t TOTAL = BAR + 64;
 };
 
 // Rescale O only when the running maximum grows by more than this (log2 units): until then the
@@ -162,7 +155,6 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
     w_lo = qi * seg;
     w_hi = w_lo + seg;
   }
-  uint32_t* rbits = reinterpret_cast<uint32_t*>(sm + FaOff::BAR + 32);   // 4 words per round
 
   // Q rows (query qi, head hh) -> SW128 halves, optionally RMS-normalised
   {
@@ -207,167 +199,182 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *sTmem;
-  const uint32_t ocol = FA_RCH * FA_CH;
+  const uint32_t ocol = FA_CH;                             // S: columns 0..63, O: 64..191
   const uint32_t trow = tbase + (uint32_t((warp & 3) * 32) << 16);
-  FaRow* rsrc = reinterpret_cast<FaRow*>(sm + FaOff::RS);
-  float m_run = -INFINITY, l_run = 0.f;
-  bool ok = true;
-  const int nrounds = (total + FA_RCH * FA_CH - 1) / (FA_RCH * FA_CH);
-  for (int rd = 0; rd < nrounds; rd++) {
-    const int r0 = rd * FA_RCH * FA_CH;
-    const int nr = min(FA_RCH * FA_CH, total - r0);
-    const int nch = (nr + FA_CH - 1) / FA_CH;
-    // resolve list row r0 + jj (jj = tid < 128, whole warps 0..3) to its store slot once
-    if (tid < FA_RCH * FA_CH) {
-      const int jj = tid, e = r0 + jj;
-      FaRow rs{-1, 0, 0};
-      if (jj < nr) {
-        if (p.mode == 1) {
-          if (e < n_a) {
-            rs.slot = (long long)b * p.comp.cap + (e % p.comp.cap);
-          } else {
-            const int tok = raw_lo + (e - n_a);
-            if (tok >= 0) { rs.slot = (long long)b * p.raw.cap + tok % p.raw.cap; rs.from_raw = 1; }
-          }
+  uint8_t* rb8 = sm + FaOff::BAR + 32;                     // [2 buffers][8 bytes]: row validity
+  const int nrounds = (total + FA_CH - 1) / FA_CH;
+
+  // gather of list rows [r0, r0 + 64) into buffer `buf`: 4 threads per row, each resolving the
+  // row's store slot and copying its share of the row's 16-byte pieces with cp.async (rows past
+  // the list, or without a source: zeros); mode 0 also records which rows are valid
+  auto gather = [&](int rd, int buf) {
+    const int r0 = rd * FA_CH, nr = min(FA_CH, total - r0);
+    const int jj = tid >> 2, qtr = tid & 3, e = r0 + jj;
+    long long slot = -1;
+    bool from_raw = false;
+    if (jj < nr) {
+      if (p.mode == 1) {
+        if (e < n_a) {
+          slot = (long long)b * p.comp.cap + (e % p.comp.cap);
         } else {
-          const int sq = e / seg, se = e - sq * seg;
-          if (se < p.k) {
-            const int ent = p.idx[((size_t)b * p.Tq + t0 + sq) * p.k + se];
-            if (ent >= 0 && ent < p.Nh) rs.slot = (long long)b * p.comp.cap + (ent % p.comp.cap);
-            else if (ent >= p.Nh || ent < -1) report(p.status, HCL_ERR_DEVICE_FAULT);
-          } else {
-            const int tok = p.q_pos[(size_t)b * p.Tq + t0 + sq] - p.W + 1 + (se - p.k);
-            if (tok >= 0) { rs.slot = (long long)b * p.raw.cap + tok % p.raw.cap; rs.from_raw = 1; }
-          }
+          const int tok = raw_lo + (e - n_a);
+          if (tok >= 0) { slot = (long long)b * p.raw.cap + tok % p.raw.cap; from_raw = true; }
+        }
+      } else {
+        const int sq = e / seg, se = e - sq * seg;
+        if (se < p.k) {
+          const int ent = p.idx[((size_t)b * p.Tq + t0 + sq) * p.k + se];
+          if (ent >= 0 && ent < p.Nh) slot = (long long)b * p.comp.cap + (ent % p.comp.cap);
+          else if (qtr == 0 && (ent >= p.Nh || ent < -1)) report(p.status, HCL_ERR_DEVICE_FAULT);
+        } else {
+          const int tok = p.q_pos[(size_t)b * p.Tq + t0 + sq] - p.W + 1 + (se - p.k);
+          if (tok >= 0) { slot = (long long)b * p.raw.cap + tok % p.raw.cap; from_raw = true; }
         }
       }
-      rsrc[jj] = rs;
-      if (p.mode == 0) {
-        // valid list rows of the round (a selected entry, or a window token >= 0)
-        const uint32_t bits = __ballot_sync(0xffffffffu, rs.slot >= 0);
-        if ((tid & 31) == 0) rbits[tid >> 5] = bits;
-      }
     }
-    __syncthreads();
-    // gather: list row r0 + jj -> KV row jj (rows past nr: zeros)
-    constexpr int PIECES = KVFMT == HCL_BF16 ? 16 : 13;
-    for (int u = tid; u < nch * FA_CH * PIECES; u += FA_THREADS) {
-      const int jj = u / PIECES, pc = u - jj * PIECES;
-      const int ch = jj / FA_CH, r = jj % FA_CH;
-      const FaRow rs = rsrc[jj];
-      const hcl_kv_t& st = rs.from_raw ? p.raw : p.comp;
-      uint8_t* kv = sm + FaOff::KV + ch * 16384;
-      if (KVFMT == HCL_BF16) {
-        uint8_t* dst = kv + (pc >> 3) * 8192 + r * 128 + (((pc & 7) ^ (r & 7)) << 4);
-        if (rs.slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.data) + rs.slot * 256 + pc * 16);
+    if (p.mode == 0) {
+      const uint32_t bal = __ballot_sync(0xffffffffu, slot >= 0);
+      uint32_t byte = 0;
+#pragma unroll
+      for (int i = 0; i < 8; i++) byte |= ((bal >> (4 * i)) & 1u) << i;
+      if ((tid & 31) == 0) rb8[buf * 8 + warp] = uint8_t(byte);   // rows 8 warp .. 8 warp + 7
+    }
+    const hcl_kv_t& st = from_raw ? p.raw : p.comp;
+    uint8_t* kv = sm + FaOff::KV + buf * 16384;
+    if (KVFMT == HCL_BF16) {
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        const int pc = qtr * 4 + i;
+        uint8_t* dst = kv + (pc >> 3) * 8192 + jj * 128 + (((pc & 7) ^ (jj & 7)) << 4);
+        if (slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.data) + slot * 256 + pc * 16);
         else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-      } else if (pc < 8) {
-        uint8_t* dst = kv + 8192 + r * 128 + ((pc ^ (r & 7)) << 4);
-        if (rs.slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.rope) + rs.slot * 128 + pc * 16);
-        else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-      } else if (pc < 12) {
-        uint8_t* dst = sm + FaOff::STG + (ch * FA_CH + r) * 64 + (pc - 8) * 16;
-        if (rs.slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.data) + rs.slot * 64 + (pc - 8) * 16);
-        else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
-      } else {
-        float* dst = reinterpret_cast<float*>(sm + FaOff::SCL) + ch * FA_CH + r;
-        if (rs.slot >= 0)
-          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)),
-                       "l"(st.scale + rs.slot)
-                       : "memory");
-        else *dst = 0.f;
       }
+    } else if (qtr < 2) {                                  // RoPE dims 64..127, as stored
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        const int pc = qtr * 4 + i;
+        uint8_t* dst = kv + 8192 + jj * 128 + ((pc ^ (jj & 7)) << 4);
+        if (slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.rope) + slot * 128 + pc * 16);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+      }
+    } else if (qtr == 2) {                                 // E4M3 codes of dims 0..63
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        uint8_t* dst = sm + FaOff::STG + buf * 4096 + jj * 64 + i * 16;
+        if (slot >= 0) cp_async16(dst, static_cast<const uint8_t*>(st.data) + slot * 64 + i * 16);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+      }
+    } else {
+      float* dst = reinterpret_cast<float*>(sm + FaOff::SCL + buf * 256) + jj;
+      if (slot >= 0)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)),
+                     "l"(st.scale + slot)
+                     : "memory");
+      else *dst = 0.f;
     }
     cp_async_commit();
-    cp_async_wait<0>();
+  };
+
+  float m_run = -INFINITY, l_run = 0.f;
+  bool ok = true;
+  const float c2 = p.scale_log2;
+  const unsigned long long c2x2 = f2_make(c2, c2);
+  if (nrounds > 0) gather(0, 0);
+  for (int rd = 0; rd < nrounds; rd++) {
+    const int buf = rd & 1, r0 = rd * FA_CH, nr = min(FA_CH, total - r0);
+    cp_async_wait<0>();                                    // gather(rd), this thread's copies
     __syncthreads();
     if (KVFMT == HCL_FP8SPLIT) {
-      for (int u = tid; u < nch * FA_CH * 8; u += FA_THREADS) {
-        const int jj = u >> 3, cc = u & 7, ch = jj / FA_CH, r = jj % FA_CH;
-        const uint2 codes = *reinterpret_cast<const uint2*>(sm + FaOff::STG + (ch * FA_CH + r) * 64 + cc * 8);
-        const float sc = reinterpret_cast<const float*>(sm + FaOff::SCL)[ch * FA_CH + r];
+      // widen: 8 codes x scale -> one 16-byte bf16 piece of the first half
+      for (int u = tid; u < FA_CH * 8; u += FA_THREADS) {
+        const int jj = u >> 3, cc = u & 7;
+        const uint2 codes = *reinterpret_cast<const uint2*>(sm + FaOff::STG + buf * 4096 + jj * 64 + cc * 8);
+        const float sc = reinterpret_cast<const float*>(sm + FaOff::SCL + buf * 256)[jj];
         uint4 v;
         v.x = fa_e4m3x2(uint16_t(codes.x & 0xffff), sc);
         v.y = fa_e4m3x2(uint16_t(codes.x >> 16), sc);
         v.z = fa_e4m3x2(uint16_t(codes.y & 0xffff), sc);
         v.w = fa_e4m3x2(uint16_t(codes.y >> 16), sc);
-        *reinterpret_cast<uint4*>(sm + FaOff::KV + ch * 16384 + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
+        *reinterpret_cast<uint4*>(sm + FaOff::KV + buf * 16384 + jj * 128 + ((cc ^ (jj & 7)) << 4)) = v;
       }
     }
     fence_proxy_async_smem();
     __syncthreads();
     tc_fence_after();
+    // S = Q K^T for the 64 rows of the round (M = 128, N = 64, K = 128 in 8 steps)
     if (tid == 0) {
       const uint32_t aq = smem_u32(sm + FaOff::Q);
-      for (int ch = 0; ch < nch; ch++) {
-        const uint32_t ak = smem_u32(sm + FaOff::KV + ch * 16384);
+      const uint32_t ak = smem_u32(sm + FaOff::KV + buf * 16384);
 #pragma unroll
-        for (int ks = 0; ks < 8; ks++) {
-          const uint32_t h = ks >> 2, kk = ks & 3;
-          umma_bf16(tbase + ch * FA_CH, make_sdesc(aq + h * 16384 + kk * 32, 16, 1024, SMEM_SWIZZLE_128B),
-                    make_sdesc(ak + h * 8192 + kk * 32, 16, 1024, SMEM_SWIZZLE_128B),
-                    idesc_bf16(128, FA_CH), ks > 0 ? 1u : 0u);
-        }
+      for (int ks = 0; ks < 8; ks++) {
+        const uint32_t h = ks >> 2, kk = ks & 3;
+        umma_bf16(tbase, make_sdesc(aq + h * 16384 + kk * 32, 16, 1024, SMEM_SWIZZLE_128B),
+                  make_sdesc(ak + h * 8192 + kk * 32, 16, 1024, SMEM_SWIZZLE_128B),
+                  idesc_bf16(128, FA_CH), ks > 0 ? 1u : 0u);
       }
       umma_commit(bar_s);
     }
     __syncwarp();   // warp 0 reconverges before waiting (the issuing lane is not left behind)
+    // the previous round's PV has finished reading the other buffer (and P, and writing O):
+    // the next gather may start, overlapping this round's MMAs and softmax
+    if (rd > 0) ok = ok && mbar_wait(bar_o, (rd - 1) & 1, p.limit, nullptr);
+    if (rd + 1 < nrounds) gather(rd + 1, buf ^ 1);
     ok = ok && mbar_wait(bar_s, rd & 1, p.limit, nullptr);
     tc_fence_after();
-    // this thread's 32 columns of each chunk, held in registers for both softmax passes
-    uint32_t vb[FA_RCH];
-    uint32_t sv[FA_RCH][32];
-    float lmax = -INFINITY;
-#pragma unroll
-    for (int ch = 0; ch < FA_RCH; ch++) {
-      tmem_ld16(trow + ch * FA_CH + hc * 32, *reinterpret_cast<uint32_t(*)[16]>(&sv[ch][0]));
-      tmem_ld16(trow + ch * FA_CH + hc * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[ch][16]));
+    // this thread's 32 columns of the round
+    uint32_t sv[32];
+    tmem_ld16(trow + hc * 32, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
+    tmem_ld16(trow + hc * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+    uint32_t vb = 0u;
+    if (rv) {
+      const int c0 = r0 + hc * 32;
+      vb = (range_bits(c0, 0, nv_e) | range_bits(c0, w_lo, w_hi)) & range_bits(c0, r0, r0 + nr);
+      if (p.mode == 0) vb &= *reinterpret_cast<const uint32_t*>(rb8 + buf * 8 + hc * 4);
     }
     tmem_ld_wait();
+    // row maximum of the raw scores (the scale is positive, so max(s) * scale = max(s * scale))
+    float smax = -INFINITY;
+    if (vb == 0xFFFFFFFFu) {
 #pragma unroll
-    for (int ch = 0; ch < FA_RCH; ch++) {
-      vb[ch] = 0u;
-      if (ch < nch && rv) {
-        const int c0 = r0 + ch * FA_CH + hc * 32;
-        vb[ch] = (range_bits(c0, 0, nv_e) | range_bits(c0, w_lo, w_hi)) &
-                 range_bits(c0, r0, r0 + nr);
-        if (p.mode == 0) vb[ch] &= rbits[2 * ch + hc];
-      }
+      for (int j = 0; j < 32; j += 2) smax = fmax3(smax, __uint_as_float(sv[j]), __uint_as_float(sv[j + 1]));
+    } else {
 #pragma unroll
       for (int j = 0; j < 32; j++)
-        if ((vb[ch] >> j) & 1u) lmax = fmaxf(lmax, __uint_as_float(sv[ch][j]) * p.scale_log2);
+        if ((vb >> j) & 1u) smax = fmaxf(smax, __uint_as_float(sv[j]));
     }
-    xch[tid] = lmax;
+    xch[tid] = smax == -INFINITY ? -INFINITY : smax * c2;
     __syncthreads();
     const float m_cand = fmaxf(m_run, fmaxf(xch[row], xch[row + FA_ROWS]));
     // the same decision in both threads of a row: a new reference maximum only when it grew by
     // more than FA_RESCALE_LOG2 (or is the first finite one)
     const bool grow = m_cand > m_run + FA_RESCALE_LOG2;
     const float m_new = grow ? m_cand : m_run;
-    const float alpha = (grow && m_run > -INFINITY) ? exp2f(m_run - m_new) : 1.f;
+    const float alpha = (grow && m_run > -INFINITY) ? ex2_ftz(m_run - m_new) : 1.f;
     const float muse = m_new == -INFINITY ? 0.f : m_new;
-    float lsum = 0.f;
+    const unsigned long long negm = f2_make(-muse, -muse);
+    // probabilities 2^(s * scale - m) of the valid columns, bf16 into P, fp32 into the row sum
+    uint8_t* prow = sm + FaOff::P + row * 128;
+    unsigned long long lr = 0ull;
 #pragma unroll
-    for (int ch = 0; ch < FA_RCH; ch++) {
-      uint8_t* prow = sm + FaOff::P + ch * 16384 + row * 128;
+    for (int q4 = 0; q4 < 4; q4++) {
+      uint32_t pk[4];
 #pragma unroll
-      for (int q4 = 0; q4 < 4; q4++) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int i = 0; i < 8; i += 2) {
-          const int j = q4 * 8 + i;
-          const float p0 = ((vb[ch] >> j) & 1u) ? exp2f(__uint_as_float(sv[ch][j]) * p.scale_log2 - muse) : 0.f;
-          const float p1 = ((vb[ch] >> (j + 1)) & 1u) ? exp2f(__uint_as_float(sv[ch][j + 1]) * p.scale_log2 - muse) : 0.f;
-          lsum += p0 + p1;
-          pk[i >> 1] = fa_pack(p0, p1);
+      for (int i = 0; i < 8; i += 2) {
+        const int j = q4 * 8 + i;
+        const unsigned long long t = f2_fma(f2_make(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), c2x2, negm);
+        float p0 = ex2_ftz(f2_lo(t)), p1 = ex2_ftz(f2_hi(t));
+        if (vb != 0xFFFFFFFFu) {
+          p0 = ((vb >> j) & 1u) ? p0 : 0.f;
+          p1 = ((vb >> (j + 1)) & 1u) ? p1 : 0.f;
         }
-        if (ch < nch)
-          *reinterpret_cast<uint4*>(prow + (((hc * 4 + q4) ^ (row & 7)) << 4)) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        lr = f2_add(lr, f2_make(p0, p1));
+        pk[i >> 1] = fa_pack(p0, p1);
       }
+      *reinterpret_cast<uint4*>(prow + (((hc * 4 + q4) ^ (row & 7)) << 4)) =
+          make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
-    // O (complete: the previous round's PV was waited for) rescaled in TMEM where the reference
-    // maximum moved; warp-uniform (TMEM loads and stores are warp-collective)
+    // O rescaled in TMEM where the reference maximum moved (no PV in flight: the previous one
+    // was waited for above); warp-uniform (TMEM loads and stores are warp-collective)
     if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
       for (int q4 = 0; q4 < 4; q4++) {
@@ -380,28 +387,29 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
       }
       tmem_st_wait();
     }
+    const float lsum = f2_lo(lr) + f2_hi(lr);
     l_run = l_run * alpha + lsum;
     m_run = m_new;
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // O += P V (M = 128, N = 128 dims, K = 64 rows in 4 steps; V is the MN-major view of the
+    // same tile: 64-dim halves 8 KB apart, 8-row groups 1 KB apart)
     if (tid == 0) {
-      for (int ch = 0; ch < nch; ch++) {
-        const uint32_t ap = smem_u32(sm + FaOff::P + ch * 16384);
-        const uint32_t av = smem_u32(sm + FaOff::KV + ch * 16384);
+      const uint32_t ap = smem_u32(sm + FaOff::P);
+      const uint32_t av = smem_u32(sm + FaOff::KV + buf * 16384);
 #pragma unroll
-        for (int ks = 0; ks < 4; ks++)
-          umma_bf16(tbase + ocol, make_sdesc(ap + ks * 32, 16, 1024, SMEM_SWIZZLE_128B),
-                    make_sdesc(av + ks * 2048, 8192, 1024, SMEM_SWIZZLE_128B),
-                    idesc_bf16(128, FA_D) | (1u << 16), (rd > 0 || ch > 0 || ks > 0) ? 1u : 0u);
-      }
+      for (int ks = 0; ks < 4; ks++)
+        umma_bf16(tbase + ocol, make_sdesc(ap + ks * 32, 16, 1024, SMEM_SWIZZLE_128B),
+                  make_sdesc(av + ks * 2048, 8192, 1024, SMEM_SWIZZLE_128B),
+                  idesc_bf16(128, FA_D) | (1u << 16), (rd > 0 || ks > 0) ? 1u : 0u);
       umma_commit(bar_o);
     }
     __syncwarp();
-    ok = ok && mbar_wait(bar_o, rd & 1, p.limit, nullptr);   // KV, P and O free again
-    tc_fence_after();
   }
+  if (nrounds > 0) ok = ok && mbar_wait(bar_o, (nrounds - 1) & 1, p.limit, nullptr);
+  tc_fence_after();
   if (!ok) report(p.status, HCL_ERR_TIMEOUT);
   xch[FA_THREADS + tid] = l_run;
   __syncthreads();
@@ -463,6 +471,7 @@ hcl_status_t launch_flash_t(const FaParams& p, cudaStream_t st) {
 
 bool hca_flash_usable(const AttnArgs& a) {
   if (a.H > FA_ROWS || a.d != FA_D) return false;
+  if (!(a.scale > 0.f)) return false;   // the row maximum is taken before scaling
   if (!(a.comp.fmt == HCL_BF16 || a.comp.fmt == HCL_FP8SPLIT)) return false;
   const int G = std::max(1, FA_ROWS / a.H);
   const int n_groups = (a.Tq + G - 1) / G;

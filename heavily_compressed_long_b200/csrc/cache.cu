@@ -95,7 +95,7 @@ __device__ __forceinline__ uint4 pack8_bf16(const float (&v)[8]) {
 }
 
 __global__ void __launch_bounds__(AP_THREADS) cache_append_kernel(AppendParams p) {
-  __shared__ float part[3 * 2048];         // stream partials [NS][3][d] (pool.cuh), NS * d = 2048
+  __shared__ __align__(16) float part[3 * 2048];   // stream partials [NS][3][d] (pool.cuh), NS * d = 2048
   __shared__ float red[4];
   __shared__ float amax2[2];
   pdl_enter();

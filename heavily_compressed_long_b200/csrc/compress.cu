@@ -73,6 +73,58 @@ __global__ void __launch_bounds__(128, ONE ? 5 : 1) compress_entry_kernel(
   store8(out, out_fmt, ((size_t)b * out_cap + i) * d + chunk * 8, v);
 }
 
+// CSA with m = 4 (span 8) and d/8 = 2^lgG: one group of d/8 threads per entry, a grid row per
+// sequence (no index division), the bias (times log2 e) in shared memory, and entries whose 8
+// slots all lie in [0, L) loaded without per-slot checks.  Same arithmetic as pool8_any.
+__global__ void __launch_bounds__(128, 5) compress_span8_kernel(
+    const __nv_bfloat16* __restrict__ kv, const __nv_bfloat16* __restrict__ gate,
+    const float* __restrict__ bias, int L, int d, int lgG, int m, int first_off, int e0, int e1,
+    void* out, int out_fmt, int out_cap, const float* __restrict__ gamma, float eps) {
+  __shared__ float bls[8];
+  if (threadIdx.x < 8) bls[threadIdx.x] = __ldg(bias + threadIdx.x) * kPoolLog2e;
+  __syncthreads();
+  const int b = blockIdx.y;
+  const int item = blockIdx.x * 128 + threadIdx.x;
+  const int i = e0 + (item >> lgG), chunk = item & ((1 << lgG) - 1);
+  if (i >= e1) return;  // whole groups only (the group size divides 128)
+  const long long t0 = (long long)m * i + first_off;
+  const size_t rs = (size_t)d >> 3;                      // row stride in 16-byte vectors
+  const uint4* kvb = reinterpret_cast<const uint4*>(kv + (size_t)b * L * d) + chunk;
+  const uint4* gb = reinterpret_cast<const uint4*>(gate + (size_t)b * L * d) + chunk;
+  uint4 xv[8], gv[8];
+  float bl[8];
+  if (t0 >= 0 && t0 + 8 <= L) {
+    const uint4* kp = kvb + (size_t)t0 * rs;
+    const uint4* gp = gb + (size_t)t0 * rs;
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+      xv[j] = __ldg(kp + j * rs);
+      gv[j] = __ldg(gp + j * rs);
+      bl[j] = bls[j];
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+      const long long t = t0 + j;
+      xv[j] = make_uint4(0, 0, 0, 0);
+      gv[j] = make_uint4(0, 0, 0, 0);
+      bl[j] = -INFINITY;
+      if (t >= 0 && t < L) {
+        xv[j] = __ldg(kvb + (size_t)t * rs);
+        gv[j] = __ldg(gb + (size_t)t * rs);
+        bl[j] = bls[j];
+      }
+    }
+  }
+  Pool8 P;
+  P.init();
+  P.block<true>(xv, gv, bl);
+  float v[8];
+  P.result(v);
+  if (gamma != nullptr) rmsnorm8_group(v, 1 << lgG, d, chunk, gamma, eps);
+  store8(out, out_fmt, ((size_t)b * out_cap + i) * d + chunk * 8, v);
+}
+
 // One block of 256 threads per entry: thread t pools channel chunk t % G of slot stream t / G
 // (pool_streams / pool_stream_len), the block's first 128 threads merge the streams.  ONE:
 // streams of at most 8 slots.
@@ -81,7 +133,7 @@ __global__ void __launch_bounds__(256, 2) compress_streams_kernel(
     const __nv_bfloat16* __restrict__ kv, const __nv_bfloat16* __restrict__ gate,
     const float* __restrict__ bias, int L, int d, int m, int e0, int e1, void* out,
     int out_fmt, int out_cap, const float* __restrict__ gamma, float eps) {
-  __shared__ float part[3 * 2048];          // [NS][3][d]: NS * d = 2048 for every d
+  __shared__ __align__(16) float part[3 * 2048];   // [NS][3][d]: NS * d = 2048 for every d
   __shared__ float red[4];
   const int G = d >> 3;
   const int b = blockIdx.x / (e1 - e0);
@@ -136,6 +188,12 @@ hcl_status_t launch_compress(const void* kv, const void* gate, const float* bias
     else
       compress_streams_kernel<false><<<grid, 256, 0, st>>>(kvp, gp, bias, L, d, m, e0, e1, out,
                                                            out_fmt, out_cap, gamma, eps);
+  } else if (overlap && m == 4 && (G & (G - 1)) == 0 && B <= 65535) {
+    int lg = 0;
+    while ((1 << lg) < G) lg++;
+    const dim3 grid((unsigned)(((long long)(e1 - e0) * G + 127) / 128), (unsigned)B);
+    compress_span8_kernel<<<grid, 128, 0, st>>>(kvp, gp, bias, L, d, lg, m, -m, e0, e1, out,
+                                                out_fmt, out_cap, gamma, eps);
   } else {
     const long long threads = (long long)(e1 - e0) * B * G;
     const int blk = (128 / G) * G;                     // whole groups per block (G <= 128)

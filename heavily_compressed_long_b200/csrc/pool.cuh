@@ -22,54 +22,14 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "hcl_common.cuh"
+
 namespace hcl {
 
 constexpr float kPoolLog2e = 1.4426950408889634f;
 
-__device__ __forceinline__ float pool_ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
+__device__ __forceinline__ float pool_ex2(float x) { return ex2_ftz(x); }
 
-// Packed pairs of fp32 (one 64-bit register pair) and the sm_100 paired-fp32 instructions:
-// lane-wise IEEE fp32 results, the same as two scalar instructions, in one issue.
-__device__ __forceinline__ unsigned long long f2_make(float lo, float hi) {
-  unsigned long long r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ float f2_lo(unsigned long long v) {
-  float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return lo;
-}
-__device__ __forceinline__ float f2_hi(unsigned long long v) {
-  float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return hi;
-}
-__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
-                                                     unsigned long long c) {
-  unsigned long long r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
-  unsigned long long r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
-  unsigned long long r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
 // channels 2w, 2w+1 of a 16-byte row of 8 bf16, widened exactly to an fp32 pair
 __device__ __forceinline__ unsigned long long bf16_pair(const uint4& v, int w) {
   const uint32_t u = w == 0 ? v.x : w == 1 ? v.y : w == 2 ? v.z : v.w;
@@ -215,6 +175,19 @@ __host__ __device__ constexpr int pool_stream_len(int span, int d) {
   return (span + pool_streams(d) - 1) / pool_streams(d);
 }
 
+// A stream's partial state into part ([NS][3][d] floats, 16-byte aligned), as 16-byte stores.
+__device__ __forceinline__ void pool_store_partial(const Pool8& P, float* part, int d, int s,
+                                                   int chunk) {
+  float4* base = reinterpret_cast<float4*>(part + (size_t)s * 3 * d + chunk * 8);
+  const int q = d / 4;                                    // float4s per [d] row
+  base[0] = make_float4(P.M[0], P.M[1], P.M[2], P.M[3]);
+  base[1] = make_float4(P.M[4], P.M[5], P.M[6], P.M[7]);
+  base[q] = make_float4(P.S[0], P.S[1], P.S[2], P.S[3]);
+  base[q + 1] = make_float4(P.S[4], P.S[5], P.S[6], P.S[7]);
+  base[2 * q] = make_float4(P.A[0], P.A[1], P.A[2], P.A[3]);
+  base[2 * q + 1] = make_float4(P.A[4], P.A[5], P.A[6], P.A[7]);
+}
+
 // Stream s's partial (max, sum, weighted sum) of channel chunk `chunk`, stored into
 // part ([NS][3][d] floats).
 template <bool NC, bool ONE = false, class RowFn>
@@ -225,13 +198,7 @@ __device__ __forceinline__ void pool_stream_partial(RowFn row, const float* __re
   const int j0 = s * K, j1 = min(span, j0 + K);
   Pool8 P;
   pool_run<NC, ONE>(row, bias, j0, j1, chunk, P);
-  float* base = part + (size_t)s * 3 * d + chunk * 8;
-#pragma unroll
-  for (int c = 0; c < 8; c++) {
-    base[c] = P.M[c];
-    base[d + c] = P.S[c];
-    base[2 * d + c] = P.A[c];
-  }
+  pool_store_partial(P, part, d, s, chunk);
 }
 
 // Merge of the NS stream partials in `part` (complete and visible to the block) by the block's
