@@ -611,7 +611,8 @@ __global__ void attn_merge_kernel(AttnParams p) {
 // per chunk) and O (128 columns) live in TMEM.  The softmax is two-pass over the split's
 // chunks: row maximum, then exp2 / row sum / P in bf16.  Splits merge as in attn_kernel.
 constexpr int TC_MAXC = 4;          // chunks per block with a single split
-constexpr int TC_MAXC_MERGE = 2;    // chunks per block when splits merge in a cluster
+constexpr int TC_MAXC_MERGE = 2;    // chunks per block when splits merge in a cluster (its KV
+                                    // and P tiles, 64 KB, then stage the 128 x 512 B partials)
 constexpr int TC_ROWS = 128;        // head rows per block = UMMA M = TMEM lanes
 constexpr int TC_THREADS = 256;     // two threads per row (column halves)
 
@@ -666,15 +667,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
   const uint32_t ocol = uint32_t(p.cps * 64);              // O columns after the S columns
   const uint32_t ncols = ocol + D <= 256 ? 256u : 512u;
 
+  // splits > 1: the partials of this block's head rows arrive by bulk copies, counted on
+  // bar_r: S copies of rows_o rows of 512 bytes (rows_o = this block's rows, see the push)
+  uint64_t* bar_r = bar_s + 3;
+  const int rpo = p.splits > 1 ? (TC_ROWS + p.splits - 1) / p.splits : 1;
+  auto rows_of = [&](int o) { return max(0, min(rpo, p.H - o * rpo)); };
   if (tid == 0) {
     mbar_init(bar_s, 1);
     mbar_init(bar_o, 1);
+    if (p.splits > 1) {
+      mbar_init(bar_r, 1);
+      mbar_arrive_expect_tx(bar_r, uint32_t(p.splits * rows_of(split) * D * 4));
+    }
     fence_barrier_init();
   }
   if (warp == 0) {
     tmem_alloc(sTmem, ncols);
     tmem_relinquish();
   }
+  // every block's bar_r is initialised before any block may copy into it (this waits on no
+  // other kernel: it runs while the top-k still works)
+  if (p.splits > 1) cg::this_cluster().sync();
   const bool early = early_ok && c_begin * KVB >= n_a;     // window rows only
   if (!early_ok) pdl_enter();
   const int pos = p.q_pos[b];
@@ -866,22 +879,32 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
   const float mrow = fmaxf(xch[row], xch[row + TC_ROWS]);
   const float muse = mrow == -INFINITY ? 0.f : mrow;
   float lsum = 0.f;
+  const unsigned long long c2x2 = f2_make(p.scale_log2, p.scale_log2);
+  const unsigned long long negm = f2_make(-muse, -muse);
   auto emit_p = [&](int c, const uint32_t (&r32)[32]) {
     const uint32_t vb = visw[2 * c + hc];
     uint8_t* prow = sm + off.pm + c * 16384 + row * 128;
+    unsigned long long ls2 = 0ull;   // two partial sums (+0.0f each)
 #pragma unroll
     for (int q4 = 0; q4 < 4; q4++) {
       uint32_t pk[4];
 #pragma unroll
       for (int i = 0; i < 8; i += 2) {
         const int j = q4 * 8 + i;
-        const float p0 = ((vb >> j) & 1u) ? exp2f(__uint_as_float(r32[j]) * p.scale_log2 - muse) : 0.f;
-        const float p1 = ((vb >> (j + 1)) & 1u) ? exp2f(__uint_as_float(r32[j + 1]) * p.scale_log2 - muse) : 0.f;
-        lsum += p0 + p1;
+        // 2^(s * scale - m) for a pair of columns: one paired FMA, two exponentials
+        const unsigned long long t =
+            f2_fma(f2_make(__uint_as_float(r32[j]), __uint_as_float(r32[j + 1])), c2x2, negm);
+        float p0 = ex2_ftz(f2_lo(t)), p1 = ex2_ftz(f2_hi(t));
+        if (vb != 0xFFFFFFFFu) {
+          p0 = ((vb >> j) & 1u) ? p0 : 0.f;
+          p1 = ((vb >> (j + 1)) & 1u) ? p1 : 0.f;
+        }
+        ls2 = f2_add(ls2, f2_make(p0, p1));
         pk[i >> 1] = pack_bf16(p0, p1);
       }
       *reinterpret_cast<uint4*>(prow + (((hc * 4 + q4) ^ (row & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
+    lsum += f2_lo(ls2) + f2_hi(ls2);
   };
   if (inreg) {
 #pragma unroll
@@ -925,17 +948,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
   const bool hv = row < p.H;
   float m2 = mrow, l2 = xch[TC_THREADS + row] + xch[TC_THREADS + row + TC_ROWS];
   const float inv_l = l2 > 0.f ? 1.f / l2 : 0.f;
-  float* pdst = nullptr;
-  if (p.splits > 1) {
-    // row r is merged by block r / rpo (contiguous head blocks: a warp's stores reach one or
-    // two blocks), in its slot r % rpo
+  // splits > 1: row r is merged by block r / rpo (contiguous head blocks) in its slot r % rpo;
+  // the normalised partial rows are staged in this block's (now idle) KV and P tiles, XOR-
+  // swizzled in 16-byte chunks, and block o's rows then go to it as one bulk copy
+  uint8_t* stage = sm + off.kv;                   // 128 rows x 512 B (KV + P tiles, cps == 2)
+  if (p.splits > 1 && hv && hc == 0) {
     cg::cluster_group cluster = cg::this_cluster();
-    const int rpo = (TC_ROWS + p.splits - 1) / p.splits;
-    const int owner = row / rpo, slot = row % rpo;
-    pdst = cluster.map_shared_rank(recv, owner) + ((size_t)slot * p.splits + split) * D + hc * 64;
-    if (hv && hc == 0)
-      *(cluster.map_shared_rank(recv_lse, owner) + slot * p.splits + split) =
-          l2 > 0.f ? m2 + log2f(l2) : -INFINITY;
+    *(cluster.map_shared_rank(recv_lse, row / rpo) + (row % rpo) * p.splits + split) =
+        l2 > 0.f ? m2 + log2f(l2) : -INFINITY;
   }
   float f = inv_l;
   if (p.splits == 1 && p.sink) {
@@ -953,14 +973,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
     for (int q4 = 0; q4 < 4; q4++)
       tmem_ld16(trow + ocol + hc * 64 + q4 * 16, *reinterpret_cast<uint32_t(*)[16]>(&r64[q4 * 16]));
     tmem_ld_wait();
-    if (hv) {
-      if (p.splits > 1) {
+    if (p.splits > 1) {
+      // chunk c (16 bytes) of row `row` at chunk position c ^ (row & 7): conflict-free stores
 #pragma unroll
-        for (int i = 0; i < 64; i += 4)
-          *reinterpret_cast<float4*>(pdst + i) =
-              make_float4(__uint_as_float(r64[i]) * inv_l, __uint_as_float(r64[i + 1]) * inv_l,
-                          __uint_as_float(r64[i + 2]) * inv_l, __uint_as_float(r64[i + 3]) * inv_l);
-      } else {
+      for (int i = 0; i < 64; i += 4) {
+        const int c = hc * 16 + (i >> 2);
+        *reinterpret_cast<float4*>(stage + row * 512 + ((c ^ (row & 7)) << 4)) =
+            make_float4(__uint_as_float(r64[i]) * inv_l, __uint_as_float(r64[i + 1]) * inv_l,
+                        __uint_as_float(r64[i + 2]) * inv_l, __uint_as_float(r64[i + 3]) * inv_l);
+      }
+    } else if (hv) {
+      {
         __nv_bfloat16* dst = p.out + ((size_t)b * p.H + row) * D + hc * 64;
 #pragma unroll
         for (int i = 0; i < 64; i += 8) {
@@ -973,6 +996,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
       }
     }
   }
+  if (p.splits > 1) {
+    fence_proxy_async_smem();                     // staged rows -> the bulk-copy engine
+    __syncthreads();
+    if (tid == 0) {
+      // block o receives rows o*rpo .. o*rpo + rows_of(o) - 1 at recv[split][slot][D], still
+      // swizzled (chunk c of row r at c ^ (r & 7))
+      for (int o = 0; o < p.splits; o++)
+        if (rows_of(o) > 0)
+          bulk_copy_to_cluster(cluster_map(recv + (size_t)split * rpo * D, o),
+                               stage + (size_t)o * rpo * 512, uint32_t(rows_of(o) * 512),
+                               cluster_map(bar_r, o));
+    }
+  }
   if (p.splits == 1 && hv && hc == 0 && p.lse)
     p.lse[(size_t)b * p.H + row] = l2 > 0.f ? (m2 + log2f(l2)) * LN2 : -INFINITY;
   tc_fence_before();
@@ -982,11 +1018,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
     tmem_dealloc(tbase, ncols);
   }
   if (p.splits > 1) {
-    // merge the rows this block owns (row r -> block r / rpo, slot r % rpo)
+    // merge the rows this block owns (row r -> block r / rpo, slot r % rpo).  Once its own
+    // copies have all landed (bar_r), a block's outgoing copies have been read too when every
+    // block has passed the cluster barrier, which also publishes the log-sum-exps.
+    if (!mbar_wait(bar_r, 0, limit, nullptr)) report(p.status, HCL_ERR_TIMEOUT);
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();
     const int S = p.splits;
-    const int rpo = (TC_ROWS + S - 1) / S;
     for (int slot = warp; slot < rpo; slot += TC_THREADS / 32) {
       const int h = split * rpo + slot;
       if (h >= p.H) break;
@@ -1005,12 +1043,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
       for (int o2 = 16; o2 > 0; o2 >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o2);
       if (p.sink && M > -INFINITY) den += exp2f(s2 - M);
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      const float4* part = reinterpret_cast<const float4*>(recv + (size_t)slot * S * D);
+      const float4* part = reinterpret_cast<const float4*>(recv + (size_t)slot * D);
+      const int pc = lane ^ (h & 7);              // this lane's 16-byte chunk, as swizzled
 #pragma unroll
       for (int s = 0; s < MAX_CLUSTER_ROWS; s++) {
         const float wgt = __shfl_sync(0xffffffffu, wl, s);
         if (s < S && wgt != 0.f) {
-          const float4 v = part[s * (D / 4) + lane];
+          const float4 v = part[(size_t)s * rpo * (D / 4) + pc];
           acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
         }
       }
@@ -1116,7 +1155,7 @@ hcl_status_t launch_nw(const AttnParams& p, int NW, cudaStream_t st, long long g
 // block (up to 128), splits merged in a cluster (or a single split), <= TC_MAXC chunks each.
 bool tc_usable(const AttnArgs& a, const Plan& pl) {
   return a.mode == 0 && a.Tq == 1 && a.H <= TC_ROWS &&
-         ((pl.splits == 1 && pl.cps <= TC_MAXC) || (pl.cmerge && pl.cps <= TC_MAXC_MERGE));
+         ((pl.splits == 1 && pl.cps <= TC_MAXC) || (pl.cmerge && pl.cps == TC_MAXC_MERGE));
 }
 
 template <int KVFMT>

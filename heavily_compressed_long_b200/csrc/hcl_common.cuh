@@ -120,6 +120,24 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   return pol;
 }
 
+// Address of this CTA's shared-memory location `p` in the shared::cluster window of cluster
+// rank `rank` (the same offset in that CTA's shared memory).
+__device__ __forceinline__ uint32_t cluster_map(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from this CTA's
+// shared memory into another CTA's of the cluster (dst and its mbarrier as shared::cluster
+// addresses, cluster_map); completion is counted on that CTA's mbarrier (complete_tx).
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, const void* src, uint32_t bytes,
+                                                     uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "r"(smem_u32(src)), "r"(bytes), "r"(mbar)
+      : "memory");
+}
+
 // Bulk copy as bulk_load, with an L2 cache policy.
 __device__ __forceinline__ void bulk_load_hint(void* dst, const void* src, uint32_t bytes,
                                                uint64_t* bar, uint64_t policy) {
