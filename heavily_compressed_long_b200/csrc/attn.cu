@@ -83,6 +83,10 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], 
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -630,9 +634,9 @@ __host__ __device__ inline TcOff tc_offsets(int cps, int splits) {
   o.bar = o.rs + cps * 64 * (uint32_t)sizeof(RowSrc);   // 2 mbarriers + TMEM base
   o.vis = o.bar + 32;                        // row-visibility bits, 64 per chunk
   o.xch = (o.vis + 8 * cps + 15) & ~15u;     // partial maxima / sums of the two column halves
-  o.recv = o.xch + 2 * TC_THREADS * 4;       // cluster merge: rpo x splits x D floats
+  o.recv = o.xch + 2 * TC_THREADS * 4;       // cluster merge: splits x rpo x D fp16 partials
   const int rpo = splits > 1 ? (TC_ROWS + splits - 1) / splits : 0;
-  o.lse = o.recv + (uint32_t)(rpo * splits * D * 4);
+  o.lse = o.recv + (uint32_t)(rpo * splits * D * 2);
   o.total = o.lse + (uint32_t)(rpo * splits * 4);
   return o;
 }
@@ -655,7 +659,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + off.bar + 16);
   uint32_t* visw = reinterpret_cast<uint32_t*>(sm + off.vis);
   float* xch = reinterpret_cast<float*>(sm + off.xch);   // [2][TC_THREADS]: partial max, sum
-  float* recv = reinterpret_cast<float*>(sm + off.recv);
+  __half* recv_h = reinterpret_cast<__half*>(sm + off.recv);   // [splits][rpo][D] fp16 partials
   float* recv_lse = reinterpret_cast<float*>(sm + off.lse);
 
   // row list of this split: k selected entries, then the W window rows
@@ -677,7 +681,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
     mbar_init(bar_o, 1);
     if (p.splits > 1) {
       mbar_init(bar_r, 1);
-      mbar_arrive_expect_tx(bar_r, uint32_t(p.splits * rows_of(split) * D * 4));
+      mbar_arrive_expect_tx(bar_r, uint32_t(p.splits * rows_of(split) * D * 2));
     }
     fence_barrier_init();
   }
@@ -949,9 +953,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
   float m2 = mrow, l2 = xch[TC_THREADS + row] + xch[TC_THREADS + row + TC_ROWS];
   const float inv_l = l2 > 0.f ? 1.f / l2 : 0.f;
   // splits > 1: row r is merged by block r / rpo (contiguous head blocks) in its slot r % rpo;
-  // the normalised partial rows are staged in this block's (now idle) KV and P tiles, XOR-
-  // swizzled in 16-byte chunks, and block o's rows then go to it as one bulk copy
-  uint8_t* stage = sm + off.kv;                   // 128 rows x 512 B (KV + P tiles, cps == 2)
+  // the normalised partial rows (|o| <= max |v|: fp16, 11 significant bits, is exact enough for
+  // a bf16 output and halves the bytes crossing between blocks) are staged in this block's (now
+  // idle) KV tiles, XOR-swizzled in 16-byte chunks, and block o's rows then go to it as one
+  // bulk copy
+  uint8_t* stage = sm + off.kv;                   // 128 rows x 256 B (KV tiles, cps == 2)
   if (p.splits > 1 && hv && hc == 0) {
     cg::cluster_group cluster = cg::this_cluster();
     *(cluster.map_shared_rank(recv_lse, row / rpo) + (row % rpo) * p.splits + split) =
@@ -974,13 +980,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
       tmem_ld16(trow + ocol + hc * 64 + q4 * 16, *reinterpret_cast<uint32_t(*)[16]>(&r64[q4 * 16]));
     tmem_ld_wait();
     if (p.splits > 1) {
-      // chunk c (16 bytes) of row `row` at chunk position c ^ (row & 7): conflict-free stores
+      // chunk c (16 bytes = 8 fp16) of row `row` at chunk position c ^ (row & 7): conflict-free
 #pragma unroll
-      for (int i = 0; i < 64; i += 4) {
-        const int c = hc * 16 + (i >> 2);
-        *reinterpret_cast<float4*>(stage + row * 512 + ((c ^ (row & 7)) << 4)) =
-            make_float4(__uint_as_float(r64[i]) * inv_l, __uint_as_float(r64[i + 1]) * inv_l,
-                        __uint_as_float(r64[i + 2]) * inv_l, __uint_as_float(r64[i + 3]) * inv_l);
+      for (int i = 0; i < 64; i += 8) {
+        const int c = hc * 8 + (i >> 3);
+        uint4 v;
+        v.x = pack_half2(__uint_as_float(r64[i]) * inv_l, __uint_as_float(r64[i + 1]) * inv_l);
+        v.y = pack_half2(__uint_as_float(r64[i + 2]) * inv_l, __uint_as_float(r64[i + 3]) * inv_l);
+        v.z = pack_half2(__uint_as_float(r64[i + 4]) * inv_l, __uint_as_float(r64[i + 5]) * inv_l);
+        v.w = pack_half2(__uint_as_float(r64[i + 6]) * inv_l, __uint_as_float(r64[i + 7]) * inv_l);
+        *reinterpret_cast<uint4*>(stage + row * 256 + ((c ^ (row & 7)) << 4)) = v;
       }
     } else if (hv) {
       {
@@ -1004,8 +1013,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
       // swizzled (chunk c of row r at c ^ (r & 7))
       for (int o = 0; o < p.splits; o++)
         if (rows_of(o) > 0)
-          bulk_copy_to_cluster(cluster_map(recv + (size_t)split * rpo * D, o),
-                               stage + (size_t)o * rpo * 512, uint32_t(rows_of(o) * 512),
+          bulk_copy_to_cluster(cluster_map(recv_h + (size_t)split * rpo * D, o),
+                               stage + (size_t)o * rpo * 256, uint32_t(rows_of(o) * 256),
                                cluster_map(bar_r, o));
     }
   }
@@ -1043,13 +1052,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
       for (int o2 = 16; o2 > 0; o2 >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o2);
       if (p.sink && M > -INFINITY) den += exp2f(s2 - M);
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      const float4* part = reinterpret_cast<const float4*>(recv + (size_t)slot * D);
-      const int pc = lane ^ (h & 7);              // this lane's 16-byte chunk, as swizzled
+      // lane l: dims 4l .. 4l+3 = half l & 1 of 16-byte chunk l / 2, as swizzled
+      const uint8_t* part = reinterpret_cast<const uint8_t*>(recv_h + (size_t)slot * D) +
+                            ((((lane >> 1) ^ (h & 7)) << 4) | ((lane & 1) << 3));
 #pragma unroll
       for (int s = 0; s < MAX_CLUSTER_ROWS; s++) {
         const float wgt = __shfl_sync(0xffffffffu, wl, s);
         if (s < S && wgt != 0.f) {
-          const float4 v = part[(size_t)s * rpo * (D / 4) + pc];
+          const uint2 hv2 = *reinterpret_cast<const uint2*>(part + (size_t)s * rpo * D * 2);
+          const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&hv2.x));
+          const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&hv2.y));
+          const float4 v = make_float4(lo.x, lo.y, hi.x, hi.y);
           acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
         }
       }
