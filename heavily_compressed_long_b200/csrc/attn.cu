@@ -1055,15 +1055,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
       // lane l: dims 4l .. 4l+3 = half l & 1 of 16-byte chunk l / 2, as swizzled
       const uint8_t* part = reinterpret_cast<const uint8_t*>(recv_h + (size_t)slot * D) +
                             ((((lane >> 1) ^ (h & 7)) << 4) | ((lane & 1) << 3));
+      // every split's partial loaded up front (independent loads), then summed in split order
+      // (a zero weight adds 0 * v = 0: the partials are finite)
+      uint2 hv2[MAX_CLUSTER_ROWS];
+#pragma unroll
+      for (int s = 0; s < MAX_CLUSTER_ROWS; s++)
+        hv2[s] = s < S ? *reinterpret_cast<const uint2*>(part + (size_t)s * rpo * D * 2)
+                       : make_uint2(0u, 0u);
 #pragma unroll
       for (int s = 0; s < MAX_CLUSTER_ROWS; s++) {
         const float wgt = __shfl_sync(0xffffffffu, wl, s);
-        if (s < S && wgt != 0.f) {
-          const uint2 hv2 = *reinterpret_cast<const uint2*>(part + (size_t)s * rpo * D * 2);
-          const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&hv2.x));
-          const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&hv2.y));
-          const float4 v = make_float4(lo.x, lo.y, hi.x, hi.y);
-          acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
+        if (s < S) {
+          const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&hv2[s].x));
+          const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&hv2[s].y));
+          acc.x += wgt * lo.x; acc.y += wgt * lo.y; acc.z += wgt * hi.x; acc.w += wgt * hi.y;
         }
       }
       const float inv = den > 0.f ? 1.f / den : 0.f;

@@ -10,16 +10,16 @@
 // queries x H heads = up to 128 (query, head) rows = the UMMA M dimension = 128 TMEM lanes, two
 // threads per row.  The group's KV list is the visible-entry prefix of its last query followed
 // by the union of its queries' windows; it is processed in rounds of 64 rows.  A round's rows
-// are gathered with cp.async into one of three KV buffers (4 threads per row, each resolving the
-// row's store slot; split FP8 rows widened to bf16 with their scale), so the gathers of rounds
-// r + 1 and r + 2 are in flight while round r runs S = Q K^T (N = 64) into TMEM, its softmax and
+// are gathered with cp.async into one of two KV buffers (4 threads per row, each resolving the
+// row's store slot; split FP8 rows widened to bf16 with their scale), so the gather of round
+// r + 1 is in flight while round r runs S = Q K^T (N = 64) into TMEM, its softmax and
 // O += P V (V read as the MN-major operand of the same SW128 tile; O accumulates in TMEM
 // across all rounds).  The softmax runs in registers with each row's own causal mask (for
 // query q: the list rows [0, visible entries of q) and the window rows of q -- two index
 // intervals, turned into bit masks; full 32-column words skip the per-column selects), its
 // probabilities taken against a reference maximum that is raised only when the row maximum
 // grows by more than 2^8, and only then is O rescaled in TMEM (load, scale, store).  Paired
-// fp32 instructions form the exponents and sums.  Two blocks fit per SM (about 113 KB of
+// fp32 instructions form the exponents and sums.  Two blocks fit per SM (about 92 KB of
 // shared memory, 256 TMEM columns each), so one block's softmax overlaps the other's MMAs.
 //
 // CSA prefill (every query has its own selection) uses the same kernel with G = 128 / H
@@ -63,18 +63,16 @@ struct FaParams {
   long long limit;
 };
 
-constexpr int FA_NBUF = 3;       // KV buffers: rounds r + 1 and r + 2 gather while r computes
 struct FaOff {
   static constexpr uint32_t Q = 0;                          // 2 halves x 128 rows x 128 B
-  static constexpr uint32_t KV = 32768;                     // FA_NBUF x (2 halves x 64 rows x 128 B)
-  static constexpr uint32_t P = KV + FA_NBUF * 16384;       // 128 rows x 64 bf16
-  static constexpr uint32_t STG = P + 16384;                // FA_NBUF x 64 rows x 64 B codes
-  static constexpr uint32_t SCL = STG + FA_NBUF * 4096;     // FA_NBUF x 64 scales
-  static constexpr uint32_t XCH = SCL + FA_NBUF * 256;      // 2 x 256 floats
+  static constexpr uint32_t KV = 32768;                     // 2 buffers x (2 halves x 64 rows x 128 B)
+  static constexpr uint32_t P = KV + 2 * 16384;             // 128 rows x 64 bf16
+  static constexpr uint32_t STG = P + 16384;                // 2 buffers x 64 rows x 64 B codes
+  static constexpr uint32_t SCL = STG + 2 * 4096;           // 2 buffers x 64 scales
+  static constexpr uint32_t XCH = SCL + 2 * 256;            // 2 x 256 floats
   static constexpr uint32_t BAR = XCH + 2 * FA_THREADS * 4; // 2 mbarriers, TMEM base, row bits
   static constexpr uint32_t TOTAL = BAR + 64;
 };
-static_assert(2 * (FaOff::TOTAL + 2048) <= 233472, "two blocks per SM");
 
 // Rescale O only when the running maximum grows by more than this (log2 units): until then the
 // probabilities are taken against the stale maximum (values <= 2^8, exact in fp32 sums).
@@ -112,13 +110,11 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
   const int t0 = grp * p.G;
   const int gq = min(p.G, p.Tq - t0);
   float* xch = reinterpret_cast<float*>(sm + FaOff::XCH);
-  uint64_t* bar_s = reinterpret_cast<uint64_t*>(sm + FaOff::BAR);   // S of even rounds
+  uint64_t* bar_s = reinterpret_cast<uint64_t*>(sm + FaOff::BAR);
   uint64_t* bar_o = bar_s + 1;
-  uint64_t* bar_s1 = bar_s + 6;                                       // S of odd rounds
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + FaOff::BAR + 16);
   if (tid == 0) {
     mbar_init(bar_s, 1);
-    mbar_init(bar_s1, 1);
     mbar_init(bar_o, 1);
     fence_barrier_init();
   }
@@ -203,9 +199,9 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *sTmem;
-  const uint32_t ocol = 2 * FA_CH;                         // S: two buffers of 64 columns, O: 128..255
+  const uint32_t ocol = FA_CH;                             // S: columns 0..63, O: 64..191
   const uint32_t trow = tbase + (uint32_t((warp & 3) * 32) << 16);
-  uint8_t* rb8 = sm + FaOff::BAR + 24;                     // [FA_NBUF][8 bytes]: row validity
+  uint8_t* rb8 = sm + FaOff::BAR + 32;                     // [2 buffers][8 bytes]: row validity
   const int nrounds = (total + FA_CH - 1) / FA_CH;
 
   // gather of list rows [r0, r0 + 64) into buffer `buf`: 4 threads per row, each resolving the
@@ -283,13 +279,13 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
   bool ok = true;
   const float c2 = p.scale_log2;
   const unsigned long long c2x2 = f2_make(c2, c2);
-  // widen round rd's split rows (FP8 codes x scale -> bf16 first half) and issue its
-  // S = Q K^T (M = 128, N = 64, K = 128 in 8 steps) into S buffer rd & 1; the gather has landed
-  // (this thread's copies waited for; the barrier publishes everyone's)
-  auto issue_s = [&](int rd) {
-    const int buf = rd % FA_NBUF;
+  if (nrounds > 0) gather(0, 0);
+  for (int rd = 0; rd < nrounds; rd++) {
+    const int buf = rd & 1, r0 = rd * FA_CH, nr = min(FA_CH, total - r0);
+    cp_async_wait<0>();                                    // gather(rd), this thread's copies
     __syncthreads();
     if (KVFMT == HCL_FP8SPLIT) {
+      // widen: 8 codes x scale -> one 16-byte bf16 piece of the first half
       for (int u = tid; u < FA_CH * 8; u += FA_THREADS) {
         const int jj = u >> 3, cc = u & 7;
         const uint2 codes = *reinterpret_cast<const uint2*>(sm + FaOff::STG + buf * 4096 + jj * 64 + cc * 8);
@@ -305,45 +301,30 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
     fence_proxy_async_smem();
     __syncthreads();
     tc_fence_after();
+    // S = Q K^T for the 64 rows of the round (M = 128, N = 64, K = 128 in 8 steps)
     if (tid == 0) {
       const uint32_t aq = smem_u32(sm + FaOff::Q);
       const uint32_t ak = smem_u32(sm + FaOff::KV + buf * 16384);
 #pragma unroll
       for (int ks = 0; ks < 8; ks++) {
         const uint32_t h = ks >> 2, kk = ks & 3;
-        umma_bf16(tbase + (rd & 1) * FA_CH,
-                  make_sdesc(aq + h * 16384 + kk * 32, 16, 1024, SMEM_SWIZZLE_128B),
+        umma_bf16(tbase, make_sdesc(aq + h * 16384 + kk * 32, 16, 1024, SMEM_SWIZZLE_128B),
                   make_sdesc(ak + h * 8192 + kk * 32, 16, 1024, SMEM_SWIZZLE_128B),
                   idesc_bf16(128, FA_CH), ks > 0 ? 1u : 0u);
       }
-      umma_commit((rd & 1) ? bar_s1 : bar_s);
+      umma_commit(bar_s);
     }
-    __syncwarp();   // warp 0 reconverges before it waits on anything
-  };
-  if (nrounds > 0) gather(0, 0);
-  if (nrounds > 1) gather(1, 1);
-  if (nrounds > 0) {
-    if (nrounds > 1) cp_async_wait<1>();
-    else cp_async_wait<0>();
-    issue_s(0);
-  }
-  for (int rd = 0; rd < nrounds; rd++) {
-    const int buf = rd % FA_NBUF, r0 = rd * FA_CH, nr = min(FA_CH, total - r0);
-    // S of the next round goes to the tensor pipe before this round's softmax
-    if (rd + 1 < nrounds) {
-      cp_async_wait<0>();                                  // gather(rd + 1)
-      issue_s(rd + 1);
-    }
-    // the previous round's PV has finished reading its buffer (and P, and writing O): the
-    // gather two rounds ahead may reuse that buffer, overlapping this round's MMAs and softmax
+    __syncwarp();   // warp 0 reconverges before waiting (the issuing lane is not left behind)
+    // the previous round's PV has finished reading the other buffer (and P, and writing O):
+    // the next gather may start, overlapping this round's MMAs and softmax
     if (rd > 0) ok = ok && mbar_wait(bar_o, (rd - 1) & 1, p.limit, nullptr);
-    if (rd + 2 < nrounds) gather(rd + 2, (rd + 2) % FA_NBUF);
-    ok = ok && mbar_wait((rd & 1) ? bar_s1 : bar_s, (rd >> 1) & 1, p.limit, nullptr);
+    if (rd + 1 < nrounds) gather(rd + 1, buf ^ 1);
+    ok = ok && mbar_wait(bar_s, rd & 1, p.limit, nullptr);
     tc_fence_after();
     // this thread's 32 columns of the round
     uint32_t sv[32];
-    tmem_ld16(trow + (rd & 1) * FA_CH + hc * 32, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
-    tmem_ld16(trow + (rd & 1) * FA_CH + hc * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+    tmem_ld16(trow + hc * 32, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
+    tmem_ld16(trow + hc * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
     uint32_t vb = 0u;
     if (rv) {
       const int c0 = r0 + hc * 32;

@@ -1070,11 +1070,16 @@ constexpr int GM_MAX_GROUPS = GM_GPT * TK_THREADS;
 
 constexpr int GM_WWORDS = 4096;  // window histogram: 8192 digits
 constexpr int GM_POOL = 512;     // groups with several candidates staged in shared memory
+constexpr int GM_FLAT = 5120;    // candidates listed flat for the emission (more: per-thread loops)
 
 struct alignas(16) GmShared {
   union {
     uint16_t list[GM_MAX_GROUPS];    // candidate group ids, in index order (fallback)
     uint32_t praw[GM_POOL][8];       // scores of the pooled groups as copied (bf16 pairs)
+    struct {                         // the candidates in index order (emission)
+      uint32_t fent[GM_FLAT];        // entry index
+      uint16_t fkey[GM_FLAT];        // order-preserving key
+    };
   };
   uint4 gms[2][TK_THREADS];      // thread t's 16 group maxima (0: no visible entry),
   uint4 g2s[2][TK_THREADS];      // their second maxima
@@ -1178,6 +1183,41 @@ __device__ void warp_suffix(const uint32_t* hist, int w_top, int w_bot, uint32_t
   if (lane == 0) res[2] = 0;
 }
 
+// The same search by the whole block in one step: thread t counts the 8 digits of words
+// w_top - 4t - 3 .. w_top - 4t (every word of a window of <= 4 x 1024 words), one block scan
+// gives the keys above each thread's digits, and the thread whose digits hold the target-th
+// largest key writes res[0..2] as warp_suffix does.  All threads call it; res is published.
+__device__ void block_window_select(const uint32_t* hist, int w_top, int w_bot, uint32_t target,
+                                    uint32_t* scan_tmp, uint32_t* res) {
+  const int hi = w_top - 4 * (int)threadIdx.x;          // this thread's highest word
+  uint32_t c[8];                                          // descending digits
+  uint32_t tot = 0;
+#pragma unroll
+  for (int j = 0; j < 4; j++) {
+    const int w = hi - j;
+    const uint32_t v = (w >= w_bot) ? hist[w] : 0u;
+    c[2 * j] = v >> 16;                                   // digit 2w + 1
+    c[2 * j + 1] = v & 0xFFFFu;                           // digit 2w
+    tot += c[2 * j] + c[2 * j + 1];
+  }
+  if (threadIdx.x == 0) res[2] = 0;
+  uint32_t total;
+  const uint32_t before = block_scan_total(tot, scan_tmp, total);
+  if (before < target && target <= before + tot) {
+    uint32_t acc = before;
+    int ti = 7;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      if (acc + c[i] >= target) { ti = i; break; }
+      acc += c[i];
+    }
+    res[0] = uint32_t(2 * (hi - (ti >> 1)) + ((ti & 1) ? 0 : 1));
+    res[1] = acc;
+    res[2] = 1;
+  }
+  __syncthreads();
+}
+
 // Radix-4 selection over 16-bit keys spread across the block, without atomics: each thread
 // counts its keys per 4-bit digit in four 64-bit words (16-bit fields, digit d in word d/4,
 // field d%4), warps add the words with shuffles, and warp 0 sums the 32 warps' counts.
@@ -1275,14 +1315,14 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
   const long long row = blockIdx.x;
   if (!prewait) pdl_enter();
   const int pos = q_pos[row];
-  if (prewait) pdl_enter();
   const int nvis = pos < 0 ? 0 : min(Nc, (pos + 1) / m);
+  const int ngv = (nvis + GM_G - 1) / GM_G;              // groups with a visible entry
+  if (prewait) pdl_enter();
   int32_t* out = idx + row * k;
   if (nvis <= k) {
     for (int j = tid; j < k; j += TK_THREADS) out[j] = j < nvis ? j : -1;
     return;
   }
-  const int ngv = (nvis + GM_G - 1) / GM_G;              // groups with a visible entry
   const uint16_t* sr = reinterpret_cast<const uint16_t*>(scores) + row * (long long)Nc;
   const bool al = (reinterpret_cast<uintptr_t>(sr) & 15) == 0;
 
@@ -1369,6 +1409,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
 
   uint32_t qm = 0, dm = 0;          // bit i: group 16t+i holds one candidate / two or more
   uint32_t ndm = 0, pbase = 0;
+  uint32_t c_own = 0;               // this thread's candidate keys
   bool inwin = false;               // every candidate key lies in the window
   for (int pass = 0; pass < 2; pass++) {
     if (need_exact) {
@@ -1457,6 +1498,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
         c += n;
       }
     }
+    c_own = c;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
     if (lane == 0 && c) atomicAdd(&S.ncand, c);
@@ -1472,8 +1514,65 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
   uint32_t T = 0u, above = 0u;
   // u16 digit counts cannot overflow while the row has fewer than 2^16 candidates
   if (inwin && S.ncand < 65536u && S.npool <= (uint32_t)GM_POOL) {
-    if (warp == 0) warp_suffix(S.wc, int((Mx - wb) >> 1), int((L - wb) >> 1), (uint32_t)k, S.res);
-    __syncthreads();
+    // the k-th largest candidate key: all candidate keys lie in [L, Mx], at most 8192 digits,
+    // searched by the whole block at once
+    block_window_select(S.wc, int((Mx - wb) >> 1), int((L - wb) >> 1), (uint32_t)k, S.scan_tmp,
+                        S.res);
+    if (S.res[2] && S.ncand <= (uint32_t)GM_FLAT) {
+      T = S.res[0] + wb;
+      above = S.res[1];
+      const uint32_t krem = (uint32_t)k - above;
+      // ---- emission from one flat candidate list in index order: every thread writes its
+      // candidates at its offset, then takes a contiguous run of at most ceil(ncand / 1024)
+      // list entries, so no warp serialises over its lanes' differing candidate counts
+      const uint32_t nc = S.ncand;
+      uint32_t ntot;
+      uint32_t o = block_scan_total(c_own, S.scan_tmp, ntot);
+      {
+        uint32_t sl = pbase;
+        for (uint32_t mm = qm | dm; mm; mm &= mm - 1u) {
+          const int i = __ffs(mm) - 1, e0 = GM_G * (GM_GPT * tid + i);
+          if ((qm >> i) & 1u) {
+            S.fkey[o] = uint16_t(gm_sh(i));
+            S.fent[o++] = uint32_t(e0) + arg_sh(i);
+          } else {
+            const uint32_t n = S.pcnt[sl++];
+            for (uint32_t e = 0; e < n; e++) {
+              const uint32_t v = S.pent[sl - 1][e];
+              S.fkey[o] = uint16_t(v >> 4);
+              S.fent[o++] = uint32_t(e0) + (v & 15u);
+            }
+          }
+        }
+      }
+      __syncthreads();
+      const uint32_t per = (nc + TK_THREADS - 1) / TK_THREADS;
+      const uint32_t j0 = min(nc, per * tid), j1 = min(nc, j0 + per);
+      uint32_t gt = 0, eq = 0;
+      for (uint32_t j = j0; j < j1; j++) {
+        const uint32_t key = S.fkey[j];
+        gt += key > T;
+        eq += key == T;
+      }
+      unsigned long long tot64;
+      const unsigned long long ex =
+          block_scan64((static_cast<unsigned long long>(eq) << 32) | gt, S.tmp64, tot64);
+      uint32_t e_before = uint32_t(ex >> 32);
+      uint32_t slot = uint32_t(ex) + min(e_before, krem);
+      for (uint32_t j = j0; j < j1; j++) {
+        const uint32_t key = S.fkey[j];
+        bool sel = key > T;
+        if (!sel && key == T) { sel = e_before < krem; e_before++; }
+        if (sel) {
+          if (slot < (uint32_t)k) S.wh[slot] = S.fent[j];
+          else report(status, HCL_ERR_DEVICE_FAULT);
+          slot++;
+        }
+      }
+      __syncthreads();
+      for (int j = tid; j < k; j += TK_THREADS) out[j] = int32_t(S.wh[j]);
+      return;
+    }
     if (S.res[2]) {
       T = S.res[0] + wb;
       above = S.res[1];
@@ -1504,7 +1603,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
           bool sel = key > T;
           if (!sel && key == T) { sel = e_before < krem; e_before++; }
           if (sel) {
-            if (slot < (uint32_t)k) out[slot] = e0 + int(v & 15u);
+            if (slot < (uint32_t)k) S.wh[slot] = uint32_t(e0 + int(v & 15u));
             else report(status, HCL_ERR_DEVICE_FAULT);
             slot++;
           }
@@ -1521,6 +1620,9 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
           }
         }
       }
+      // the k positions are filled (k < visible entries): one coalesced write of the list
+      __syncthreads();
+      for (int j = tid; j < k; j += TK_THREADS) out[j] = int32_t(S.wh[j]);
       return;
     }
   }
