@@ -1088,6 +1088,7 @@ struct alignas(16) GmShared {
   uint32_t wc[GM_WWORDS];        // the same over the candidate keys
   uint32_t pent[GM_POOL][GM_G];  // candidates of the pooled groups: key << 4 | position
   uint32_t pcnt[GM_POOL];        // and their number
+  uint16_t pgrp[GM_POOL];        // and the group of each slot
   uint32_t ncand;                // candidate keys in the row
   uint32_t npool;                // pool slots asked for
   uint32_t wcnt[TK_WARPS][16];   // per-warp digit counts of one radix pass
@@ -1460,44 +1461,47 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
     pbase = ndm ? atomicAdd(&S.npool, ndm) : 0u;
     if (ndm && pbase + ndm <= GM_POOL) {
       uint32_t sl = pbase;
-      for (uint32_t mm = dm; mm; mm &= mm - 1u, sl++) {
-        const int e0 = GM_G * (g0 + __ffs(mm) - 1);
-        if (al && e0 + GM_G <= nvis) {
-          cp_async16(&S.praw[sl][0], sr + e0);
-          cp_async16(&S.praw[sl][4], sr + e0 + 8);
-        } else {
-#pragma unroll
-          for (int w = 0; w < 8; w++)
-            S.praw[sl][w] = uint32_t(sr[min(e0 + 2 * w, nvis - 1)]) |
-                            (uint32_t(sr[min(e0 + 2 * w + 1, nvis - 1)]) << 16);
-        }
-      }
-      cp_async_commit();
-      cp_async_wait<0>();
-      sl = pbase;
-      for (uint32_t mm = dm; mm; mm &= mm - 1u, sl++) {
-        // keys of the group in place, the mask of those >= L among the visible ones, then
-        // one pass over the set bits
-        const int nv = nvis - GM_G * (g0 + __ffs(mm) - 1);
-        uint32_t msk = 0u;
-#pragma unroll
-        for (int w = 0; w < 8; w++) {
-          const uint32_t kk = ordered_key_bf16x2(S.praw[sl][w]);
-          S.praw[sl][w] = kk;
-          msk |= (uint32_t((kk & 0xFFFFu) >= L1) | (uint32_t((kk >> 16) >= L1) << 1)) << (2 * w);
-        }
-        if (nv < GM_G) msk &= (1u << nv) - 1u;
-        uint32_t n = 0;
-        for (; msk; msk &= msk - 1u) {
-          const int j = __ffs(msk) - 1;
-          const uint32_t key = (S.praw[sl][j >> 1] >> ((j & 1) * 16)) & 0xFFFFu;
-          S.pent[sl][n++] = (key << 4) | uint32_t(j);
-          if (inwin) atomicAdd(&S.wc[(key - wb) >> 1], 1u << (((key - wb) & 1) << 4));
-        }
-        S.pcnt[sl] = n;
-        c += n;
-      }
+      for (uint32_t mm = dm; mm; mm &= mm - 1u, sl++) S.pgrp[sl] = uint16_t(g0 + __ffs(mm) - 1);
     }
+    __syncthreads();
+    // the pooled groups (two or more candidates) one per thread: all their score loads in
+    // flight together, the keys >= L listed in the slot and counted in the window histogram
+    if (S.npool <= (uint32_t)GM_POOL && tid < (int)S.npool) {
+      const int sl = tid;
+      const int e0 = GM_G * int(S.pgrp[sl]);
+      uint32_t kw[8];
+      if (al && e0 + GM_G <= nvis) {
+        const uint4 a = *reinterpret_cast<const uint4*>(sr + e0);
+        const uint4 b2 = *reinterpret_cast<const uint4*>(sr + e0 + 8);
+        kw[0] = a.x; kw[1] = a.y; kw[2] = a.z; kw[3] = a.w;
+        kw[4] = b2.x; kw[5] = b2.y; kw[6] = b2.z; kw[7] = b2.w;
+      } else {
+#pragma unroll
+        for (int w = 0; w < 8; w++)
+          kw[w] = uint32_t(sr[min(e0 + 2 * w, nvis - 1)]) |
+                  (uint32_t(sr[min(e0 + 2 * w + 1, nvis - 1)]) << 16);
+      }
+      const int nv = nvis - e0;
+      uint32_t msk = 0u;
+#pragma unroll
+      for (int w = 0; w < 8; w++) {
+        kw[w] = ordered_key_bf16x2(kw[w]);
+        msk |= (uint32_t((kw[w] & 0xFFFFu) >= L1) | (uint32_t((kw[w] >> 16) >= L1) << 1)) << (2 * w);
+      }
+      if (nv < GM_G) msk &= (1u << nv) - 1u;
+      uint32_t n = 0;
+#pragma unroll
+      for (int j = 0; j < GM_G; j++) {
+        if (!((msk >> j) & 1u)) continue;
+        const uint32_t key = (kw[j >> 1] >> ((j & 1) * 16)) & 0xFFFFu;
+        S.pent[sl][n++] = (key << 4) | uint32_t(j);
+        if (inwin) atomicAdd(&S.wc[(key - wb) >> 1], 1u << (((key - wb) & 1) << 4));
+      }
+      S.pcnt[sl] = n;
+    }
+    __syncthreads();
+    if (ndm && pbase + ndm <= GM_POOL)
+      for (uint32_t sl = pbase; sl < pbase + ndm; sl++) c += S.pcnt[sl];
     c_own = c;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);

@@ -310,6 +310,8 @@ def hcl_kv(data, scale=None, rope=None):
     (1, 1, 8, 1024, 64, 64, False, False),      # cfg-1 shape
     (2, 1, 64, 5000, 512, 128, False, True),    # split-KV + sink
     (2, 1, 128, 9000, 1024, 128, True, False),  # cfg-4 shape, FP8 split rows
+    (2, 1, 100, 5000, 512, 128, True, True),    # heads over two blocks: slices of 64 and 36
+    (3, 1, 72, 4000, 300, 64, False, False),    # slices of 64 and 8
     (1, 3, 16, 700, 100, 37, False, False),     # ragged list, several queries
     (2, 2, 128, 3000, 64, 0, True, True),       # no window
     (1, 1, 128, 9000, 4096, 128, True, True),   # long list: splits merged via the workspace
