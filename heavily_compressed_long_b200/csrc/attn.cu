@@ -58,7 +58,6 @@ struct AttnParams {
   int G, n_groups, splits, cps, rows_pad;
   int cmerge;  // 1: the splits of a group form one cluster and merge through DSMEM
   int hsplit;  // blocks sharing one group's (query, head) rows (cluster merge only)
-  int tch;     // tcgen05 decode: heads per block (a block per slice of tch heads)
   int prewait; // 1: q, q_pos and the raw window store are not written by the previous kernel in
                // the stream, so they may be read before waiting for it (fused decode step only)
   int32_t* status;
@@ -652,11 +651,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
   const int row = tid & (TC_ROWS - 1);   // head row = TMEM lane (warps w and w+4 share a quadrant)
   const int hc = tid / TC_ROWS;          // which half of the columns this thread handles
   const int split = blockIdx.x % p.splits;
-  // block = (sequence, slice of p.tch heads, split): head h0 + r lives in TMEM lane r < nh
-  const int nhs = (p.H + p.tch - 1) / p.tch;
-  const int b = blockIdx.x / p.splits / nhs;
-  const int h0 = (blockIdx.x / p.splits % nhs) * p.tch;
-  const int nh = min(p.tch, p.H - h0);
+  const int b = blockIdx.x / p.splits;
   const TcOff off = tc_offsets(p.cps, p.splits);
   uint8_t* sQ = sm + off.q;
   uint64_t* bar_s = reinterpret_cast<uint64_t*>(sm + off.bar);
@@ -679,8 +674,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
   // splits > 1: the partials of this block's head rows arrive by bulk copies, counted on
   // bar_r: S copies of rows_o rows of 512 bytes (rows_o = this block's rows, see the push)
   uint64_t* bar_r = bar_s + 3;
-  const int rpo = p.splits > 1 ? (nh + p.splits - 1) / p.splits : 1;
-  auto rows_of = [&](int o) { return max(0, min(rpo, nh - o * rpo)); };
+  const int rpo = p.splits > 1 ? (TC_ROWS + p.splits - 1) / p.splits : 1;
+  auto rows_of = [&](int o) { return max(0, min(rpo, p.H - o * rpo)); };
   if (tid == 0) {
     mbar_init(bar_s, 1);
     mbar_init(bar_o, 1);
@@ -704,10 +699,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
 
   // Q: thread (row, hc) loads dims 64*hc .. 64*hc+63 of head `row` into SW128 half hc
   {
-    const uint4* src = reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.H + h0 + min(row, nh - 1)) * D) + hc * 8;
+    const uint4* src = reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.H + row) * D) + hc * 8;
     uint4 qv[8];
 #pragma unroll
-    for (int c = 0; c < 8; c++) qv[c] = row < nh ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    for (int c = 0; c < 8; c++) qv[c] = row < p.H ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
     if (p.q_gamma != nullptr) {
       // RMSNorm of the head's query row [Tripbot §5]: the two threads of a row add their
       // halves' sums of squares through shared memory; fp32, rounded back to bf16
@@ -915,10 +910,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
     }
     lsum += f2_lo(ls2) + f2_hi(ls2);
   };
-  if ((row & ~31) >= nh) {
-    // a warp without heads: its P rows are left as they are (an output row depends on its
-    // own P row only); warp-uniform, as the TMEM loads below are warp-collective
-  } else if (inreg) {
+  if (inreg) {
 #pragma unroll
     for (int c = 0; c < 2; c++)
       if (c < nch) emit_p(c, sv[c]);
@@ -957,7 +949,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
   tc_fence_after();
 
   // output dims 64*hc .. 64*hc+63 of head `row`: normalised partial (o, lse) or the output
-  const bool hv = row < nh;
+  const bool hv = row < p.H;
   float m2 = mrow, l2 = xch[TC_THREADS + row] + xch[TC_THREADS + row + TC_ROWS];
   const float inv_l = l2 > 0.f ? 1.f / l2 : 0.f;
   // splits > 1: row r is merged by block r / rpo (contiguous head blocks) in its slot r % rpo;
@@ -973,7 +965,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
   }
   float f = inv_l;
   if (p.splits == 1 && p.sink) {
-    const float s2 = p.sink[h0 + min(row, nh - 1)] * LOG2E;
+    const float s2 = p.sink[min(row, p.H - 1)] * LOG2E;
     const float mm = fmaxf(m2, s2);
     const float fa = l2 > 0.f ? exp2f(m2 - mm) : 0.f;
     const float l3 = l2 * fa + exp2f(s2 - mm);
@@ -1001,7 +993,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
       }
     } else if (hv) {
       {
-        __nv_bfloat16* dst = p.out + ((size_t)b * p.H + h0 + row) * D + hc * 64;
+        __nv_bfloat16* dst = p.out + ((size_t)b * p.H + row) * D + hc * 64;
 #pragma unroll
         for (int i = 0; i < 64; i += 8) {
           reinterpret_cast<uint4*>(dst + i)[0] =
@@ -1027,7 +1019,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
     }
   }
   if (p.splits == 1 && hv && hc == 0 && p.lse)
-    p.lse[(size_t)b * p.H + h0 + row] = l2 > 0.f ? (m2 + log2f(l2)) * LN2 : -INFINITY;
+    p.lse[(size_t)b * p.H + row] = l2 > 0.f ? (m2 + log2f(l2)) * LN2 : -INFINITY;
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -1043,8 +1035,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
     cluster.sync();
     const int S = p.splits;
     for (int slot = warp; slot < rpo; slot += TC_THREADS / 32) {
-      if (split * rpo + slot >= nh) break;
-      const int h = h0 + split * rpo + slot;
+      const int h = split * rpo + slot;
+      if (h >= p.H) break;
       const float ls = lane < S ? recv_lse[slot * S + lane] : -INFINITY;
       float M = ls;
 #pragma unroll
@@ -1201,7 +1193,7 @@ hcl_status_t launch_tc(const AttnParams& p, cudaStream_t st) {
   attr[1].val.clusterDim.x = p.splits;
   attr[1].val.clusterDim.y = 1;
   attr[1].val.clusterDim.z = 1;
-  cfg.gridDim = dim3((unsigned)(p.B * ((p.H + p.tch - 1) / p.tch) * p.splits));
+  cfg.gridDim = dim3((unsigned)(p.B * p.splits));
   cfg.blockDim = dim3(TC_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -1249,9 +1241,6 @@ hcl_status_t launch_attn(const AttnArgs& a, void* ws, size_t ws_bytes, cudaStrea
   p.rows_pad = pl.rows_pad;
   p.cmerge = pl.cmerge;
   p.hsplit = pl.hsplit;
-  // tcgen05 decode: more than 64 heads go to two blocks per split (half the exponentials and
-  // half the partial rows per block, twice the blocks); a function of H only
-  p.tch = a.H > 64 ? 64 : a.H;
   p.prewait = a.prewait;
   p.status = a.status;
   p.ws_o = nullptr;
