@@ -637,7 +637,7 @@ __host__ __device__ inline TcOff tc_offsets(int cps, int splits) {
   o.recv = o.xch + 2 * TC_THREADS * 4;       // cluster merge: splits x rpo x D fp16 partials
   const int rpo = splits > 1 ? (TC_ROWS + splits - 1) / splits : 0;
   o.lse = o.recv + (uint32_t)(rpo * splits * D * 2);
-  o.total = o.lse + (uint32_t)(rpo * splits * 4);
+  o.total = o.lse + (uint32_t)(((rpo + 3) & ~3) * splits * 4);   // [splits][rpo rounded to 4]
   return o;
 }
 
@@ -675,13 +675,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
   // bar_r: S copies of rows_o rows of 512 bytes (rows_o = this block's rows, see the push)
   uint64_t* bar_r = bar_s + 3;
   const int rpo = p.splits > 1 ? (TC_ROWS + p.splits - 1) / p.splits : 1;
+  const int rpo4 = (rpo + 3) & ~3;                          // log-sum-exps per split, 16-byte rows
   auto rows_of = [&](int o) { return max(0, min(rpo, p.H - o * rpo)); };
   if (tid == 0) {
     mbar_init(bar_s, 1);
     mbar_init(bar_o, 1);
     if (p.splits > 1) {
       mbar_init(bar_r, 1);
-      mbar_arrive_expect_tx(bar_r, uint32_t(p.splits * rows_of(split) * D * 2));
+      mbar_arrive_expect_tx(bar_r, rows_of(split) > 0
+                                       ? uint32_t(p.splits * (rows_of(split) * D * 2 + rpo4 * 4))
+                                       : 0u);
     }
     fence_barrier_init();
   }
@@ -958,11 +961,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
   // idle) KV tiles, XOR-swizzled in 16-byte chunks, and block o's rows then go to it as one
   // bulk copy
   uint8_t* stage = sm + off.kv;                   // 128 rows x 256 B (KV tiles, cps == 2)
-  if (p.splits > 1 && hv && hc == 0) {
-    cg::cluster_group cluster = cg::this_cluster();
-    *(cluster.map_shared_rank(recv_lse, row / rpo) + (row % rpo) * p.splits + split) =
-        l2 > 0.f ? m2 + log2f(l2) : -INFINITY;
-  }
+  float* stage_lse = reinterpret_cast<float*>(sm + off.pm);   // [owner][rpo4] (P tiles)
+  if (p.splits > 1 && hv && hc == 0)
+    stage_lse[(row / rpo) * rpo4 + row % rpo] = l2 > 0.f ? m2 + log2f(l2) : -INFINITY;
   float f = inv_l;
   if (p.splits == 1 && p.sink) {
     const float s2 = p.sink[min(row, p.H - 1)] * LOG2E;
@@ -1012,10 +1013,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
       // block o receives rows o*rpo .. o*rpo + rows_of(o) - 1 at recv[split][slot][D], still
       // swizzled (chunk c of row r at c ^ (r & 7))
       for (int o = 0; o < p.splits; o++)
-        if (rows_of(o) > 0)
+        if (rows_of(o) > 0) {
           bulk_copy_to_cluster(cluster_map(recv_h + (size_t)split * rpo * D, o),
                                stage + (size_t)o * rpo * 256, uint32_t(rows_of(o) * 256),
                                cluster_map(bar_r, o));
+          bulk_copy_to_cluster(cluster_map(recv_lse + (size_t)split * rpo4, o),
+                               stage_lse + (size_t)o * rpo4, uint32_t(rpo4 * 4),
+                               cluster_map(bar_r, o));
+        }
     }
   }
   if (p.splits == 1 && hv && hc == 0 && p.lse)
@@ -1027,56 +1032,69 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
     tmem_dealloc(tbase, ncols);
   }
   if (p.splits > 1) {
-    // merge the rows this block owns (row r -> block r / rpo, slot r % rpo).  Once its own
-    // copies have all landed (bar_r), a block's outgoing copies have been read too when every
-    // block has passed the cluster barrier, which also publishes the log-sum-exps.
+    // merge the rows this block owns (row r -> block r / rpo, slot r % rpo) once its own
+    // copies (partials and log-sum-exps) have landed (bar_r).  Every block arrives on the
+    // cluster barrier after that and waits on it only before exiting: when it passes, every
+    // block's copies out of this block's shared memory have been received
     if (!mbar_wait(bar_r, 0, limit, nullptr)) report(p.status, HCL_ERR_TIMEOUT);
-    cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
+    asm volatile("barrier.cluster.arrive.aligned;" ::: "memory");
     const int S = p.splits;
-    for (int slot = warp; slot < rpo; slot += TC_THREADS / 32) {
+    // two heads per warp, one per 16-lane half: lane hl holds dims 8 hl .. 8 hl + 7 (16-byte
+    // chunk hl of the row, stored at chunk hl ^ (h & 7)) and, for hl < S, split hl's weight
+    const int hl = lane & 15, hb = lane & 16;
+    for (int slot0 = 2 * warp; slot0 < rpo; slot0 += 2 * (TC_THREADS / 32)) {
+      const int slot = min(slot0 + (lane >> 4), rpo - 1);
       const int h = split * rpo + slot;
-      if (h >= p.H) break;
-      const float ls = lane < S ? recv_lse[slot * S + lane] : -INFINITY;
+      const bool act = slot0 + (lane >> 4) < rpo && h < p.H;
+      const float ls = (act && hl < S) ? recv_lse[hl * rpo4 + slot] : -INFINITY;
       float M = ls;
 #pragma unroll
-      for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
+      for (int o2 = 8; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
       float s2 = -INFINITY;
       if (p.sink) {
-        s2 = p.sink[h] * LOG2E;
+        s2 = p.sink[min(h, p.H - 1)] * LOG2E;
         M = fmaxf(M, s2);
       }
       const float wl = (ls == -INFINITY || M == -INFINITY) ? 0.f : exp2f(ls - M);
       float den = wl;
 #pragma unroll
-      for (int o2 = 16; o2 > 0; o2 >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o2);
+      for (int o2 = 8; o2 > 0; o2 >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o2);
       if (p.sink && M > -INFINITY) den += exp2f(s2 - M);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      // lane l: dims 4l .. 4l+3 = half l & 1 of 16-byte chunk l / 2, as swizzled
-      const uint8_t* part = reinterpret_cast<const uint8_t*>(recv_h + (size_t)slot * D) +
-                            ((((lane >> 1) ^ (h & 7)) << 4) | ((lane & 1) << 3));
+      const uint8_t* part =
+          reinterpret_cast<const uint8_t*>(recv_h + (size_t)slot * D) + ((hl ^ (h & 7)) << 4);
       // every split's partial loaded up front (independent loads), then summed in split order
       // (a zero weight adds 0 * v = 0: the partials are finite)
-      uint2 hv2[MAX_CLUSTER_ROWS];
+      uint4 hv4[MAX_CLUSTER_ROWS];
 #pragma unroll
       for (int s = 0; s < MAX_CLUSTER_ROWS; s++)
-        hv2[s] = s < S ? *reinterpret_cast<const uint2*>(part + (size_t)s * rpo * D * 2)
-                       : make_uint2(0u, 0u);
+        hv4[s] = (act && s < S) ? *reinterpret_cast<const uint4*>(part + (size_t)s * rpo * D * 2)
+                                : make_uint4(0u, 0u, 0u, 0u);
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; i++) acc[i] = 0.f;
 #pragma unroll
       for (int s = 0; s < MAX_CLUSTER_ROWS; s++) {
-        const float wgt = __shfl_sync(0xffffffffu, wl, s);
+        const float wgt = __shfl_sync(0xffffffffu, wl, hb | s);
         if (s < S) {
-          const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&hv2[s].x));
-          const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&hv2[s].y));
-          acc.x += wgt * lo.x; acc.y += wgt * lo.y; acc.z += wgt * hi.x; acc.w += wgt * hi.y;
+          const uint32_t w4[4] = {hv4[s].x, hv4[s].y, hv4[s].z, hv4[s].w};
+#pragma unroll
+          for (int i = 0; i < 4; i++) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[i]));
+            acc[2 * i] += wgt * f.x;
+            acc[2 * i + 1] += wgt * f.y;
+          }
         }
       }
       const float inv = den > 0.f ? 1.f / den : 0.f;
       const size_t orow = (size_t)b * p.H + h;
-      reinterpret_cast<uint2*>(p.out + orow * D)[lane] =
-          make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
-      if (p.lse && lane == 0) p.lse[orow] = den > 0.f ? (M + log2f(den)) * LN2 : -INFINITY;
+      if (act) {
+        reinterpret_cast<uint4*>(p.out + orow * D)[hl] =
+            make_uint4(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv),
+                       pack_bf16(acc[4] * inv, acc[5] * inv), pack_bf16(acc[6] * inv, acc[7] * inv));
+        if (p.lse && hl == 0) p.lse[orow] = den > 0.f ? (M + log2f(den)) * LN2 : -INFINITY;
+      }
     }
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
   }
 }
 

@@ -10,16 +10,17 @@
 // queries x H heads = up to 128 (query, head) rows = the UMMA M dimension = 128 TMEM lanes, two
 // threads per row.  The group's KV list is the visible-entry prefix of its last query followed
 // by the union of its queries' windows; it is processed in rounds of 64 rows.  A round's rows
-// are gathered with cp.async into one of two KV buffers (4 threads per row, each resolving the
+// are gathered with cp.async into one of three KV buffers (4 threads per row, each resolving the
 // row's store slot; split FP8 rows widened to bf16 with their scale), so the gather of round
-// r + 1 is in flight while round r runs S = Q K^T (N = 64) into TMEM, its softmax and
+// r + 1, issued right after round r's S, is in flight while round r runs S = Q K^T (N = 64)
+// into TMEM, its softmax and
 // O += P V (V read as the MN-major operand of the same SW128 tile; O accumulates in TMEM
 // across all rounds).  The softmax runs in registers with each row's own causal mask (for
 // query q: the list rows [0, visible entries of q) and the window rows of q -- two index
 // intervals, turned into bit masks; full 32-column words skip the per-column selects), its
 // probabilities taken against a reference maximum that is raised only when the row maximum
 // grows by more than 2^8, and only then is O rescaled in TMEM (load, scale, store).  Paired
-// fp32 instructions form the exponents and sums.  Two blocks fit per SM (about 92 KB of
+// fp32 instructions form the exponents and sums.  Two blocks fit per SM (about 113 KB of
 // shared memory, 256 TMEM columns each), so one block's softmax overlaps the other's MMAs.
 //
 // CSA prefill (every query has its own selection) uses the same kernel with G = 128 / H
@@ -63,16 +64,18 @@ struct FaParams {
   long long limit;
 };
 
+constexpr int FA_NBUF = 3;       // KV buffers: round r + 1 gathers while r and r - 1 are read
 struct FaOff {
   static constexpr uint32_t Q = 0;                          // 2 halves x 128 rows x 128 B
-  static constexpr uint32_t KV = 32768;                     // 2 buffers x (2 halves x 64 rows x 128 B)
-  static constexpr uint32_t P = KV + 2 * 16384;             // 128 rows x 64 bf16
-  static constexpr uint32_t STG = P + 16384;                // 2 buffers x 64 rows x 64 B codes
-  static constexpr uint32_t SCL = STG + 2 * 4096;           // 2 buffers x 64 scales
-  static constexpr uint32_t XCH = SCL + 2 * 256;            // 2 x 256 floats
+  static constexpr uint32_t KV = 32768;                     // FA_NBUF x (2 halves x 64 rows x 128 B)
+  static constexpr uint32_t P = KV + FA_NBUF * 16384;       // 128 rows x 64 bf16
+  static constexpr uint32_t STG = P + 16384;                // FA_NBUF x 64 rows x 64 B codes
+  static constexpr uint32_t SCL = STG + FA_NBUF * 4096;     // FA_NBUF x 64 scales
+  static constexpr uint32_t XCH = SCL + FA_NBUF * 256;      // 2 x 256 floats
   static constexpr uint32_t BAR = XCH + 2 * FA_THREADS * 4; // 2 mbarriers, TMEM base, row bits
   static constexpr uint32_t TOTAL = BAR + 64;
 };
+static_assert(2 * (FaOff::TOTAL + 2048) <= 233472, "two blocks per SM");
 
 // Rescale O only when the running maximum grows by more than this (log2 units): until then the
 // probabilities are taken against the stale maximum (values <= 2^8, exact in fp32 sums).
@@ -201,7 +204,7 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
   const uint32_t tbase = *sTmem;
   const uint32_t ocol = FA_CH;                             // S: columns 0..63, O: 64..191
   const uint32_t trow = tbase + (uint32_t((warp & 3) * 32) << 16);
-  uint8_t* rb8 = sm + FaOff::BAR + 32;                     // [2 buffers][8 bytes]: row validity
+  uint8_t* rb8 = sm + FaOff::BAR + 24;                     // [FA_NBUF][8 bytes]: row validity
   const int nrounds = (total + FA_CH - 1) / FA_CH;
 
   // gather of list rows [r0, r0 + 64) into buffer `buf`: 4 threads per row, each resolving the
@@ -281,7 +284,7 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
   const unsigned long long c2x2 = f2_make(c2, c2);
   if (nrounds > 0) gather(0, 0);
   for (int rd = 0; rd < nrounds; rd++) {
-    const int buf = rd & 1, r0 = rd * FA_CH, nr = min(FA_CH, total - r0);
+    const int buf = rd % FA_NBUF, r0 = rd * FA_CH, nr = min(FA_CH, total - r0);
     cp_async_wait<0>();                                    // gather(rd), this thread's copies
     __syncthreads();
     if (KVFMT == HCL_FP8SPLIT) {
@@ -315,10 +318,11 @@ __global__ void __launch_bounds__(FA_THREADS, 2) hca_flash_kernel(FaParams p) {
       umma_commit(bar_s);
     }
     __syncwarp();   // warp 0 reconverges before waiting (the issuing lane is not left behind)
-    // the previous round's PV has finished reading the other buffer (and P, and writing O):
-    // the next gather may start, overlapping this round's MMAs and softmax
-    if (rd > 0) ok = ok && mbar_wait(bar_o, (rd - 1) & 1, p.limit, nullptr);
-    if (rd + 1 < nrounds) gather(rd + 1, buf ^ 1);
+    // the next round's rows go into the buffer the PV two rounds back read (finished: this
+    // block saw the S after it complete), while this round's S and the previous PV run
+    if (rd + 1 < nrounds) gather(rd + 1, (rd + 1) % FA_NBUF);
+    // S completes after every earlier MMA of this thread: the previous PV has finished reading
+    // P and its KV buffer and writing O
     ok = ok && mbar_wait(bar_s, rd & 1, p.limit, nullptr);
     tc_fence_after();
     // this thread's 32 columns of the round
