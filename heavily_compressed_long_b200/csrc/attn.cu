@@ -1055,11 +1055,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
         s2 = p.sink[min(h, p.H - 1)] * LOG2E;
         M = fmaxf(M, s2);
       }
-      const float wl = (ls == -INFINITY || M == -INFINITY) ? 0.f : exp2f(ls - M);
+      const float wl = (ls == -INFINITY || M == -INFINITY) ? 0.f : ex2_ftz(ls - M);
       float den = wl;
 #pragma unroll
       for (int o2 = 8; o2 > 0; o2 >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o2);
-      if (p.sink && M > -INFINITY) den += exp2f(s2 - M);
+      if (p.sink && M > -INFINITY) den += ex2_ftz(s2 - M);
       const uint8_t* part =
           reinterpret_cast<const uint8_t*>(recv_h + (size_t)slot * D) + ((hl ^ (h & 7)) << 4);
       // every split's partial loaded up front (independent loads), then summed in split order
@@ -1085,13 +1085,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(AttnParams p) {
           }
         }
       }
-      const float inv = den > 0.f ? 1.f / den : 0.f;
+      const float inv = den > 0.f ? __fdividef(1.f, den) : 0.f;
       const size_t orow = (size_t)b * p.H + h;
       if (act) {
         reinterpret_cast<uint4*>(p.out + orow * D)[hl] =
             make_uint4(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv),
                        pack_bf16(acc[4] * inv, acc[5] * inv), pack_bf16(acc[6] * inv, acc[7] * inv));
-        if (p.lse && hl == 0) p.lse[orow] = den > 0.f ? (M + log2f(den)) * LN2 : -INFINITY;
+        if (p.lse && hl == 0) p.lse[orow] = den > 0.f ? (M + __log2f(den)) * LN2 : -INFINITY;
       }
     }
     asm volatile("barrier.cluster.wait.aligned;" ::: "memory");

@@ -377,7 +377,8 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
       }
       // Drain: every issued copy has landed before the block may exit.
       for (int i = max(0, issued - STAGES); i < issued; i++)
-        mbar_wait(&full[i % STAGES], (i / STAGES) & 1, p.limit, nullptr);
+        if (!mbar_wait(&full[i % STAGES], (i / STAGES) & 1, p.limit, nullptr))
+          report(p.status, HCL_ERR_TIMEOUT);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -460,7 +461,7 @@ __global__ void __launch_bounds__(64 + 32 * EPI, 1)
     }
     if (lane == 0) umma_commit(drain);
     __syncwarp();
-    mbar_wait(drain, 0, p.limit, nullptr);
+    if (!mbar_wait(drain, 0, p.limit, nullptr) && lane == 0) report(p.status, HCL_ERR_TIMEOUT);
   } else {
     // ---------------- epilogue ----------------
     // EPI/4 groups of four warps (one warp per TMEM lane quarter) split the tile's queries

@@ -191,14 +191,23 @@ def test_cfg4_csa_1m_mxfp4_fp8(hcl):
         assert np.abs(as_f64(pipe.out[sl]) - o_ref).max() <= 5e-2
         assert np.abs(as_f64(pipe.lse[sl]) - l_ref).max() <= 5e-2
     assert pipe.status.item() == 0
-    # the fused C-ABI decode step (q_I quantised inside the indexer; selection and attention
-    # in one cluster kernel): the same selection bit for bit, and its attention against the
-    # oracle on every sequence
+    # the fused C-ABI decode step (q_I quantised inside the indexer, the top-k from its group
+    # summaries): the same selection bit for bit, and its attention against the oracle on
+    # every sequence.  Repeated steps on the same workspace must give the same bits.
     idx1 = pipe.idx.clone()
     pipe.idx.fill_(-7)
     pipe.step()
     torch.cuda.synchronize()
     assert torch.equal(idx1, pipe.idx)
+    assert pipe.status.item() == 0
+    out1, lse1 = pipe.out.clone(), pipe.lse.clone()
+    for _ in range(3):
+        pipe.idx.fill_(-7)
+        pipe.out.zero_()
+        pipe.step()
+        torch.cuda.synchronize()
+        assert torch.equal(idx1, pipe.idx)
+        assert torch.equal(out1, pipe.out) and torch.equal(lse1, pipe.lse)
     assert pipe.status.item() == 0
     for b in range(B):
         sl = slice(b, b + 1)
