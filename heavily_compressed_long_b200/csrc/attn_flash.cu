@@ -471,6 +471,411 @@ hcl_status_t launch_flash_t(const FaParams& p, cudaStream_t st) {
                     "hca flash attention launch");
 }
 
+
+// ---------------------------------------------------------------------------------------
+// HCA prefill, warp-specialised: two query tiles per block share the KV rounds.
+//
+// Block = (sequence, pair of query groups): tile t in {0, 1} holds group 2 * pair + t (up to
+// 128 (query, head) rows each).  The pair's KV list is the visible-entry prefix of its last
+// query plus the union of its queries' windows, in rounds of 64 rows.  Warps 0..3 and 4..7
+// are the softmax warpgroups of tiles 0 and 1 (one thread per row, the row's 64 columns of a
+// round in registers, no exchange between threads); warps 8 and 9 gather the rounds' rows
+// with cp.async into a ring of three KV buffers (one row per thread); one thread of warp 11
+// issues every MMA from descriptors built once.  The MMA
+// issue order S_0(r+1), PV_0(r), S_1(r+1), PV_1(r) lets one tile's softmax run while the tensor
+// pipe works on the other tile, and each S_t(r+1) as soon as tile t's softmax has read S_t(r).
+// TMEM: S_0, S_1 (64 columns each), O_0, O_1 (128 each) -- 512 columns, one block per SM.
+//
+//   kv_full[b]  (64 gather threads)   round rows landed in buffer b (copies done, proxy-fenced)
+//   kv_empty[b] (MMA commit)          both tiles' PV of the buffer's round completed
+//   s_full[t]   (MMA commit)          S_t of the round in TMEM
+//   s_free[t]   (128 softmax threads) S_t read into registers
+//   p_full[t]   (128 softmax threads) P_t in shared memory (and O_t rescaled)
+//   o_done[t]   (MMA commit)          PV_t of the round completed (P_t free, O_t stable)
+// Every wait is bounded; a timeout sets the block's abort flag and HCL_ERR_TIMEOUT.
+
+constexpr int WS_WARPS = 12;
+constexpr int WS_GATHER = 64;   // warps 8, 9 (warp 10 idles: warps are allocated in fours)
+constexpr int WS_THREADS = WS_WARPS * 32;
+constexpr int WS_NBUF = 3;
+struct WsOff {
+  static constexpr uint32_t Q = 0;                            // 2 tiles x 2 halves x 128 x 128 B
+  static constexpr uint32_t KV = 65536;                       // 3 x (2 halves x 64 rows x 128 B)
+  static constexpr uint32_t P = KV + WS_NBUF * 16384;         // 2 tiles x 128 rows x 128 B
+  static constexpr uint32_t BAR = P + 32768;                  // mbarriers
+  static constexpr int NBAR = 2 * WS_NBUF + 4 * 2 + 1;        // kv_full/empty, s/p/o x 2, drain
+  static constexpr uint32_t MISC = BAR + NBAR * 8;            // TMEM base, abort flag
+  static constexpr uint32_t TOTAL = MISC + 16;
+};
+static_assert(WsOff::TOTAL + 1024 <= 232448, "shared memory");
+
+__global__ void __launch_bounds__(WS_THREADS, 1) hca_flash_ws_kernel(FaParams p) {
+  extern __shared__ __align__(1024) uint8_t ws_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ws_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_pairs = (p.n_groups + 1) / 2;
+  const int pair = blockIdx.x % n_pairs, b = blockIdx.x / n_pairs;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + WsOff::BAR);
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = bars + WS_NBUF;
+  uint64_t* s_full = bars + 2 * WS_NBUF;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_full + 4;
+  uint64_t* o_done = s_full + 6;
+  uint64_t* drain = s_full + 8;
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + WsOff::MISC);
+  volatile int* sAbort = reinterpret_cast<volatile int*>(sm + WsOff::MISC + 4);
+  if (tid == 0) {
+    for (int i = 0; i < WS_NBUF; i++) { mbar_init(&kv_full[i], WS_GATHER); mbar_init(&kv_empty[i], 1); }
+    for (int t = 0; t < 2; t++) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&s_free[t], 128);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&o_done[t], 1);
+    }
+    mbar_init(drain, 1);
+    *sAbort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 11) {
+    tmem_alloc(sTmem, 512);
+    tmem_relinquish();
+  }
+  pdl_enter();
+
+  // the pair's queries [q_lo, q_hi) and its KV list: visible-entry prefix [0, n_a) of the last
+  // query, then window tokens raw_lo .. raw_lo + n_raw - 1
+  const int q_lo = 2 * pair * p.G, q_hi = min(p.Tq, q_lo + 2 * p.G);
+  int pmin = 0x7fffffff, pmax = -1;
+  for (int i = q_lo; i < q_hi; i++) {
+    const int pp = p.q_pos[(size_t)b * p.Tq + i];
+    pmin = min(pmin, pp);
+    pmax = max(pmax, pp);
+  }
+  const int n_a = pmax < 0 ? 0 : min(p.Nh, (pmax + 1) / p.mh);
+  const int raw_lo = pmin - p.W + 1;
+  const int n_raw = (p.W > 0 && pmax >= 0) ? max(0, pmax - raw_lo + 1) : 0;
+  const int total = n_a + n_raw;
+  const int nrounds = (total + FA_CH - 1) / FA_CH;
+
+  // softmax threads: this thread's tile, row, query and visibility intervals
+  const int t = (tid >> 7) & 1, row = tid & 127;
+  const int t0 = q_lo + t * p.G, gq = max(0, min(p.G, p.Tq - t0));
+  const int qi = row / p.H, hh = row % p.H;
+  const bool rv = warp < 8 && qi < gq;
+  int nv_e = 0, w_lo = 0, w_hi = 0;
+  if (rv) {
+    const int my_p = p.q_pos[(size_t)b * p.Tq + t0 + qi];
+    nv_e = my_p < 0 ? 0 : min(n_a, (my_p + 1) / p.mh);
+    if (my_p >= 0 && p.W > 0) {
+      const int u_lo = max(0, my_p - p.W + 1);
+      w_lo = n_a + (u_lo - raw_lo);
+      w_hi = n_a + (my_p - raw_lo) + 1;
+    }
+  }
+  if (warp < 8) {
+    // Q row (query t0 + qi, head hh) -> tile t's SW128 halves, optionally RMS-normalised
+    const uint4* src = reinterpret_cast<const uint4*>(
+        p.q + (((size_t)b * p.Tq + t0 + (rv ? qi : 0)) * p.H + hh) * FA_D);
+    uint4 qv[16];
+#pragma unroll
+    for (int i = 0; i < 16; i++) qv[i] = rv ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+    if (p.q_gamma != nullptr) {
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; i++) {
+        const uint32_t w4[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+          const float lo = __uint_as_float(w4[j] << 16), hi = __uint_as_float(w4[j] & 0xFFFF0000u);
+          ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+        }
+      }
+      const float rn = 1.f / sqrtf(ss / float(FA_D) + p.q_eps);
+#pragma unroll
+      for (int i = 0; i < 16; i++) {
+        uint32_t w4[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+          const int dim = i * 8 + 2 * j;
+          const float lo = __uint_as_float(w4[j] << 16), hi = __uint_as_float(w4[j] & 0xFFFF0000u);
+          w4[j] = fa_pack(lo * rn * __ldg(p.q_gamma + dim), hi * rn * __ldg(p.q_gamma + dim + 1));
+        }
+        qv[i] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
+    }
+    uint8_t* qt = sm + WsOff::Q + t * 32768;
+#pragma unroll
+    for (int i = 0; i < 16; i++)
+      *reinterpret_cast<uint4*>(qt + (i >> 3) * 16384 + row * 128 + (((i & 7) ^ (row & 7)) << 4)) = qv[i];
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *sTmem;
+
+  if (warp == 8 || warp == 9) {
+    // ---------------- gather: one list row per thread, 16 16-byte pieces ----------------
+    // a round is signalled as soon as its own copies have landed, so the MMA warp never waits
+    // for the gather of a later round
+    const int jj = tid - 256;
+    for (int rd = 0; rd < nrounds; rd++) {
+      const int buf = rd % WS_NBUF;
+      if (rd >= WS_NBUF && !mbar_wait(&kv_empty[buf], ((rd / WS_NBUF) & 1) ^ 1, p.limit, sAbort)) {
+        *sAbort = 1;
+        report(p.status, HCL_ERR_TIMEOUT);
+        break;
+      }
+      const int e = rd * FA_CH + jj;
+      long long slot = -1;
+      bool from_raw = false;
+      if (e < total) {
+        if (e < n_a) {
+          slot = (long long)b * p.comp.cap + (e < p.comp.cap ? e : e % p.comp.cap);
+        } else {
+          const int tok = raw_lo + (e - n_a);
+          if (tok >= 0) {
+            slot = (long long)b * p.raw.cap + (tok < p.raw.cap ? tok : tok % p.raw.cap);
+            from_raw = true;
+          }
+        }
+      }
+      const uint8_t* srow = static_cast<const uint8_t*>(from_raw ? p.raw.data : p.comp.data) +
+                            (slot < 0 ? 0 : slot) * 256;
+      uint8_t* dst = sm + WsOff::KV + buf * 16384 + jj * 128;
+#pragma unroll
+      for (int i = 0; i < 16; i++) {
+        uint8_t* d = dst + (i >> 3) * 8192 + (((i & 7) ^ (jj & 7)) << 4);
+        if (slot >= 0) cp_async16(d, srow + i * 16);
+        else *reinterpret_cast<uint4*>(d) = make_uint4(0, 0, 0, 0);
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      mbar_arrive(&kv_full[buf]);
+    }
+    cp_async_wait<0>();
+  } else if (warp == 11) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0 && nrounds > 0) {
+      // descriptors built once; a k-step moves the start address field (16-byte units)
+      const uint64_t dq = make_sdesc(smem_u32(sm + WsOff::Q), 16, 1024, SMEM_SWIZZLE_128B);
+      const uint64_t dk = make_sdesc(smem_u32(sm + WsOff::KV), 16, 1024, SMEM_SWIZZLE_128B);
+      const uint64_t dp = make_sdesc(smem_u32(sm + WsOff::P), 16, 1024, SMEM_SWIZZLE_128B);
+      const uint64_t dv = make_sdesc(smem_u32(sm + WsOff::KV), 8192, 1024, SMEM_SWIZZLE_128B);
+      constexpr uint32_t idS = idesc_bf16(128, FA_CH), idPV = idesc_bf16(128, FA_D) | (1u << 16);
+      auto issue_s = [&](int tt, int rd) {
+        const uint64_t a0 = dq + uint64_t(tt * (32768 >> 4));
+        const uint64_t b0 = dk + uint64_t((rd % WS_NBUF) * (16384 >> 4));
+#pragma unroll
+        for (int ks = 0; ks < 8; ks++) {
+          const uint32_t off_a = (ks >> 2) * (16384 >> 4) + (ks & 3) * 2;
+          const uint32_t off_b = (ks >> 2) * (8192 >> 4) + (ks & 3) * 2;
+          umma_bf16(tbase + tt * FA_CH, a0 + off_a, b0 + off_b, idS, ks > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[tt]);
+      };
+      auto issue_pv = [&](int tt, int rd) {
+        const uint64_t a0 = dp + uint64_t(tt * (16384 >> 4));
+        const uint64_t b0 = dv + uint64_t((rd % WS_NBUF) * (16384 >> 4));
+#pragma unroll
+        for (int ks = 0; ks < 4; ks++)
+          umma_bf16(tbase + 2 * FA_CH + tt * FA_D, a0 + uint32_t(ks * 2), b0 + uint32_t(ks * (2048 >> 4)),
+                    idPV, (rd > 0 || ks > 0) ? 1u : 0u);
+        umma_commit(&o_done[tt]);
+      };
+      bool ok = mbar_wait(&kv_full[0], 0, p.limit, sAbort);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+      }
+      for (int rd = 0; ok && rd < nrounds; rd++) {
+        for (int tt = 0; tt < 2 && ok; tt++) {
+          if (rd + 1 < nrounds) {
+            const int nb = (rd + 1) % WS_NBUF;
+            if (tt == 0) ok = mbar_wait(&kv_full[nb], ((rd + 1) / WS_NBUF) & 1, p.limit, sAbort);
+            ok = ok && mbar_wait(&s_free[tt], rd & 1, p.limit, sAbort);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(tt, rd + 1);
+          }
+          ok = mbar_wait(&p_full[tt], rd & 1, p.limit, sAbort);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(tt, rd);
+          if (tt == 1) umma_commit(&kv_empty[rd % WS_NBUF]);
+        }
+      }
+      if (!ok) {
+        *sAbort = 1;
+        report(p.status, HCL_ERR_TIMEOUT);
+      }
+      // every MMA issued has completed before TMEM may be freed
+      umma_commit(drain);
+      if (!mbar_wait(drain, 0, p.limit, nullptr)) report(p.status, HCL_ERR_TIMEOUT);
+    }
+    __syncwarp();
+  } else if (warp < 8) {
+    // ---------------- softmax of tile t: this thread's row ----------------
+    const uint32_t lq = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t tS = tbase + lq + t * FA_CH;
+    const uint32_t tO = tbase + lq + 2 * FA_CH + t * FA_D;
+    uint8_t* prow = sm + WsOff::P + t * 16384 + row * 128;
+    const float c2 = p.scale_log2;
+    const unsigned long long c2x2 = f2_make(c2, c2);
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int rd = 0; rd < nrounds; rd++) {
+      const int r0 = rd * FA_CH;
+      ok = mbar_wait(&s_full[t], rd & 1, p.limit, sAbort);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sv[64];
+      tmem_ld16(tS, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
+      tmem_ld16(tS + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+      tmem_ld16(tS + 32, *reinterpret_cast<uint32_t(*)[16]>(&sv[32]));
+      tmem_ld16(tS + 48, *reinterpret_cast<uint32_t(*)[16]>(&sv[48]));
+      uint32_t vb[2] = {0u, 0u};
+      if (rv) {
+#pragma unroll
+        for (int w = 0; w < 2; w++) {
+          const int c0 = r0 + 32 * w;
+          vb[w] = range_bits(c0, 0, nv_e) | range_bits(c0, w_lo, w_hi);
+        }
+      }
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&s_free[t]);
+      // row maximum of the raw scores over the valid columns (scale > 0)
+      float smax = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < 2; w++) {
+        if (vb[w] == 0xFFFFFFFFu) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 2)
+            smax = fmax3(smax, __uint_as_float(sv[32 * w + j]), __uint_as_float(sv[32 * w + j + 1]));
+        } else if (vb[w] != 0u) {
+#pragma unroll
+          for (int j = 0; j < 32; j++)
+            if ((vb[w] >> j) & 1u) smax = fmaxf(smax, __uint_as_float(sv[32 * w + j]));
+        }
+      }
+      const float m_cand = fmaxf(m_run, smax == -INFINITY ? -INFINITY : smax * c2);
+      const bool grow = m_cand > m_run + FA_RESCALE_LOG2;
+      const float m_new = grow ? m_cand : m_run;
+      const float alpha = (grow && m_run > -INFINITY) ? ex2_ftz(m_run - m_new) : 1.f;
+      const float muse = m_new == -INFINITY ? 0.f : m_new;
+      const unsigned long long negm = f2_make(-muse, -muse);
+      // the packed bf16 pair of columns j, j + 1 goes to sv[j / 2] (already consumed)
+      unsigned long long lr = 0ull;
+#pragma unroll
+      for (int j = 0; j < 64; j += 2) {
+        const unsigned long long x =
+            f2_fma(f2_make(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), c2x2, negm);
+        float p0 = ex2_ftz(f2_lo(x)), p1 = ex2_ftz(f2_hi(x));
+        const uint32_t bits = vb[j >> 5];
+        if (bits != 0xFFFFFFFFu) {
+          p0 = ((bits >> (j & 31)) & 1u) ? p0 : 0.f;
+          p1 = ((bits >> ((j + 1) & 31)) & 1u) ? p1 : 0.f;
+        }
+        lr = f2_add(lr, f2_make(p0, p1));
+        sv[j >> 1] = fa_pack(p0, p1);
+      }
+      // P_t and O_t belong to the previous round's PV until it completes
+      if (rd > 0) {
+        ok = mbar_wait(&o_done[t], (rd - 1) & 1, p.limit, sAbort);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+        for (int q8 = 0; q8 < 8; q8++) {
+          uint32_t r16[16];
+          tmem_ld16(tO + q8 * 16, r16);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; i++) r16[i] = __float_as_uint(__uint_as_float(r16[i]) * alpha);
+          tmem_st16(tO + q8 * 16, r16);
+        }
+        tmem_st_wait();
+      }
+#pragma unroll
+      for (int c = 0; c < 8; c++)
+        *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
+            make_uint4(sv[4 * c], sv[4 * c + 1], sv[4 * c + 2], sv[4 * c + 3]);
+      l_run = l_run * alpha + (f2_lo(lr) + f2_hi(lr));
+      m_run = m_new;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[t]);
+    }
+    if (ok && nrounds > 0) {
+      ok = mbar_wait(&o_done[t], (nrounds - 1) & 1, p.limit, sAbort);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (!ok) {
+      *sAbort = 1;
+      report(p.status, HCL_ERR_TIMEOUT);
+    }
+    tc_fence_after();
+    // epilogue: O / l (with the optional sink), bf16 rows, log-sum-exp
+    float l2 = l_run, m2 = m_run;
+    float f = l2 > 0.f ? 1.f / l2 : 0.f;
+    if (p.sink) {
+      const float s2 = p.sink[hh] * FA_LOG2E;
+      const float mm = fmaxf(m2, s2);
+      const float fa = l2 > 0.f ? exp2f(m2 - mm) : 0.f;
+      const float l3 = l2 * fa + exp2f(s2 - mm);
+      f = l3 > 0.f ? fa / l3 : 0.f;
+      l2 = l3;
+      m2 = mm;
+    }
+    const bool have_o = nrounds > 0 && ok;
+    const size_t orow = ((size_t)b * p.Tq + t0 + qi) * p.H + hh;
+#pragma unroll
+    for (int q8 = 0; q8 < 8; q8++) {
+      uint32_t r16[16];
+      tmem_ld16(tO + q8 * 16, r16);
+      tmem_ld_wait();
+      if (!have_o) {
+#pragma unroll
+        for (int i = 0; i < 16; i++) r16[i] = 0u;
+      }
+      if (rv) {
+        __nv_bfloat16* dst = p.out + orow * FA_D + q8 * 16;
+#pragma unroll
+        for (int i = 0; i < 16; i += 8)
+          *reinterpret_cast<uint4*>(dst + i) = make_uint4(
+              fa_pack(__uint_as_float(r16[i]) * f, __uint_as_float(r16[i + 1]) * f),
+              fa_pack(__uint_as_float(r16[i + 2]) * f, __uint_as_float(r16[i + 3]) * f),
+              fa_pack(__uint_as_float(r16[i + 4]) * f, __uint_as_float(r16[i + 5]) * f),
+              fa_pack(__uint_as_float(r16[i + 6]) * f, __uint_as_float(r16[i + 7]) * f));
+      }
+    }
+    if (rv && p.lse) p.lse[orow] = l2 > 0.f ? (m2 + log2f(l2)) * FA_LN2 : -INFINITY;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 11) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+hcl_status_t launch_flash_ws(const FaParams& p, cudaStream_t st) {
+  auto kern = hca_flash_ws_kernel;
+  const int smem = (int)WsOff::TOTAL + 1024;
+  hcl_status_t e = set_kernel_attrs(reinterpret_cast<const void*>(kern), smem, false);
+  if (e != HCL_OK) return e;
+  const long long n_pairs = (p.n_groups + 1) / 2;
+  return check_cuda(launch_pdl(kern, dim3((unsigned)((long long)p.B * n_pairs)),
+                               dim3(WS_THREADS), (size_t)smem, st, 1, p),
+                    "hca flash attention (warp-specialised) launch");
+}
+
 }  // namespace
 
 bool hca_flash_usable(const AttnArgs& a) {
@@ -504,6 +909,8 @@ hcl_status_t launch_hca_flash(const AttnArgs& a, cudaStream_t st) {
   p.lse = a.lse;
   p.status = a.status;
   p.limit = wait_limit_cycles();
+  // HCA over bf16 rows: two query tiles per block, warp-specialised
+  if (a.mode == 1 && a.comp.fmt == HCL_BF16 && a.raw.fmt == HCL_BF16) return launch_flash_ws(p, st);
   return a.comp.fmt == HCL_FP8SPLIT ? launch_flash_t<HCL_FP8SPLIT>(p, st) : launch_flash_t<HCL_BF16>(p, st);
 }
 

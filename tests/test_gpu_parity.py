@@ -402,6 +402,12 @@ def test_hca_attn_query_rmsnorm(hcl, Tq):
     (1, 261, 32, 128 * 33 + 100, 128, True, True),
     (1, 70, 64, 128 * 12, 200, False, True),
     (1, 40, 128, 128 * 4 + 9, 128, False, False),
+    # bf16 rows: two query groups per block (warp-specialised); an odd group count leaves the
+    # last block's second tile empty; a chunk at the start of the context (no visible entries
+    # for the first queries, windows reaching before token 0)
+    (3, 520, 16, 128 * 40 + 1, 128, False, False),
+    (1, 300, 16, 300, 128, False, True),
+    (1, 33 * 4, 32, 128 * 7 + 5, 64, False, False),
 ])
 def test_hca_attn(hcl, B, Tq, H, L, W, fp8, sink):
     d, mh = 128, 128
@@ -409,14 +415,16 @@ def test_hca_attn(hcl, B, Tq, H, L, W, fp8, sink):
     ent, raw = rbf16(B, Nh, d), rbf16(B, L, d)
     q = rbf16(B, Tq, H, d)
     pos = torch.arange(L - Tq, L, dtype=torch.int32).repeat(B, 1).contiguous()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
     sk = torch.from_numpy(RNG.standard_normal(H).astype(np.float32)) if sink else None
     okc, gkc, okr, gkr = _kv_pair(ent, raw, fp8)
     o_ref, l_ref = oracle.hca_attn(q, okc, Nh, mh, okr, W, pos, sink=sk)
     out = torch.empty(B, Tq, H, d, dtype=torch.bfloat16, device="cuda")
     lse = torch.empty(B, Tq, H, device="cuda")
     hcl.hcl_hca_dense_attn(cuda(q), gkc, Nh, mh, gkr, L, W, cuda(pos), out, lse=lse,
-                           sink=None if sk is None else cuda(sk))
+                           sink=None if sk is None else cuda(sk), status=status)
     torch.cuda.synchronize()
+    assert status.item() == 0
     tol = 5e-2 if fp8 else 2e-2
     assert np.abs(as_f64(out) - o_ref).max() <= tol
     assert np.abs(as_f64(lse) - l_ref).max() <= tol
