@@ -484,25 +484,41 @@ hcl_status_t launch_flash_t(const FaParams& p, cudaStream_t st) {
 // issues every MMA from descriptors built once.  The MMA
 // issue order S_0(r+1), PV_0(r), S_1(r+1), PV_1(r) lets one tile's softmax run while the tensor
 // pipe works on the other tile, and each S_t(r+1) as soon as tile t's softmax has read S_t(r).
-// TMEM: S_0, S_1 (64 columns each), O_0, O_1 (128 each) -- 512 columns, one block per SM.
+// The softmax writes P (bf16) into TMEM and PV reads it from there as its A operand, so the
+// MMAs' shared-memory traffic is Q, K and V only (an N = 64 MMA with both operands in shared
+// memory is bound by shared-memory bandwidth, and P stores would compete with it).
+// TMEM: S_0, S_1 (64 columns each), O_0, O_1 (128 each), P_0, P_1 (32 each) -- one block per SM.
 //
 //   kv_full[b]  (64 gather threads)   round rows landed in buffer b (copies done, proxy-fenced)
 //   kv_empty[b] (MMA commit)          both tiles' PV of the buffer's round completed
 //   s_full[t]   (MMA commit)          S_t of the round in TMEM
 //   s_free[t]   (128 softmax threads) S_t read into registers
-//   p_full[t]   (128 softmax threads) P_t in shared memory (and O_t rescaled)
+//   p_full[t]   (128 softmax threads) P_t in TMEM (and O_t rescaled)
 //   o_done[t]   (MMA commit)          PV_t of the round completed (P_t free, O_t stable)
 // Every wait is bounded; a timeout sets the block's abort flag and HCL_ERR_TIMEOUT.
+
+// D (+)= A B with A (M = 128 rows in the TMEM lanes, K packed two bf16 per column) read from
+// tensor memory and B from shared memory.
+__device__ __forceinline__ void umma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 
 constexpr int WS_WARPS = 12;
 constexpr int WS_GATHER = 64;   // warps 8, 9 (warp 10 idles: warps are allocated in fours)
 constexpr int WS_THREADS = WS_WARPS * 32;
 constexpr int WS_NBUF = 3;
+constexpr uint32_t WS_OCOL = 128;   // TMEM: S_0, S_1 at 0, 64; O_0, O_1 at 128, 256;
+constexpr uint32_t WS_PCOL = 384;   // P_0, P_1 (64 bf16 per row) at 384, 416
 struct WsOff {
   static constexpr uint32_t Q = 0;                            // 2 tiles x 2 halves x 128 x 128 B
   static constexpr uint32_t KV = 65536;                       // 3 x (2 halves x 64 rows x 128 B)
-  static constexpr uint32_t P = KV + WS_NBUF * 16384;         // 2 tiles x 128 rows x 128 B
-  static constexpr uint32_t BAR = P + 32768;                  // mbarriers
+  static constexpr uint32_t BAR = KV + WS_NBUF * 16384;       // mbarriers
   static constexpr int NBAR = 2 * WS_NBUF + 4 * 2 + 1;        // kv_full/empty, s/p/o x 2, drain
   static constexpr uint32_t MISC = BAR + NBAR * 8;            // TMEM base, abort flag
   static constexpr uint32_t TOTAL = MISC + 16;
@@ -663,7 +679,6 @@ __global__ void __launch_bounds__(WS_THREADS, 1) hca_flash_ws_kernel(FaParams p)
       // descriptors built once; a k-step moves the start address field (16-byte units)
       const uint64_t dq = make_sdesc(smem_u32(sm + WsOff::Q), 16, 1024, SMEM_SWIZZLE_128B);
       const uint64_t dk = make_sdesc(smem_u32(sm + WsOff::KV), 16, 1024, SMEM_SWIZZLE_128B);
-      const uint64_t dp = make_sdesc(smem_u32(sm + WsOff::P), 16, 1024, SMEM_SWIZZLE_128B);
       const uint64_t dv = make_sdesc(smem_u32(sm + WsOff::KV), 8192, 1024, SMEM_SWIZZLE_128B);
       constexpr uint32_t idS = idesc_bf16(128, FA_CH), idPV = idesc_bf16(128, FA_D) | (1u << 16);
       auto issue_s = [&](int tt, int rd) {
@@ -678,12 +693,11 @@ __global__ void __launch_bounds__(WS_THREADS, 1) hca_flash_ws_kernel(FaParams p)
         umma_commit(&s_full[tt]);
       };
       auto issue_pv = [&](int tt, int rd) {
-        const uint64_t a0 = dp + uint64_t(tt * (16384 >> 4));
         const uint64_t b0 = dv + uint64_t((rd % WS_NBUF) * (16384 >> 4));
 #pragma unroll
         for (int ks = 0; ks < 4; ks++)
-          umma_bf16(tbase + 2 * FA_CH + tt * FA_D, a0 + uint32_t(ks * 2), b0 + uint32_t(ks * (2048 >> 4)),
-                    idPV, (rd > 0 || ks > 0) ? 1u : 0u);
+          umma_bf16_ta(tbase + WS_OCOL + tt * FA_D, tbase + WS_PCOL + tt * 32 + ks * 8,
+                       b0 + uint32_t(ks * (2048 >> 4)), idPV, (rd > 0 || ks > 0) ? 1u : 0u);
         umma_commit(&o_done[tt]);
       };
       bool ok = mbar_wait(&kv_full[0], 0, p.limit, sAbort);
@@ -722,8 +736,8 @@ __global__ void __launch_bounds__(WS_THREADS, 1) hca_flash_ws_kernel(FaParams p)
     // ---------------- softmax of tile t: this thread's row ----------------
     const uint32_t lq = uint32_t((warp & 3) * 32) << 16;
     const uint32_t tS = tbase + lq + t * FA_CH;
-    const uint32_t tO = tbase + lq + 2 * FA_CH + t * FA_D;
-    uint8_t* prow = sm + WsOff::P + t * 16384 + row * 128;
+    const uint32_t tO = tbase + lq + WS_OCOL + t * FA_D;
+    const uint32_t tP = tbase + lq + WS_PCOL + t * 32;
     const float c2 = p.scale_log2;
     const unsigned long long c2x2 = f2_make(c2, c2);
     float m_run = -INFINITY, l_run = 0.f;
@@ -802,13 +816,12 @@ __global__ void __launch_bounds__(WS_THREADS, 1) hca_flash_ws_kernel(FaParams p)
         }
         tmem_st_wait();
       }
-#pragma unroll
-      for (int c = 0; c < 8; c++)
-        *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
-            make_uint4(sv[4 * c], sv[4 * c + 1], sv[4 * c + 2], sv[4 * c + 3]);
+      // P_t (bf16, two per column: the A operand of PV read from TMEM)
+      tmem_st16(tP, *reinterpret_cast<const uint32_t(*)[16]>(&sv[0]));
+      tmem_st16(tP + 16, *reinterpret_cast<const uint32_t(*)[16]>(&sv[16]));
       l_run = l_run * alpha + (f2_lo(lr) + f2_hi(lr));
       m_run = m_new;
-      fence_proxy_async_smem();
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
     }
