@@ -6,6 +6,9 @@
 // row is both key and value of the one shared KV head.  [Tripbot §3.1 step 2] CSA attends
 // over the query's own top-k entries plus the same window.
 //
+// HCA over bf16 rows runs on the warp-specialised two-tile kernel at the end of this file; the
+// kernel described next serves FP8 split rows and CSA prefill.
+//
 // Design (B200): one block of 256 threads per query group: G = floor(128 / H) consecutive
 // queries x H heads = up to 128 (query, head) rows = the UMMA M dimension = 128 TMEM lanes, two
 // threads per row.  The group's KV list is the visible-entry prefix of its last query followed
