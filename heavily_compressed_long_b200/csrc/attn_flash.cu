@@ -480,22 +480,23 @@ hcl_status_t launch_flash_t(const FaParams& p, cudaStream_t st) {
 //
 // Block = (sequence, pair of query groups): tile t in {0, 1} holds group 2 * pair + t (up to
 // 128 (query, head) rows each).  The pair's KV list is the visible-entry prefix of its last
-// query plus the union of its queries' windows, in rounds of 64 rows.  Warps 0..3 and 4..7
-// are the softmax warpgroups of tiles 0 and 1 (one thread per row, the row's 64 columns of a
-// round in registers, no exchange between threads); warps 8 and 9 gather the rounds' rows
-// with cp.async into a ring of three KV buffers (one row per thread); one thread of warp 11
-// issues every MMA from descriptors built once.  The MMA
-// issue order S_0(r+1), PV_0(r), S_1(r+1), PV_1(r) lets one tile's softmax run while the tensor
-// pipe works on the other tile, and each S_t(r+1) as soon as tile t's softmax has read S_t(r).
-// The softmax writes P (bf16) into TMEM and PV reads it from there as its A operand, so the
-// MMAs' shared-memory traffic is Q, K and V only (an N = 64 MMA with both operands in shared
-// memory is bound by shared-memory bandwidth, and P stores would compete with it).
-// TMEM: S_0, S_1 (64 columns each), O_0, O_1 (128 each), P_0, P_1 (32 each) -- one block per SM.
+// query plus the union of its queries' windows, in rounds of 128 rows.  Warps 0..3 and 4..7
+// are the softmax warpgroups of tiles 0 and 1 (one thread per row, no exchange between
+// threads); warps 8 and 9 gather the rounds' rows with cp.async into a ring of three KV
+// buffers (two rows per thread); one thread of warp 11 issues every MMA from descriptors built
+// once.  S = Q K^T is an N = 128 MMA (full tensor rate; at N = 64 with both operands in shared
+// memory it is bound by shared-memory bandwidth).  The softmax reads a round's 128 scores of
+// its row from TMEM twice (row maximum, then exponentials) and writes P (bf16) over the first
+// 64 columns of its S; PV reads P from TMEM as its A operand, so the MMAs' shared-memory
+// traffic is Q, K and V only.  Issue order per round: PV_0(r), S_0(r+1), PV_1(r), S_1(r+1);
+// S_t(r+1) waits until PV_t(r) has completed (it overwrites P_t), and while tile t's softmax
+// runs the tensor pipe works on the other tile.
+// TMEM: S_0 / P_0, S_1 / P_1 (128 columns each), O_0, O_1 (128 each) -- one block per SM.
 //
 //   kv_full[b]  (64 gather threads)   round rows landed in buffer b (copies done, proxy-fenced)
 //   kv_empty[b] (MMA commit)          both tiles' PV of the buffer's round completed
-//   s_full[t]   (MMA commit)          S_t of the round in TMEM
-//   s_free[t]   (128 softmax threads) S_t read into registers
+//   s_full[t]   (MMA commit)          S_t of the round in TMEM (and PV_t of the previous round
+//                                     completed: O_t stable)
 //   p_full[t]   (128 softmax threads) P_t in TMEM (and O_t rescaled)
 //   o_done[t]   (MMA commit)          PV_t of the round completed (P_t free, O_t stable)
 // Every wait is bounded; a timeout sets the block's abort flag and HCL_ERR_TIMEOUT.
@@ -516,13 +517,13 @@ constexpr int WS_WARPS = 12;
 constexpr int WS_GATHER = 64;   // warps 8, 9 (warp 10 idles: warps are allocated in fours)
 constexpr int WS_THREADS = WS_WARPS * 32;
 constexpr int WS_NBUF = 3;
-constexpr uint32_t WS_OCOL = 128;   // TMEM: S_0, S_1 at 0, 64; O_0, O_1 at 128, 256;
-constexpr uint32_t WS_PCOL = 384;   // P_0, P_1 (64 bf16 per row) at 384, 416
+constexpr int WS_CH = 128;          // list rows per round
+constexpr uint32_t WS_OCOL = 256;   // TMEM: S_0, S_1 at 0, 128; O_0, O_1 at 256, 384
 struct WsOff {
   static constexpr uint32_t Q = 0;                            // 2 tiles x 2 halves x 128 x 128 B
-  static constexpr uint32_t KV = 65536;                       // 3 x (2 halves x 64 rows x 128 B)
-  static constexpr uint32_t BAR = KV + WS_NBUF * 16384;       // mbarriers
-  static constexpr int NBAR = 2 * WS_NBUF + 4 * 2 + 1;        // kv_full/empty, s/p/o x 2, drain
+  static constexpr uint32_t KV = 65536;                       // 3 x (2 halves x 128 rows x 128 B)
+  static constexpr uint32_t BAR = KV + WS_NBUF * 32768;       // mbarriers
+  static constexpr int NBAR = 2 * WS_NBUF + 3 * 2 + 1;        // kv_full/empty, s/p/o x 2, drain
   static constexpr uint32_t MISC = BAR + NBAR * 8;            // TMEM base, abort flag
   static constexpr uint32_t TOTAL = MISC + 16;
 };
@@ -539,17 +540,15 @@ __global__ void __launch_bounds__(WS_THREADS, 1) hca_flash_ws_kernel(FaParams p)
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = bars + WS_NBUF;
   uint64_t* s_full = bars + 2 * WS_NBUF;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_full + 4;
-  uint64_t* o_done = s_full + 6;
-  uint64_t* drain = s_full + 8;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_done = s_full + 4;
+  uint64_t* drain = s_full + 6;
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + WsOff::MISC);
   volatile int* sAbort = reinterpret_cast<volatile int*>(sm + WsOff::MISC + 4);
   if (tid == 0) {
     for (int i = 0; i < WS_NBUF; i++) { mbar_init(&kv_full[i], WS_GATHER); mbar_init(&kv_empty[i], 1); }
     for (int t = 0; t < 2; t++) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&s_free[t], 128);
       mbar_init(&p_full[t], 128);
       mbar_init(&o_done[t], 1);
     }
@@ -576,7 +575,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) hca_flash_ws_kernel(FaParams p)
   const int raw_lo = pmin - p.W + 1;
   const int n_raw = (p.W > 0 && pmax >= 0) ? max(0, pmax - raw_lo + 1) : 0;
   const int total = n_a + n_raw;
-  const int nrounds = (total + FA_CH - 1) / FA_CH;
+  const int nrounds = (total + WS_CH - 1) / WS_CH;
 
   // softmax threads: this thread's tile, row, query and visibility intervals
   const int t = (tid >> 7) & 1, row = tid & 127;
@@ -636,7 +635,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) hca_flash_ws_kernel(FaParams p)
   const uint32_t tbase = *sTmem;
 
   if (warp == 8 || warp == 9) {
-    // ---------------- gather: one list row per thread, 16 16-byte pieces ----------------
+    // ---------------- gather: list rows jj and jj + 64 of each round, 16 pieces each ----------
     // a round is signalled as soon as its own copies have landed, so the MMA warp never waits
     // for the gather of a later round
     const int jj = tid - 256;
@@ -647,28 +646,31 @@ __global__ void __launch_bounds__(WS_THREADS, 1) hca_flash_ws_kernel(FaParams p)
         report(p.status, HCL_ERR_TIMEOUT);
         break;
       }
-      const int e = rd * FA_CH + jj;
-      long long slot = -1;
-      bool from_raw = false;
-      if (e < total) {
-        if (e < n_a) {
-          slot = (long long)b * p.comp.cap + (e < p.comp.cap ? e : e % p.comp.cap);
-        } else {
-          const int tok = raw_lo + (e - n_a);
-          if (tok >= 0) {
-            slot = (long long)b * p.raw.cap + (tok < p.raw.cap ? tok : tok % p.raw.cap);
-            from_raw = true;
+#pragma unroll
+      for (int hr = 0; hr < 2; hr++) {
+        const int rr = jj + 64 * hr, e = rd * WS_CH + rr;
+        long long slot = -1;
+        bool from_raw = false;
+        if (e < total) {
+          if (e < n_a) {
+            slot = (long long)b * p.comp.cap + (e < p.comp.cap ? e : e % p.comp.cap);
+          } else {
+            const int tok = raw_lo + (e - n_a);
+            if (tok >= 0) {
+              slot = (long long)b * p.raw.cap + (tok < p.raw.cap ? tok : tok % p.raw.cap);
+              from_raw = true;
+            }
           }
         }
-      }
-      const uint8_t* srow = static_cast<const uint8_t*>(from_raw ? p.raw.data : p.comp.data) +
-                            (slot < 0 ? 0 : slot) * 256;
-      uint8_t* dst = sm + WsOff::KV + buf * 16384 + jj * 128;
+        const uint8_t* srow = static_cast<const uint8_t*>(from_raw ? p.raw.data : p.comp.data) +
+                              (slot < 0 ? 0 : slot) * 256;
+        uint8_t* dst = sm + WsOff::KV + buf * 32768 + rr * 128;
 #pragma unroll
-      for (int i = 0; i < 16; i++) {
-        uint8_t* d = dst + (i >> 3) * 8192 + (((i & 7) ^ (jj & 7)) << 4);
-        if (slot >= 0) cp_async16(d, srow + i * 16);
-        else *reinterpret_cast<uint4*>(d) = make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < 16; i++) {
+          uint8_t* d = dst + (i >> 3) * 16384 + (((i & 7) ^ (rr & 7)) << 4);
+          if (slot >= 0) cp_async16(d, srow + i * 16);
+          else *reinterpret_cast<uint4*>(d) = make_uint4(0, 0, 0, 0);
+        }
       }
       cp_async_commit();
       cp_async_wait<0>();
@@ -682,24 +684,24 @@ __global__ void __launch_bounds__(WS_THREADS, 1) hca_flash_ws_kernel(FaParams p)
       // descriptors built once; a k-step moves the start address field (16-byte units)
       const uint64_t dq = make_sdesc(smem_u32(sm + WsOff::Q), 16, 1024, SMEM_SWIZZLE_128B);
       const uint64_t dk = make_sdesc(smem_u32(sm + WsOff::KV), 16, 1024, SMEM_SWIZZLE_128B);
-      const uint64_t dv = make_sdesc(smem_u32(sm + WsOff::KV), 8192, 1024, SMEM_SWIZZLE_128B);
-      constexpr uint32_t idS = idesc_bf16(128, FA_CH), idPV = idesc_bf16(128, FA_D) | (1u << 16);
+      const uint64_t dv = make_sdesc(smem_u32(sm + WsOff::KV), 16384, 1024, SMEM_SWIZZLE_128B);
+      constexpr uint32_t idS = idesc_bf16(128, WS_CH), idPV = idesc_bf16(128, FA_D) | (1u << 16);
       auto issue_s = [&](int tt, int rd) {
         const uint64_t a0 = dq + uint64_t(tt * (32768 >> 4));
-        const uint64_t b0 = dk + uint64_t((rd % WS_NBUF) * (16384 >> 4));
+        const uint64_t b0 = dk + uint64_t((rd % WS_NBUF) * (32768 >> 4));
 #pragma unroll
         for (int ks = 0; ks < 8; ks++) {
           const uint32_t off_a = (ks >> 2) * (16384 >> 4) + (ks & 3) * 2;
-          const uint32_t off_b = (ks >> 2) * (8192 >> 4) + (ks & 3) * 2;
-          umma_bf16(tbase + tt * FA_CH, a0 + off_a, b0 + off_b, idS, ks > 0 ? 1u : 0u);
+          const uint32_t off_b = (ks >> 2) * (16384 >> 4) + (ks & 3) * 2;
+          umma_bf16(tbase + tt * WS_CH, a0 + off_a, b0 + off_b, idS, ks > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[tt]);
       };
       auto issue_pv = [&](int tt, int rd) {
-        const uint64_t b0 = dv + uint64_t((rd % WS_NBUF) * (16384 >> 4));
+        const uint64_t b0 = dv + uint64_t((rd % WS_NBUF) * (32768 >> 4));
 #pragma unroll
-        for (int ks = 0; ks < 4; ks++)
-          umma_bf16_ta(tbase + WS_OCOL + tt * FA_D, tbase + WS_PCOL + tt * 32 + ks * 8,
+        for (int ks = 0; ks < 8; ks++)
+          umma_bf16_ta(tbase + WS_OCOL + tt * FA_D, tbase + tt * WS_CH + ks * 8,
                        b0 + uint32_t(ks * (2048 >> 4)), idPV, (rd > 0 || ks > 0) ? 1u : 0u);
         umma_commit(&o_done[tt]);
       };
@@ -711,19 +713,19 @@ __global__ void __launch_bounds__(WS_THREADS, 1) hca_flash_ws_kernel(FaParams p)
       }
       for (int rd = 0; ok && rd < nrounds; rd++) {
         for (int tt = 0; tt < 2 && ok; tt++) {
-          if (rd + 1 < nrounds) {
-            const int nb = (rd + 1) % WS_NBUF;
-            if (tt == 0) ok = mbar_wait(&kv_full[nb], ((rd + 1) / WS_NBUF) & 1, p.limit, sAbort);
-            ok = ok && mbar_wait(&s_free[tt], rd & 1, p.limit, sAbort);
-            if (!ok) break;
-            tc_fence_after();
-            issue_s(tt, rd + 1);
-          }
           ok = mbar_wait(&p_full[tt], rd & 1, p.limit, sAbort);
           if (!ok) break;
           tc_fence_after();
           issue_pv(tt, rd);
           if (tt == 1) umma_commit(&kv_empty[rd % WS_NBUF]);
+          if (rd + 1 < nrounds) {
+            // S_t(r + 1) overwrites P_t: PV_t(r) must have completed
+            if (tt == 0) ok = mbar_wait(&kv_full[(rd + 1) % WS_NBUF], ((rd + 1) / WS_NBUF) & 1, p.limit, sAbort);
+            ok = ok && mbar_wait(&o_done[tt], rd & 1, p.limit, sAbort);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(tt, rd + 1);
+          }
         }
       }
       if (!ok) {
@@ -738,46 +740,46 @@ __global__ void __launch_bounds__(WS_THREADS, 1) hca_flash_ws_kernel(FaParams p)
   } else if (warp < 8) {
     // ---------------- softmax of tile t: this thread's row ----------------
     const uint32_t lq = uint32_t((warp & 3) * 32) << 16;
-    const uint32_t tS = tbase + lq + t * FA_CH;
+    const uint32_t tS = tbase + lq + t * WS_CH;            // S_t; P_t over its first 64 columns
     const uint32_t tO = tbase + lq + WS_OCOL + t * FA_D;
-    const uint32_t tP = tbase + lq + WS_PCOL + t * 32;
     const float c2 = p.scale_log2;
     const unsigned long long c2x2 = f2_make(c2, c2);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int rd = 0; rd < nrounds; rd++) {
-      const int r0 = rd * FA_CH;
+      const int r0 = rd * WS_CH;
       ok = mbar_wait(&s_full[t], rd & 1, p.limit, sAbort);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sv[64];
-      tmem_ld16(tS, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
-      tmem_ld16(tS + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
-      tmem_ld16(tS + 32, *reinterpret_cast<uint32_t(*)[16]>(&sv[32]));
-      tmem_ld16(tS + 48, *reinterpret_cast<uint32_t(*)[16]>(&sv[48]));
-      uint32_t vb[2] = {0u, 0u};
+      uint32_t vb[4] = {0u, 0u, 0u, 0u};
       if (rv) {
 #pragma unroll
-        for (int w = 0; w < 2; w++) {
+        for (int w = 0; w < 4; w++) {
           const int c0 = r0 + 32 * w;
           vb[w] = range_bits(c0, 0, nv_e) | range_bits(c0, w_lo, w_hi);
         }
       }
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&s_free[t]);
       // row maximum of the raw scores over the valid columns (scale > 0)
+      uint32_t sv[64];
       float smax = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < 2; w++) {
-        if (vb[w] == 0xFFFFFFFFu) {
+      for (int hf = 0; hf < 2; hf++) {
 #pragma unroll
-          for (int j = 0; j < 32; j += 2)
-            smax = fmax3(smax, __uint_as_float(sv[32 * w + j]), __uint_as_float(sv[32 * w + j + 1]));
-        } else if (vb[w] != 0u) {
+        for (int k = 0; k < 4; k++)
+          tmem_ld16(tS + hf * 64 + 16 * k, *reinterpret_cast<uint32_t(*)[16]>(&sv[16 * k]));
+        tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; j++)
-            if ((vb[w] >> j) & 1u) smax = fmaxf(smax, __uint_as_float(sv[32 * w + j]));
+        for (int w = 0; w < 2; w++) {
+          const uint32_t bits = vb[2 * hf + w];
+          if (bits == 0xFFFFFFFFu) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 2)
+              smax = fmax3(smax, __uint_as_float(sv[32 * w + j]), __uint_as_float(sv[32 * w + j + 1]));
+          } else if (bits != 0u) {
+#pragma unroll
+            for (int j = 0; j < 32; j++)
+              if ((bits >> j) & 1u) smax = fmaxf(smax, __uint_as_float(sv[32 * w + j]));
+          }
         }
       }
       const float m_cand = fmaxf(m_run, smax == -INFINITY ? -INFINITY : smax * c2);
@@ -786,27 +788,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) hca_flash_ws_kernel(FaParams p)
       const float alpha = (grow && m_run > -INFINITY) ? ex2_ftz(m_run - m_new) : 1.f;
       const float muse = m_new == -INFINITY ? 0.f : m_new;
       const unsigned long long negm = f2_make(-muse, -muse);
-      // the packed bf16 pair of columns j, j + 1 goes to sv[j / 2] (already consumed)
-      unsigned long long lr = 0ull;
-#pragma unroll
-      for (int j = 0; j < 64; j += 2) {
-        const unsigned long long x =
-            f2_fma(f2_make(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), c2x2, negm);
-        float p0 = ex2_ftz(f2_lo(x)), p1 = ex2_ftz(f2_hi(x));
-        const uint32_t bits = vb[j >> 5];
-        if (bits != 0xFFFFFFFFu) {
-          p0 = ((bits >> (j & 31)) & 1u) ? p0 : 0.f;
-          p1 = ((bits >> ((j + 1) & 31)) & 1u) ? p1 : 0.f;
-        }
-        lr = f2_add(lr, f2_make(p0, p1));
-        sv[j >> 1] = fa_pack(p0, p1);
-      }
-      // P_t and O_t belong to the previous round's PV until it completes
-      if (rd > 0) {
-        ok = mbar_wait(&o_done[t], (rd - 1) & 1, p.limit, sAbort);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        tc_fence_after();
-      }
+      // O_t is stable: s_full of this round came after PV_t of the previous one completed
       if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
         for (int q8 = 0; q8 < 8; q8++) {
@@ -817,11 +799,32 @@ __global__ void __launch_bounds__(WS_THREADS, 1) hca_flash_ws_kernel(FaParams p)
           for (int i = 0; i < 16; i++) r16[i] = __float_as_uint(__uint_as_float(r16[i]) * alpha);
           tmem_st16(tO + q8 * 16, r16);
         }
-        tmem_st_wait();
       }
-      // P_t (bf16, two per column: the A operand of PV read from TMEM)
-      tmem_st16(tP, *reinterpret_cast<const uint32_t(*)[16]>(&sv[0]));
-      tmem_st16(tP + 16, *reinterpret_cast<const uint32_t(*)[16]>(&sv[16]));
+      // probabilities, 32 columns at a time: P of columns 32c .. 32c + 31 (16 TMEM columns of
+      // bf16 pairs) goes over S columns 16c .. 16c + 15, whose scores this thread has already
+      // used (its own lane; later loads read columns >= 32 (c + 1))
+      unsigned long long lr = 0ull;
+#pragma unroll
+      for (int c = 0; c < 4; c++) {
+        tmem_ld16(tS + 32 * c, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
+        tmem_ld16(tS + 32 * c + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+        tmem_ld_wait();
+        const uint32_t bits = vb[c];
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const unsigned long long x =
+              f2_fma(f2_make(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), c2x2, negm);
+          float p0 = ex2_ftz(f2_lo(x)), p1 = ex2_ftz(f2_hi(x));
+          if (bits != 0xFFFFFFFFu) {
+            p0 = ((bits >> j) & 1u) ? p0 : 0.f;
+            p1 = ((bits >> (j + 1)) & 1u) ? p1 : 0.f;
+          }
+          lr = f2_add(lr, f2_make(p0, p1));
+          pk[j >> 1] = fa_pack(p0, p1);
+        }
+        tmem_st16(tS + 16 * c, pk);
+      }
       l_run = l_run * alpha + (f2_lo(lr) + f2_hi(lr));
       m_run = m_new;
       tmem_st_wait();
