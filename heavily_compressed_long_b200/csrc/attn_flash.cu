@@ -800,30 +800,32 @@ __global__ void __launch_bounds__(WS_THREADS, 1) hca_flash_ws_kernel(FaParams p)
           tmem_st16(tO + q8 * 16, r16);
         }
       }
-      // probabilities, 32 columns at a time: P of columns 32c .. 32c + 31 (16 TMEM columns of
-      // bf16 pairs) goes over S columns 16c .. 16c + 15, whose scores this thread has already
-      // used (its own lane; later loads read columns >= 32 (c + 1))
+      // probabilities, 64 columns per TMEM wait: P of columns 64c .. 64c + 63 (32 TMEM columns
+      // of bf16 pairs) goes over S columns 32c .. 32c + 31, whose scores this thread has
+      // already used (its own lane; the next load reads columns 64 .. 127)
       unsigned long long lr = 0ull;
 #pragma unroll
-      for (int c = 0; c < 4; c++) {
-        tmem_ld16(tS + 32 * c, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
-        tmem_ld16(tS + 32 * c + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
-        tmem_ld_wait();
-        const uint32_t bits = vb[c];
-        uint32_t pk[16];
+      for (int c = 0; c < 2; c++) {
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
+        for (int k = 0; k < 4; k++)
+          tmem_ld16(tS + 64 * c + 16 * k, *reinterpret_cast<uint32_t(*)[16]>(&sv[16 * k]));
+        tmem_ld_wait();
+        uint32_t pk[32];
+#pragma unroll
+        for (int j = 0; j < 64; j += 2) {
+          const uint32_t bits = vb[2 * c + (j >> 5)];
           const unsigned long long x =
               f2_fma(f2_make(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), c2x2, negm);
           float p0 = ex2_ftz(f2_lo(x)), p1 = ex2_ftz(f2_hi(x));
           if (bits != 0xFFFFFFFFu) {
-            p0 = ((bits >> j) & 1u) ? p0 : 0.f;
-            p1 = ((bits >> (j + 1)) & 1u) ? p1 : 0.f;
+            p0 = ((bits >> (j & 31)) & 1u) ? p0 : 0.f;
+            p1 = ((bits >> ((j + 1) & 31)) & 1u) ? p1 : 0.f;
           }
           lr = f2_add(lr, f2_make(p0, p1));
           pk[j >> 1] = fa_pack(p0, p1);
         }
-        tmem_st16(tS + 16 * c, pk);
+        tmem_st16(tS + 32 * c, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
+        tmem_st16(tS + 32 * c + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
       }
       l_run = l_run * alpha + (f2_lo(lr) + f2_hi(lr));
       m_run = m_new;
