@@ -209,6 +209,16 @@ def test_cfg4_csa_1m_mxfp4_fp8(hcl):
         assert torch.equal(idx1, pipe.idx)
         assert torch.equal(out1, pipe.out) and torch.equal(lse1, pipe.lse)
     assert pipe.status.item() == 0
+    # a wait that ran to its bounded limit (about a second) would show here even if its result
+    # were not reported: 20 steps take about 1 ms, the bound is generous
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(20):
+        pipe.step()
+    e1.record()
+    torch.cuda.synchronize()
+    assert e0.elapsed_time(e1) / 20 < 5.0
+    assert pipe.status.item() == 0
     for b in range(B):
         sl = slice(b, b + 1)
         cn, cs, cr = oracle.quant_kv_fp8(gen.comp_kv(cfg, [b], Nc))
